@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""Benchmark of the Medusa decode-verify step on B200.
+
+One step = heads + top-k, tree build, tree attention, verify/accept and KV
+compaction for one batch (the five C-ABI calls).  Default workload: the
+Llama-3-8B-shaped configuration (batch 8, hidden 4096, vocab 128256, 4 heads,
+64-node sparse tree, GQA 32/8 heads of 128, ragged prefixes 4096..8192, bf16,
+greedy acceptance).  Inputs are seeded synthetic data of those shapes; every
+step touches ~4.7 GB (larger than the 126 MB L2), so no flush is needed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own batch (sequences are independent; no
+collective on the data path): weak scaling, value = all ranks' steps / the
+slowest rank's time.  `--impl reference` times the CPU oracle (the only
+reference implementation) on a bounded sample, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "Medusa decode-verify steps/s (heads+tree attn+accept); % of HBM roofline"
+UNIT = "steps/s"
+KERNELS_PER_STEP = 9  # W1 GEMM, W2 GEMM, top-k merge, tree build, attention, combine,
+#                       verify rows, verify path, KV compaction
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def algorithmic_bytes(w, prefix_lens, N):
+    """Bytes the step must move at minimum (bf16 = 2 B)."""
+    e = 2 if w.dtype == "bf16" else 4
+    heads = w.K * (w.d * w.d + w.d + w.V * w.d) * e + w.B * w.d * e
+    kv_prefix = sum(int(p) for p in prefix_lens) * w.Hkv * w.dh * 2 * e
+    tree_qkv = w.B * N * (w.Hq + 2 * w.Hkv) * w.dh * e
+    tree_out = w.B * N * w.Hq * w.dh * e
+    tree_kv_write = w.B * N * w.Hkv * w.dh * 2 * e
+    logits = w.B * N * w.V * e
+    return {"heads": heads, "attention": kv_prefix + tree_qkv + tree_out + tree_kv_write,
+            "verify": logits, "total": heads + kv_prefix + tree_qkv + tree_out + tree_kv_write + logits}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.lines = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", gpu_index], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _gpu_index(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample
+# ---------------------------------------------------------------------------
+def oracle_sample(w, n_nodes=None, seed=0):
+    """Time the CPU oracle on a bounded sample of one step and extrapolate to a
+    whole step.  Sample: head 0 on a 16384-token slice of its vocabulary for
+    every sequence (scaled by K * V / 16384); tree attention of 4 (sequence,
+    node) query rows with all heads (scaled by B*N/4); verification statistics
+    of 8 rows (scaled by B*N/8); tree build and KV compaction in full."""
+    from oracle import medusa_oracle as O
+    from speculative_decoding_medusa_b200 import workloads as W
+
+    N = n_nodes or w.N
+    spec = W.tree_for(w, n_nodes=N)
+    f64 = lambda t: t.to(torch.float64).numpy()
+    rows_v = min(16384, w.V)
+    h = f64(W.randn((w.B, w.d), seed, 1, 1.0, w.dtype))
+    W1 = f64(W.randn((1, w.d, w.d), seed, 2, 0.02, w.dtype))
+    b1 = f64(W.randn((1, w.d), seed, 3, 0.02, w.dtype))
+    W2 = f64(W.randn((1, rows_v, w.d), seed, 4, 0.02, w.dtype))
+    P = W.prefix_lengths(w, seed).numpy().astype(np.int64)
+    cap = w.ctx_hi + N
+    b0 = int(np.argmax(P))
+    q = f64(W.randn((1, N, w.Hq, w.dh), seed, 11, 1.0, w.dtype))
+    kn = f64(W.randn((1, N, w.Hkv, w.dh), seed, 12, 1.0, w.dtype))
+    vn = f64(W.randn((1, N, w.Hkv, w.dh), seed, 13, 1.0, w.dtype))
+    Kc = f64(W.randn((1, w.Hkv, cap, w.dh), seed, 14, 1.0, w.dtype))
+    Vc = f64(W.randn((1, w.Hkv, cap, w.dh), seed, 15, 1.0, w.dtype))
+    logits = f64(W.randn((1, 9, w.V), seed, 21, 1.0, w.dtype))
+
+    t = {}
+    t0 = time.perf_counter()
+    z = O.head_logits(h, W1, b1, W2)
+    O.topk(z, w.kmax)
+    t["heads"] = (time.perf_counter() - t0) * w.K * (w.V / rows_v)
+    t0 = time.perf_counter()
+    ids = np.zeros((w.B, w.K, w.kmax), dtype=np.int64)
+    tb = O.tree_build(spec.parent, spec.depth, spec.rank, np.zeros(w.B, np.int64), ids, P)
+    t["tree_build"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    # 4 query nodes (all heads) of the longest sequence: the oracle over a
+    # 4-node chain (root + 3 descendants) of that sequence
+    chain = [0]
+    while len(chain) < 4 and any(spec.parent[c] == chain[-1] for c in range(1, N)):
+        chain.append(next(c for c in range(1, N) if spec.parent[c] == chain[-1]))
+    mm = np.zeros((len(chain), 1), dtype=np.uint32)
+    for r in range(len(chain)):
+        mm[r, 0] = (1 << (r + 1)) - 1
+    O.tree_attention(q[:, chain], kn[:, chain], vn[:, chain], Kc, Vc, P[b0:b0 + 1], mm,
+                     1.0 / math.sqrt(w.dh))
+    t["attention"] = (time.perf_counter() - t0) * w.B * N / len(chain) * \
+        (float(np.mean(P)) + N / 2) / (float(P[b0]) + len(chain) / 2)
+    t0 = time.perf_counter()
+    O.row_argmax(logits[:, :8])
+    if w.accept == "typical":  # a 9-node chain: statistics of its first 8 rows
+        O.typical_log_margin(logits, np.zeros((1, 9), np.int64), np.arange(-1, 8),
+                             w.temperature, w.eps, w.delta)
+    t["verify"] = (time.perf_counter() - t0) * w.B * N / 8
+    t0 = time.perf_counter()
+    nodes = np.full((1, spec.max_depth + 1), -1, dtype=np.int64)
+    nodes[0, 0] = 0
+    O.kv_compact(Kc, Vc, P[b0:b0 + 1], nodes, np.array([0]))
+    t["kv_compact"] = (time.perf_counter() - t0) * w.B
+    sec = sum(t.values())
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    sample = (f"head 0 on {rows_v} of {w.V} vocab rows x {w.B} sequences (x{w.K * w.V / rows_v:.1f}); "
+              f"{len(chain)} query nodes x {w.Hq} heads of one sequence (x{w.B * N / len(chain):.0f}, "
+              f"scaled by mean prefix); verify stats of 8 rows (x{w.B * N / 8:.0f}); tree build and "
+              f"compaction in full; fp64 numpy")
+    return {"seconds_per_step": sec, "stages": t, "cores": int(cores), "sample": sample}
+
+
+# ---------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama3_8b")
+    ap.add_argument("--nodes", type=int, default=None, help="tree size override (long: 16/64/128)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    return ap.parse_args()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from speculative_decoding_medusa_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    N = args.nodes or w.N
+    times = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(w, N, seed=i)
+        if i >= args.warmup:
+            times.append(r["seconds_per_step"])
+        if sum(times) > 120:  # keep the whole run within a few minutes
+            break
+    sec = statistics.mean(times)
+    value = 1.0 / sec
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
+            "n_gpus": args.gpus, "steps": len(times), "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "global_batch": w.B, "n_nodes": N,
+                       "prefix": [w.ctx_lo, w.ctx_hi], "parallelism": "none (CPU oracle)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import speculative_decoding_medusa_b200 as M
+    from speculative_decoding_medusa_b200 import workloads as W
+    from speculative_decoding_medusa_b200.step import DecodeVerifyStep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    M.lib()  # fails loudly when the library is missing
+
+    w = W.WORKLOADS[args.workload]
+    N = args.nodes or w.N
+    if args.nodes:
+        w = W.scaled(w, N=N)
+    spec = W.tree_for(w, n_nodes=N)
+    seed = rank
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    # weights and caches drawn on the device (seeded); parity is tested elsewhere
+    hin = W.heads_inputs(w, seed=seed, device=dev)
+    att = W.attention_inputs(w, seed=seed, device=dev, n_nodes=N)
+    root = W.random_root_tokens(w, seed, device=dev)
+    tree = M.Tree.from_spec(spec, dev)
+    step = DecodeVerifyStep(B=w.B, d=w.d, V=w.V, K=w.K, kmax=w.kmax, tree=tree, Hq=w.Hq, Hkv=w.Hkv,
+                            dh=w.dh, cap=w.cap, max_prefix=w.ctx_hi, dtype=dt, accept=w.accept,
+                            temperature=w.temperature, eps=w.eps, delta=w.delta, device=dev)
+    # candidates of this batch -> verify logits that agree with some of them
+    M.medusa_heads_topk(hin["h"], hin["W1"], hin["b1"], hin["W2"], w.kmax, step.topk_ids,
+                        step.topk_vals, None, step.ws_heads, step.status)
+    M.medusa_tree_build(tree, root, step.topk_ids, att["prefix_len"], step.cand_ids, step.pos_ids,
+                        step.anc_mask, step.retrieve, step.status)
+    torch.cuda.synchronize()
+    logits = W.verify_logits(w, spec, step.cand_ids, seed=seed, device=dev)
+    prefix0 = att["prefix_len"].clone()
+    prefix_list = prefix0.tolist()
+    stream = torch.cuda.current_stream()
+
+    def one_step(evs=None):
+        att["prefix_len"].copy_(prefix0)  # same prefixes every step
+        if evs is None:
+            step.run(hin["h"], hin["W1"], hin["b1"], hin["W2"], root, att["q"], att["k_new"],
+                     att["v_new"], att["Kc"], att["Vc"], att["prefix_len"], logits)
+            return
+        evs[0].record(stream)
+        M.medusa_heads_topk(hin["h"], hin["W1"], hin["b1"], hin["W2"], w.kmax, step.topk_ids,
+                            step.topk_vals, None, step.ws_heads, step.status)
+        evs[1].record(stream)
+        M.medusa_tree_build(tree, root, step.topk_ids, att["prefix_len"], step.cand_ids,
+                            step.pos_ids, step.anc_mask, step.retrieve, step.status)
+        evs[2].record(stream)
+        M.medusa_tree_attention(att["q"], att["k_new"], att["v_new"], att["Kc"], att["Vc"],
+                                att["prefix_len"], step.anc_mask, w.ctx_hi, step.attn_out, None,
+                                step.ws_attn, step.status)
+        evs[3].record(stream)
+        M.medusa_verify_accept(logits, step.cand_ids, tree, step.accept_len, step.accepted_nodes,
+                               step.accepted_tokens, step.bonus, step.mode, w.temperature, w.eps,
+                               w.delta, step.ws_verify, step.status)
+        evs[4].record(stream)
+        M.medusa_kv_compact(att["Kc"], att["Vc"], att["prefix_len"], step.accepted_nodes,
+                            step.accept_len, step.compact_src, step.status)
+        evs[5].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        one_step()
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0, f"device status {int(step.status.item())}"
+
+    sampler = ClockSampler(_gpu_index(local_rank))
+    time.sleep(0.2)
+    # ---- timed region: K steps, stage events recorded between the calls ----
+    stage_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        one_step(stage_evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    names = ["heads_topk", "tree_build", "tree_attention", "verify_accept", "kv_compact"]
+    stages = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in stage_evs) * 1e3
+              for i, n in enumerate(names)}  # us
+    assert int(step.status.item()) == 0
+
+    # ---- end to end through the public API with host buffers ----
+    host_in = {k: v.cpu().pin_memory() for k, v in
+               {"h": hin["h"], "root": root, "q": att["q"], "k_new": att["k_new"],
+                "v_new": att["v_new"], "logits": logits, "prefix_len": prefix0}.items()}
+    dev_in = {"h": hin["h"], "root": root, "q": att["q"], "k_new": att["k_new"],
+              "v_new": att["v_new"], "logits": logits, "prefix_len": att["prefix_len"]}
+    host_out = {k: torch.empty_like(getattr(step, k), device="cpu").pin_memory()
+                for k in ("accept_len", "accepted_tokens", "bonus", "compact_src")}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def e2e_step():
+        for k, t in host_in.items():
+            dev_in[k].copy_(t, non_blocking=True)
+        step.run(dev_in["h"], hin["W1"], hin["b1"], hin["W2"], dev_in["root"], dev_in["q"],
+                 dev_in["k_new"], dev_in["v_new"], att["Kc"], att["Vc"], dev_in["prefix_len"],
+                 dev_in["logits"])
+        for k, t in host_out.items():
+            t.copy_(getattr(step, k), non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    n_e2e = max(1, args.e2e_steps)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms_e2e = float(tt.item())
+    e2e_value = world * n_e2e / (ms_e2e / 1e3)
+
+    # ---- roofline of the dominant call (heads_topk: W1 + W2 weight stream) ----
+    hbm_peak, _, peak_kind = _peaks()
+    ab = algorithmic_bytes(w, prefix_list, N)
+    heads_gbs = ab["heads"] / (stages["heads_topk"] * 1e-6) / 1e9
+    step_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
+    value = world * args.steps / (ms_total / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = oracle_sample(w, N)
+        cpu = {"value": 1.0 / r["seconds_per_step"], "unit": UNIT, "cores": r["cores"],
+               "kind": "oracle", "sample": r["sample"]}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
+            "data": "synthetic (seeded, on-device draws of the workload's shapes; random weights)",
+            "config": {"workload": args.workload, "global_batch": w.B * world, "batch_per_gpu": w.B,
+                       "hidden": w.d, "vocab": w.V, "heads": w.K, "kmax": w.kmax, "n_nodes": N,
+                       "attn_heads": [w.Hq, w.Hkv, w.dh], "prefix": [w.ctx_lo, w.ctx_hi],
+                       "accept": w.accept, "parallelism": f"dp{world} (independent batches)",
+                       "l2": "no flush: each step streams ~%.2f GB (> 126 MB L2)" % (ab["total"] / 1e9)},
+            "hbm_roofline_frac_step": step_gbs / hbm_peak,
+            "step_bytes": ab["total"],
+            "stages_us": stages,
+            "roofline": {"bound": "hbm", "kernel": "medusa_heads_topk (W1 GEMM + W2 GEMM + top-k merge)",
+                         "achieved": heads_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": heads_gbs / hbm_peak, "traffic": None,
+                         "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": ab["heads"]},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": n_e2e},
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "clocks": clocks,
+            "mean_accept_len": float(step.accept_len.float().mean().item()),
+        }
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,293 @@
+/*
+ * medusa.h - C ABI of the Medusa decode-verify step on NVIDIA B200 (sm_100a).
+ *
+ * One decode-verify step of Medusa speculative decoding, in five calls:
+ *
+ *   medusa_heads_topk      K Medusa heads on the last hidden state, then a
+ *                          top-k over the vocabulary per head;
+ *   medusa_tree_build      candidate tree from those top-k lists: candidate
+ *                          ids, position ids, ancestor mask, retrieve paths;
+ *   medusa_tree_attention  attention of every tree node over the cached
+ *                          prefix and its own ancestors;
+ *   medusa_verify_accept   the longest branch the base model agrees with
+ *                          (greedy match or typical acceptance);
+ *   medusa_kv_compact      the kept branch's K/V moved into contiguous slots.
+ *
+ * Sources (page title, then section):
+ *   "Medusa Heads" glossary - "Comment les têtes prédisent les tokens
+ *     suivants" (the head) and "Attention arborescente et acceptation" (tree,
+ *     tree mask, greedy and typical acceptance, longest kept branch);
+ *   "Medusa Decoding Heads" overview - "Diepe duik" (one-pass verification of
+ *     the whole tree, losslessness);
+ *   "Medusa no contexto de LLMs" - "o que significa medusa na prática de
+ *     deploy" (accepted tokens enter the sequence without another pass; the
+ *     conventionally generated token on rejection);
+ *   "Medusa: Simple LLM Inference Acceleration Framework with Multiple
+ *     Decoding Heads" - abstract (tree-based attention over candidate
+ *     continuations, one decoding step).
+ *
+ * Conventions for every call
+ *   - Pointers named as device pointers must point to memory of the current
+ *     CUDA device; host pointers are read before the call returns.  The
+ *     caller owns every buffer.  The library never allocates device memory
+ *     and never synchronises: all work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *   - All arrays are dense, row-major, with the layouts given per call.
+ *     bf16 arrays are IEEE bfloat16 bit patterns (uint16).
+ *   - Errors the host can see (null pointer, unsupported size, misaligned
+ *     pointer, workspace too small) are returned before anything is launched.
+ *     MEDUSA_ERR_CUDA reports a failed launch; medusa_last_error() then holds
+ *     the CUDA error text.
+ *   - Errors only the device can see (an index out of range in a tree or an
+ *     accepted path, a NaN logit, a bounded wait that ran out) are written
+ *     into *dev_status (device int32, 0 = OK) with an atomic compare-and-swap,
+ *     so the first error sticks.  The caller zeroes it once and reads it after
+ *     its own synchronisation.  No kernel traps; outputs of a call that set a
+ *     device error are unspecified but every write stays inside its buffer.
+ *   - The library is re-entrant.  Calls on the same stream run in order; the
+ *     caller orders calls on different streams.
+ */
+#ifndef MEDUSA_B200_H
+#define MEDUSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MEDUSA_API __attribute__((visibility("default")))
+#else
+#define MEDUSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MEDUSA_OK = 0,
+  MEDUSA_ERR_INVALID_ARG = 1,  /* null pointer, bad enum, negative size      */
+  MEDUSA_ERR_SHAPE = 2,        /* sizes outside the supported limits          */
+  MEDUSA_ERR_UNSUPPORTED = 3,  /* valid request this build does not handle    */
+  MEDUSA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed           */
+  MEDUSA_ERR_TIMEOUT = 5,      /* device: a bounded wait ran out              */
+  MEDUSA_ERR_DEVICE_CHECK = 6, /* device: index out of range, NaN input       */
+  MEDUSA_ERR_WORKSPACE = 7,    /* workspace pointer null or too small         */
+  MEDUSA_ERR_ALIGNMENT = 8     /* pointer not aligned as the call requires    */
+} medusa_status_t;
+
+typedef enum { MEDUSA_BF16 = 0, MEDUSA_F32 = 1 } medusa_dtype_t;
+typedef enum { MEDUSA_ACCEPT_GREEDY = 0, MEDUSA_ACCEPT_TYPICAL = 1 } medusa_accept_t;
+
+/* Limits of this build. */
+#define MEDUSA_MAX_NODES 256   /* tree nodes, root included                  */
+#define MEDUSA_MAX_KMAX 32     /* top-k width per head                       */
+#define MEDUSA_MAX_HEADS 16    /* Medusa heads = deepest possible tree level */
+#define MEDUSA_MAX_BATCH 128   /* sequences per call (bf16 heads)            */
+
+/*
+ * A candidate tree.  Nodes are in breadth-first order (parents before
+ * children); node 0 is the root.  The struct lives in host memory; the three
+ * arrays are DEVICE arrays of n_nodes int32 each:
+ *   parent[i]  parent node (parent[0] = -1, 0 <= parent[i] < i otherwise);
+ *   depth[i]   depth (depth[0] = 0, depth[i] = depth[parent[i]] + 1);
+ *   rank[i]    for i > 0, which entry of head depth[i]'s top-k list the node
+ *              carries (0 <= rank[i] < kmax).
+ * max_depth is the largest depth[i]; n_leaves the number of nodes without a
+ * child.  Kernels check these relations and report violations through
+ * dev_status.
+ */
+typedef struct medusa_tree {
+  int32_t n_nodes;
+  int32_t max_depth;
+  int32_t n_leaves;
+  const int32_t* parent;
+  const int32_t* depth;
+  const int32_t* rank;
+} medusa_tree_t;
+
+/* Text for a status code (static storage). */
+MEDUSA_API const char* medusa_status_string(medusa_status_t status);
+/* Text of the last failing call on this host thread ("" if none). */
+MEDUSA_API const char* medusa_last_error(void);
+/* ABI version: major*10000 + minor*100 + patch. */
+MEDUSA_API int medusa_version(void);
+
+/* ------------------------------------------------------------------------
+ * medusa_heads_topk
+ *
+ * "Medusa Heads" glossary, "Comment les têtes prédisent les tokens
+ * suivants": head k is one feed-forward layer with a SiLU activation and a
+ * residual connection, followed by a projection to the vocabulary; every
+ * head reads the same last hidden state.  "Attention arborescente et
+ * acceptation": the heads' top choices (top-2, top-3, ...) feed the tree.
+ *
+ *   y_k   = h + SiLU(W1_k h + b1_k)
+ *   z_k   = W2_k y_k                      (no bias)
+ *   top-kmax of z_k per (sequence, head): values descending, equal values by
+ *   ascending token id.
+ *
+ * Inputs (device, dtype dt for h/W1/b1/W2):
+ *   h  [B, d]        last hidden state per sequence
+ *   W1 [K, d, d]     W1[k][j][:] = weights of output feature j (Linear layout)
+ *   b1 [K, d]
+ *   W2 [K, V, d]     W2[k][v][:] = weights of token v
+ * Outputs (device):
+ *   topk_ids  [B, K, kmax] int32
+ *   topk_vals [B, K, kmax] float32
+ *   logits    [B, K, V] float32, or NULL to skip (parity checks).
+ * Workspace: ws of at least medusa_heads_topk_workspace_size(...) bytes,
+ *   256-byte aligned; contents on entry are ignored.
+ * Precision: bf16 inputs, fp32 accumulation; y is fed to the vocabulary
+ *   projection as the sum of two bf16 terms (hi + lo) so its rounding stays
+ *   far below the fp32 accumulation error.  dt = MEDUSA_F32 runs an fp32
+ *   CUDA-core path (small shapes).
+ * Limits: 1 <= B <= MEDUSA_MAX_BATCH, 1 <= K <= MEDUSA_MAX_HEADS,
+ *   1 <= kmax <= min(MEDUSA_MAX_KMAX, V); bf16: d % 64 == 0, all pointers
+ *   16-byte aligned.
+ * ---------------------------------------------------------------------- */
+MEDUSA_API size_t medusa_heads_topk_workspace_size(int B, int d, int V, int K, int kmax,
+                                        medusa_dtype_t dt);
+MEDUSA_API medusa_status_t medusa_heads_topk(const void* h, const void* W1, const void* b1,
+                                  const void* W2, medusa_dtype_t dt, int B, int d,
+                                  int V, int K, int kmax, int32_t* topk_ids,
+                                  float* topk_vals, float* logits, void* ws,
+                                  size_t ws_bytes, int32_t* dev_status,
+                                  void* stream);
+
+/* ------------------------------------------------------------------------
+ * medusa_tree_build
+ *
+ * "Medusa Heads" glossary, "Attention arborescente et acceptation": the
+ * heads' top choices combine into candidate continuations forming a tree
+ * (a Cartesian product, or a sparse selection of it); head 2 proposes the
+ * same tokens under every head-1 branch; a mask lets each token see only its
+ * ancestors in the tree.
+ *
+ *   cand_ids[b][0] = root_tok[b] (the base model's own next token);
+ *   cand_ids[b][i] = topk_ids[b][depth[i]-1][rank[i]] for i > 0;
+ *   pos_ids[b][i]  = prefix_len[b] + depth[i];
+ *   anc_mask[i][w] bit t set iff node 32*w+t is i or an ancestor of i;
+ *   retrieve[p][t] = node at depth t on the path root -> p-th leaf (leaves in
+ *                    node order), -1 past the leaf.
+ *
+ * Inputs (device): root_tok [B] int32, topk_ids [B, K, kmax] int32,
+ *   prefix_len [B] int32; tree as above (depth[i] <= K required).
+ * Outputs (device): cand_ids [B, N], pos_ids [B, N] int32;
+ *   anc_mask [N, ceil(N/32)] uint32; retrieve [n_leaves, max_depth+1] int32.
+ * Limits: N <= MEDUSA_MAX_NODES, max_depth <= K <= MEDUSA_MAX_HEADS,
+ *   kmax <= MEDUSA_MAX_KMAX.
+ * ---------------------------------------------------------------------- */
+MEDUSA_API medusa_status_t medusa_tree_build(const medusa_tree_t* tree, const int32_t* root_tok,
+                                  const int32_t* topk_ids, int K, int kmax,
+                                  const int32_t* prefix_len, int B, int32_t* cand_ids,
+                                  int32_t* pos_ids, uint32_t* anc_mask,
+                                  int32_t* retrieve, int32_t* dev_status,
+                                  void* stream);
+
+/* ------------------------------------------------------------------------
+ * medusa_tree_attention
+ *
+ * "Medusa Heads" glossary, "Attention arborescente et acceptation": every
+ * candidate token is appended to the input at once and attends only to its
+ * ancestors, so one forward pass scores every branch; abstract of the Medusa
+ * paper: tree-based attention verifies all candidates in one step.
+ *
+ * The N tree tokens' K/V are written to cache slots prefix_len[b] + i.  Query
+ * (node i, head hq) then attends with weights softmax(scale * q.k) to slots
+ * [0, prefix_len[b]) and to slots prefix_len[b] + j for every j set in
+ * anc_mask row i.  Query head hq reads kv head hq / (Hq / Hkv).  No
+ * positional rotation is applied: q and k are taken as already positioned.
+ *
+ * Inputs (device, dtype dt): q [B, N, Hq, dh]; k_new, v_new [B, N, Hkv, dh];
+ *   caches Kc, Vc [B, Hkv, cap, dh] (read, and written at the tree slots);
+ *   prefix_len [B] int32 with prefix_len[b] <= max_prefix and
+ *   prefix_len[b] + N <= cap; anc_mask from medusa_tree_build.
+ * Output (device): out [B, N, Hq, dh] of dtype out_dt (bf16 or f32).
+ * max_prefix: host-side upper bound on every prefix_len[b]; sizes the launch.
+ * Workspace: medusa_tree_attention_workspace_size(...) bytes (split-KV
+ *   partial results), 256-byte aligned.
+ * Precision: bf16 q/k/v, fp32 scores, fp32 softmax statistics; the softmax
+ *   weights enter the value product as two bf16 terms (hi + lo).
+ *   dt = MEDUSA_F32 runs an fp32 CUDA-core path.
+ * Limits: Hq % Hkv == 0; bf16: dh in {64, 128}, pointers 16-byte aligned;
+ *   f32: dh <= 256 and dh % 32 == 0; N <= MEDUSA_MAX_NODES.
+ * ---------------------------------------------------------------------- */
+MEDUSA_API size_t medusa_tree_attention_workspace_size(int B, int N, int Hq, int Hkv, int dh,
+                                            int max_prefix, medusa_dtype_t dt);
+MEDUSA_API medusa_status_t medusa_tree_attention(const void* q, const void* k_new, const void* v_new,
+                                      void* Kc, void* Vc, const int32_t* prefix_len,
+                                      const uint32_t* anc_mask, medusa_dtype_t dt, int B,
+                                      int N, int Hq, int Hkv, int dh, int cap,
+                                      int max_prefix, float scale, void* out,
+                                      medusa_dtype_t out_dt, void* ws, size_t ws_bytes,
+                                      int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
+ * medusa_verify_accept
+ *
+ * "Medusa Heads" glossary, "Attention arborescente et acceptation": the
+ * longest branch the model agrees with is kept.  Greedy: a candidate is
+ * accepted when it equals the model's first choice.  Typical: a candidate is
+ * kept when its probability under the base model exceeds a threshold tied to
+ * the entropy of the distribution; here thr = min(eps, delta * exp(-H(p))),
+ * p = softmax(logits / temperature), H in nats, strict ">".  "Medusa no
+ * contexto de LLMs": on rejection the conventionally generated token is
+ * used (the bonus token).
+ *
+ *   g[i]   = argmax_v logits[b][i][v] (lowest v among equal maxima);
+ *   node c > 0 passes iff g[parent[c]] == cand_ids[b][c] (greedy) or
+ *          p_parent[c](cand_ids[b][c]) > thr_parent[c] (typical);
+ *   the root is accepted; c is accepted iff it passes and parent[c] is;
+ *   kept node = deepest accepted node, lowest index among equally deep;
+ *   accept_len[b] = its depth; accepted_nodes[b] = root..kept node, then -1;
+ *   accepted_tokens[b] = kept candidates' tokens (root excluded), then the
+ *   bonus token, then -1; bonus[b] = g[kept node].
+ *
+ * Inputs (device): logits [B, N, V] of dtype dt; cand_ids [B, N] int32; tree.
+ * Outputs (device): accept_len [B], accepted_nodes [B, max_depth+1],
+ *   accepted_tokens [B, max_depth+1], bonus [B], all int32.
+ * Workspace: medusa_verify_accept_workspace_size(...) bytes, 256-byte aligned.
+ * Limits: N <= MEDUSA_MAX_NODES; temperature > 0 (typical); eps, delta >= 0.
+ * Device checks: a NaN logit, a candidate id outside [0, V).
+ * ---------------------------------------------------------------------- */
+MEDUSA_API size_t medusa_verify_accept_workspace_size(int B, int N, int V);
+MEDUSA_API medusa_status_t medusa_verify_accept(const void* logits, medusa_dtype_t dt,
+                                     const int32_t* cand_ids, const medusa_tree_t* tree,
+                                     int B, int V, medusa_accept_t mode, float temperature,
+                                     float eps, float delta, int32_t* accept_len,
+                                     int32_t* accepted_nodes, int32_t* accepted_tokens,
+                                     int32_t* bonus, void* ws, size_t ws_bytes,
+                                     int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
+ * medusa_kv_compact
+ *
+ * "Medusa no contexto de LLMs": an accepted candidate enters the sequence
+ * without another full pass; "Medusa Heads" glossary: only the longest
+ * accepted branch is kept.  The cache therefore keeps the kept branch's K/V
+ * in contiguous slots after the prefix and drops the rest of the tree.
+ *
+ *   for j = 0..L (L = accept_len[b], P = prefix_len[b]):
+ *       slot P + j of Kc and Vc (every kv head) <- slot P + accepted_nodes[b][j]
+ *   (as if done for ascending j; the kernel stages the sources first, so the
+ *   result is the same whichever slots overlap);
+ *   compact_src[b][j] = P + accepted_nodes[b][j] for j <= L, else -1;
+ *   prefix_len[b] = P + L + 1.
+ *
+ * In/out (device): Kc, Vc [B, Hkv, cap, dh] of dtype dt; prefix_len [B] int32.
+ * Inputs (device): accepted_nodes [B, max_depth+1], accept_len [B] int32.
+ * Output (device): compact_src [B, max_depth+1] int32.
+ * Limits: max_depth < MEDUSA_MAX_HEADS; bf16 pointers 16-byte aligned.
+ * Device checks: accept_len outside [0, max_depth], a source slot outside
+ *   [P, cap).
+ * ---------------------------------------------------------------------- */
+MEDUSA_API medusa_status_t medusa_kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
+                                  const int32_t* accepted_nodes, const int32_t* accept_len,
+                                  int B, int Hkv, int dh, int cap, int max_depth,
+                                  int32_t* compact_src, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MEDUSA_B200_H */

@@ -1,0 +1,244 @@
+"""ctypes binding of libmedusa_b200.so: one Python function per C entry point,
+same names, argument marshalling only (tensor -> pointer and sizes, stream
+handle).  Every step of the computation runs in the library's CUDA kernels;
+there is no fallback: a missing library or a non-OK status raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmedusa_b200.so")
+
+MEDUSA_BF16 = 0
+MEDUSA_F32 = 1
+MEDUSA_ACCEPT_GREEDY = 0
+MEDUSA_ACCEPT_TYPICAL = 1
+MAX_NODES = 256
+MAX_KMAX = 32
+MAX_HEADS = 16
+
+STATUS_NAMES = {
+    0: "MEDUSA_OK", 1: "MEDUSA_ERR_INVALID_ARG", 2: "MEDUSA_ERR_SHAPE",
+    3: "MEDUSA_ERR_UNSUPPORTED", 4: "MEDUSA_ERR_CUDA", 5: "MEDUSA_ERR_TIMEOUT",
+    6: "MEDUSA_ERR_DEVICE_CHECK", 7: "MEDUSA_ERR_WORKSPACE", 8: "MEDUSA_ERR_ALIGNMENT",
+}
+
+# exported symbols declared in include/medusa.h
+EXPORTS = (
+    "medusa_status_string", "medusa_last_error", "medusa_version",
+    "medusa_heads_topk_workspace_size", "medusa_heads_topk",
+    "medusa_tree_build",
+    "medusa_tree_attention_workspace_size", "medusa_tree_attention",
+    "medusa_verify_accept_workspace_size", "medusa_verify_accept",
+    "medusa_kv_compact",
+)
+
+
+class MedusaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class medusa_tree_t(ctypes.Structure):
+    _fields_ = [("n_nodes", ctypes.c_int32), ("max_depth", ctypes.c_int32),
+                ("n_leaves", ctypes.c_int32), ("parent", ctypes.c_void_p),
+                ("depth", ctypes.c_void_p), ("rank", ctypes.c_void_p)]
+
+
+_lib = None
+
+_V, _I, _Z, _F, _U = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float, ctypes.c_int
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (built by ``speculative_decoding_medusa_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: run `python -m speculative_decoding_medusa_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.medusa_status_string.restype = ctypes.c_char_p
+    L.medusa_status_string.argtypes = [_I]
+    L.medusa_last_error.restype = ctypes.c_char_p
+    L.medusa_last_error.argtypes = []
+    L.medusa_version.restype = _I
+    L.medusa_heads_topk_workspace_size.restype = _Z
+    L.medusa_heads_topk_workspace_size.argtypes = [_I] * 5 + [_I]
+    L.medusa_heads_topk.restype = _I
+    L.medusa_heads_topk.argtypes = [_V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _V, _V, _V, _V, _Z, _V, _V]
+    L.medusa_tree_build.restype = _I
+    L.medusa_tree_build.argtypes = [ctypes.POINTER(medusa_tree_t), _V, _V, _I, _I, _V, _I,
+                                    _V, _V, _V, _V, _V, _V]
+    L.medusa_tree_attention_workspace_size.restype = _Z
+    L.medusa_tree_attention_workspace_size.argtypes = [_I] * 6 + [_I]
+    L.medusa_tree_attention.restype = _I
+    L.medusa_tree_attention.argtypes = [_V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _I, _I,
+                                        _F, _V, _I, _V, _Z, _V, _V]
+    L.medusa_verify_accept_workspace_size.restype = _Z
+    L.medusa_verify_accept_workspace_size.argtypes = [_I, _I, _I]
+    L.medusa_verify_accept.restype = _I
+    L.medusa_verify_accept.argtypes = [_V, _I, _V, ctypes.POINTER(medusa_tree_t), _I, _I, _I, _F, _F,
+                                       _F, _V, _V, _V, _V, _V, _Z, _V, _V]
+    L.medusa_kv_compact.restype = _I
+    L.medusa_kv_compact.argtypes = [_V, _V, _I, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V, _V]
+    _lib = L
+    return L
+
+
+def _check(st: int) -> None:
+    if st != 0:
+        raise MedusaError(st, lib().medusa_last_error().decode())
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MEDUSA_BF16
+    if t.dtype == torch.float32:
+        return MEDUSA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _req(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def new_status(device=None) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A 256-byte aligned byte buffer (torch's caching allocator aligns to 512)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+class Tree:
+    """A candidate tree on the device (parent/depth/rank int32 arrays)."""
+
+    def __init__(self, parent, depth, rank, n_leaves: int, device=None):
+        dev = device or "cuda"
+        self.parent = torch.as_tensor(parent, dtype=torch.int32).to(dev).contiguous()
+        self.depth = torch.as_tensor(depth, dtype=torch.int32).to(dev).contiguous()
+        self.rank = torch.as_tensor(rank, dtype=torch.int32).to(dev).contiguous()
+        self.n_nodes = int(self.parent.numel())
+        self.max_depth = int(torch.as_tensor(depth).max().item()) if self.n_nodes else 0
+        self.n_leaves = int(n_leaves)
+
+    @classmethod
+    def from_spec(cls, spec, device=None) -> "Tree":
+        return cls(spec.parent, spec.depth, spec.rank, spec.n_leaves, device)
+
+    def c(self) -> medusa_tree_t:
+        return medusa_tree_t(self.n_nodes, self.max_depth, self.n_leaves,
+                             self.parent.data_ptr(), self.depth.data_ptr(), self.rank.data_ptr())
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+
+
+def medusa_heads_topk_workspace_size(B: int, d: int, V: int, K: int, kmax: int, dt: int) -> int:
+    return int(lib().medusa_heads_topk_workspace_size(B, d, V, K, kmax, dt))
+
+
+def medusa_heads_topk(h, W1, b1, W2, kmax: int, topk_ids, topk_vals, logits=None, ws=None,
+                      dev_status=None, stream=None) -> None:
+    """h [B,d], W1 [K,d,d], b1 [K,d], W2 [K,V,d] -> topk_ids/vals [B,K,kmax]
+    (and logits [B,K,V] fp32 when given)."""
+    for t, n in ((h, "h"), (W1, "W1"), (b1, "b1"), (W2, "W2"), (topk_ids, "topk_ids"),
+                 (topk_vals, "topk_vals")):
+        _req(t, n)
+    B, d = h.shape
+    K, V, _ = W2.shape
+    dt = _dt(W2)
+    if ws is None:
+        ws = workspace(medusa_heads_topk_workspace_size(B, d, V, K, kmax, dt), h.device)
+    _check(lib().medusa_heads_topk(_p(h), _p(W1), _p(b1), _p(W2), dt, B, d, V, K, kmax,
+                                   _p(topk_ids), _p(topk_vals), _p(logits), _p(ws), ws.numel(),
+                                   _p(dev_status), _stream(stream)))
+
+
+def medusa_tree_build(tree: Tree, root_tok, topk_ids, prefix_len, cand_ids, pos_ids, anc_mask,
+                      retrieve, dev_status=None, stream=None) -> None:
+    B, K, kmax = topk_ids.shape
+    ct = tree.c()
+    _check(lib().medusa_tree_build(ctypes.byref(ct), _p(root_tok), _p(topk_ids), K, kmax,
+                                   _p(prefix_len), B, _p(cand_ids), _p(pos_ids), _p(anc_mask),
+                                   _p(retrieve), _p(dev_status), _stream(stream)))
+
+
+def medusa_tree_attention_workspace_size(B: int, N: int, Hq: int, Hkv: int, dh: int,
+                                         max_prefix: int, dt: int) -> int:
+    return int(lib().medusa_tree_attention_workspace_size(B, N, Hq, Hkv, dh, max_prefix, dt))
+
+
+def medusa_tree_attention(q, k_new, v_new, Kc, Vc, prefix_len, anc_mask, max_prefix: int, out,
+                          scale: Optional[float] = None, ws=None, dev_status=None,
+                          stream=None) -> None:
+    """q [B,N,Hq,dh], k_new/v_new [B,N,Hkv,dh], Kc/Vc [B,Hkv,cap,dh] -> out [B,N,Hq,dh]."""
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (Kc, "Kc"), (Vc, "Vc"),
+                 (out, "out")):
+        _req(t, n)
+    B, N, Hq, dh = q.shape
+    Hkv, cap = Kc.shape[1], Kc.shape[2]
+    dt = _dt(q)
+    if scale is None:
+        scale = dh ** -0.5
+    if ws is None:
+        ws = workspace(medusa_tree_attention_workspace_size(B, N, Hq, Hkv, dh, max_prefix, dt),
+                       q.device)
+    _check(lib().medusa_tree_attention(_p(q), _p(k_new), _p(v_new), _p(Kc), _p(Vc),
+                                       _p(prefix_len), _p(anc_mask), dt, B, N, Hq, Hkv, dh, cap,
+                                       max_prefix, float(scale), _p(out), _dt(out), _p(ws),
+                                       ws.numel(), _p(dev_status), _stream(stream)))
+
+
+def medusa_verify_accept_workspace_size(B: int, N: int, V: int) -> int:
+    return int(lib().medusa_verify_accept_workspace_size(B, N, V))
+
+
+def medusa_verify_accept(logits, cand_ids, tree: Tree, accept_len, accepted_nodes,
+                         accepted_tokens, bonus, mode: int = MEDUSA_ACCEPT_GREEDY,
+                         temperature: float = 1.0, eps: float = 0.09, delta: float = 0.3,
+                         ws=None, dev_status=None, stream=None) -> None:
+    """logits [B,N,V] -> accept_len [B], accepted_nodes/tokens [B,Dmax+1], bonus [B]."""
+    _req(logits, "logits")
+    B, N, V = logits.shape
+    if ws is None:
+        ws = workspace(medusa_verify_accept_workspace_size(B, N, V), logits.device)
+    ct = tree.c()
+    _check(lib().medusa_verify_accept(_p(logits), _dt(logits), _p(cand_ids), ctypes.byref(ct), B, V,
+                                      mode, float(temperature), float(eps), float(delta),
+                                      _p(accept_len), _p(accepted_nodes), _p(accepted_tokens),
+                                      _p(bonus), _p(ws), ws.numel(), _p(dev_status),
+                                      _stream(stream)))
+
+
+def medusa_kv_compact(Kc, Vc, prefix_len, accepted_nodes, accept_len, compact_src,
+                      dev_status=None, stream=None) -> None:
+    _req(Kc, "Kc")
+    _req(Vc, "Vc")
+    B, Hkv, cap, dh = Kc.shape
+    max_depth = accepted_nodes.shape[1] - 1
+    _check(lib().medusa_kv_compact(_p(Kc), _p(Vc), _dt(Kc), _p(prefix_len), _p(accepted_nodes),
+                                   _p(accept_len), B, Hkv, dh, cap, max_depth, _p(compact_src),
+                                   _p(dev_status), _stream(stream)))

@@ -1,0 +1,51 @@
+// Internal host-side interface between the C entry points (abi.cu) and the
+// per-stage launchers.  Every launcher assumes its arguments were validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/medusa.h"
+
+namespace medusa {
+
+// record a message for medusa_last_error() and return `code`
+medusa_status_t fail(medusa_status_t code, const char* msg);
+// MEDUSA_OK, or MEDUSA_ERR_CUDA with the launch error text recorded
+medusa_status_t check_launch(const char* what);
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+size_t heads_topk_workspace_size(int B, int d, int V, int K, int kmax, medusa_dtype_t dt);
+medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const void* W2,
+                           medusa_dtype_t dt, int B, int d, int V, int K, int kmax,
+                           int32_t* topk_ids, float* topk_vals, float* logits, void* ws,
+                           int32_t* status, cudaStream_t stream);
+
+medusa_status_t tree_build(const medusa_tree_t& tree, const int32_t* root_tok,
+                           const int32_t* topk_ids, int K, int kmax, const int32_t* prefix_len,
+                           int B, int32_t* cand_ids, int32_t* pos_ids, uint32_t* anc_mask,
+                           int32_t* retrieve, int32_t* status, cudaStream_t stream);
+
+size_t tree_attention_workspace_size(int B, int N, int Hq, int Hkv, int dh, int max_prefix,
+                                     medusa_dtype_t dt);
+medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_new, void* Kc,
+                               void* Vc, const int32_t* prefix_len, const uint32_t* anc_mask,
+                               medusa_dtype_t dt, int B, int N, int Hq, int Hkv, int dh, int cap,
+                               int max_prefix, float scale, void* out, medusa_dtype_t out_dt,
+                               void* ws, int32_t* status, cudaStream_t stream);
+
+size_t verify_accept_workspace_size(int B, int N, int V);
+medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32_t* cand_ids,
+                              const medusa_tree_t& tree, int B, int V, medusa_accept_t mode,
+                              float temperature, float eps, float delta, int32_t* accept_len,
+                              int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
+                              void* ws, int32_t* status, cudaStream_t stream);
+
+medusa_status_t kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
+                           const int32_t* accepted_nodes, const int32_t* accept_len, int B,
+                           int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,
+                           int32_t* status, cudaStream_t stream);
+
+}  // namespace medusa

@@ -1,0 +1,520 @@
+// Medusa heads + per-head top-k.
+//
+// "Medusa Heads" glossary, "Comment les têtes prédisent les tokens suivants":
+// head k = h + SiLU(W1_k h + b1_k), then a projection W2_k to the vocabulary.
+//
+// bf16 path: two launches of one weight-streaming tcgen05 GEMM and a merge.
+//   1. W1 stage: U = W1 * h^T (rows = K*d output features, columns = batch).
+//      Epilogue: y = h + SiLU(U + b1), written as two bf16 rows (hi, lo) per
+//      sequence into Y [K, 2B, d] so that y enters the next GEMM at ~16-bit
+//      mantissa precision.
+//   2. W2 stage: Z = W2 * Y^T (rows = K*V tokens, columns = 2B); the epilogue
+//      adds the hi/lo columns, optionally stores the fp32 logits and keeps a
+//      per-warp top-kmax of every 32-row slice (warp bitonic sort).
+//   3. topk_merge: per (sequence, head), the best kmax of all slices.
+// The weights are the only large operand (K*(d^2 + V*d) bf16): every CTA
+// streams 128-row weight tiles through a TMA -> shared memory -> tcgen05.mma
+// pipeline; the batch sits in the MMA's N dimension (weight rows fill M=128).
+//
+// fp32 path (small shapes): warp-per-row CUDA-core dot products, same merge.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "abi_internal.h"
+#include "common.cuh"
+
+namespace medusa {
+
+// ----------------------------------------------------------------------------
+// weight-streaming GEMM on tcgen05
+// ----------------------------------------------------------------------------
+
+constexpr int kTileM = 128;  // weight rows per tile = UMMA M
+constexpr int kTileK = 64;   // bf16 elements per 128-byte swizzled row
+constexpr int kGemmThreads = 192;
+
+enum GemmMode { kModeW1 = 0, kModeW2 = 1 };
+
+struct GemmParams {
+  int rows_per_head;  // d (W1) or V (W2)
+  int n_heads;        // K
+  int d;              // reduction length
+  int B;              // sequences
+  int tiles_per_head;
+  int n_tiles;
+  int b_head_stride;  // 0: one B operand for all heads (W1), 1: per head (W2)
+  int kmax;
+  const __nv_bfloat16* h;     // [B, d] (W1 epilogue)
+  const __nv_bfloat16* b1;    // [K, d] (W1 epilogue)
+  __nv_bfloat16* Y;           // [K, 2B, d] (W1 epilogue output)
+  float* logits;              // [B, K, V] or null (W2 epilogue)
+  float* part_vals;           // [B*K, tiles_per_head*4, kmax] (W2)
+  int32_t* part_ids;
+  int32_t* status;
+};
+
+template <int NB, int S>
+struct GemmSmem {
+  static constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB
+  static constexpr int kBBytes = NB * kTileK * 2;
+  static constexpr int kStageTx = kABytes + kBBytes;
+  static constexpr int kAOff = 0;
+  static constexpr int kBOff = S * kABytes;
+  static constexpr int kBarOff = kBOff + S * kBBytes;
+  // full[S], empty[S], tfull[2], tempty[2], drain
+  static constexpr int kNumBars = 2 * S + 5;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // room to align the base
+};
+
+template <int NB>
+__host__ __device__ constexpr uint32_t tmem_cols() {
+  return (2 * NB) < 32 ? 32u : static_cast<uint32_t>(2 * NB);
+}
+
+template <int NB, int S, int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    heads_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+  using L = GemmSmem<NB, S>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* drain = bars + 2 * S + 4;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nkb = p.d / kTileK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, tmem_cols<NB>());
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      const uint64_t pol_a = l2_policy_evict_first();
+      const uint64_t pol_b = l2_policy_evict_last();
+      int g = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x) {
+        const int head = tile / p.tiles_per_head;
+        const int m0 = (tile - head * p.tiles_per_head) * kTileM;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % S;
+          const uint32_t ph = (g / S) & 1;
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], L::kStageTx);
+          tma_load_3d(smem + L::kAOff + s * L::kABytes, &tmA, &full[s], kb * kTileK, m0, head,
+                      pol_a);
+          tma_load_3d(smem + L::kBOff + s * L::kBBytes, &tmB, &full[s], kb * kTileK, 0,
+                      head * p.b_head_stride, pol_b);
+        }
+      }
+      // let every copy this thread issued land before the CTA can exit
+      const int first = g > S ? g - S : 0;
+      for (int x = first; x < g; ++x) {
+        int dummy_abort = 0;
+        mbar_wait_bounded(&full[x % S], (x / S) & 1, &dummy_abort, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(kTileM, NB);
+      int g = 0, it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[acc], aph ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * NB;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % S;
+          const uint32_t ph = (g / S) & 1;
+          if (!mbar_wait_bounded(&full[s], ph, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + L::kAOff + s * L::kABytes);
+          const uint32_t b_addr = smem_u32(smem + L::kBOff + s * L::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 16; ++kk) {
+            umma_bf16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32),
+                      idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&tfull[acc]);
+      }
+      // every MMA this thread issued must finish before TMEM is released
+      umma_commit(drain);
+      int dummy_abort = 0;
+      mbar_wait_bounded(drain, 0, &dummy_abort, p.status);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    const int row = quad * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!mbar_wait_bounded(&tfull[acc], aph, abort_flag, p.status)) break;
+      tc_fence_after();
+      const int head = tile / p.tiles_per_head;
+      const int tile_in_head = tile - head * p.tiles_per_head;
+      const int r = tile_in_head * kTileM + row;  // row within the head
+      const bool valid = r < p.rows_per_head;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * NB;
+#pragma unroll 1
+      for (int c0 = 0; c0 < NB; c0 += 16) {
+        float v[16];
+        tmem_ld16(taddr + c0, v);
+        tmem_ld_wait();
+        if (MODE == kModeW1) {
+          if (valid) {
+            const float bias = __bfloat162float(p.b1[(size_t)head * p.d + r]);
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              const int b = c0 + t;
+              if (b < p.B) {
+                const float u = v[t] + bias;
+                const float y = __bfloat162float(p.h[(size_t)b * p.d + r]) + u / (1.0f + expf(-u));
+                const __nv_bfloat16 hi = __float2bfloat16_rn(y);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(y - __bfloat162float(hi));
+                const size_t base = ((size_t)head * 2 * p.B + 2 * b) * p.d + r;
+                p.Y[base] = hi;
+                p.Y[base + p.d] = lo;
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int b = (c0 >> 1) + t;
+            if (b >= p.B) continue;  // uniform across the warp
+            const float z = v[2 * t] + v[2 * t + 1];
+            const size_t row_bk = (size_t)b * p.n_heads + head;
+            if (p.logits != nullptr && valid) p.logits[row_bk * p.rows_per_head + r] = z;
+            float sv = valid ? z : -INFINITY;
+            int si = valid ? r : 0x7fffffff;
+            warp_sort_desc(sv, si);
+            if (lane < p.kmax) {
+              const size_t o = ((row_bk * p.tiles_per_head + tile_in_head) * 4 + quad) * p.kmax + lane;
+              p.part_vals[o] = sv;
+              p.part_ids[o] = si;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols<NB>());
+  }
+}
+
+// ----------------------------------------------------------------------------
+// top-k merge: best kmax of C candidates per row
+// ----------------------------------------------------------------------------
+constexpr int kMergeWarps = 8;
+
+__global__ void __launch_bounds__(kMergeWarps * 32)
+    topk_merge_kernel(const float* __restrict__ vals, const int32_t* __restrict__ ids, long long C,
+                      int kmax, int32_t* __restrict__ out_ids, float* __restrict__ out_vals) {
+  __shared__ float sv[kMergeWarps][32];
+  __shared__ int si[kMergeWarps][32];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const size_t base = (size_t)blockIdx.x * C;
+  float rv = -INFINITY;
+  int ri = 0x7fffffff;
+  float tv = -INFINITY;
+  int ti = 0x7fffffff;
+  for (long long c = (long long)warp * 32; c < C; c += kMergeWarps * 32) {
+    const long long e = c + lane;
+    float v = -INFINITY;
+    int i = 0x7fffffff;
+    if (e < C) {
+      v = vals[base + e];
+      i = ids != nullptr ? ids[base + e] : static_cast<int>(e);
+    }
+    if (__any_sync(0xffffffffu, better(v, i, tv, ti))) {
+      warp_sort_desc(v, i);
+      warp_merge_top32(rv, ri, v, i);
+      tv = __shfl_sync(0xffffffffu, rv, kmax - 1);
+      ti = __shfl_sync(0xffffffffu, ri, kmax - 1);
+    }
+  }
+  sv[warp][lane] = rv;
+  si[warp][lane] = ri;
+  __syncthreads();
+  if (warp == 0) {
+    for (int w = 1; w < kMergeWarps; ++w) warp_merge_top32(rv, ri, sv[w][lane], si[w][lane]);
+    if (lane < kmax) {
+      out_ids[(size_t)blockIdx.x * kmax + lane] = ri;
+      out_vals[(size_t)blockIdx.x * kmax + lane] = rv;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// fp32 CUDA-core path
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// y[b][k][j] = h[b][j] + SiLU(W1[k][j] . h[b] + b1[k][j]); one warp per j.
+__global__ void __launch_bounds__(256)
+    heads_f32_w1_kernel(const float* __restrict__ h, const float* __restrict__ W1,
+                        const float* __restrict__ b1, int B, int d, int K, float* __restrict__ y) {
+  const int k = blockIdx.y;
+  const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (j >= d) return;
+  const float* w = W1 + ((size_t)k * d + j) * d;
+  for (int b = 0; b < B; ++b) {
+    float s = 0.f;
+    for (int e = lane; e < d; e += 32) s += w[e] * h[(size_t)b * d + e];
+    s = warp_sum(s);
+    if (lane == 0) {
+      const float u = s + b1[(size_t)k * d + j];
+      y[((size_t)b * K + k) * d + j] = h[(size_t)b * d + j] + u / (1.0f + expf(-u));
+    }
+  }
+}
+
+// z[b][k][v] = W2[k][v] . y[b][k]; one warp per v.
+__global__ void __launch_bounds__(256)
+    heads_f32_w2_kernel(const float* __restrict__ y, const float* __restrict__ W2, int B, int d,
+                        int V, int K, float* __restrict__ z) {
+  const int k = blockIdx.y;
+  const int v = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (v >= V) return;
+  const float* w = W2 + ((size_t)k * V + v) * d;
+  for (int b = 0; b < B; ++b) {
+    const float* yy = y + ((size_t)b * K + k) * d;
+    float s = 0.f;
+    for (int e = lane; e < d; e += 32) s += w[e] * yy[e];
+    s = warp_sum(s);
+    if (lane == 0) z[((size_t)b * K + k) * V + v] = s;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// host side
+// ----------------------------------------------------------------------------
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+  }
+  return fn;
+}
+
+// bf16 tensor [dim2][dim1][dim0] (dim0 contiguous), box {64, box1, 1},
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                 uint32_t box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {dim0, dim1, dim2};
+  cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kTileK), box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int NB, int S, int MODE>
+medusa_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
+                            cudaStream_t stream) {
+  using L = GemmSmem<NB, S>;
+  auto kern = heads_gemm_kernel<NB, S, MODE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
+      cudaSuccess)
+    return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(heads_gemm) failed");
+  const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
+  kern<<<grid, kGemmThreads, L::kAlloc, stream>>>(a, b, p);
+  return check_launch("heads_gemm");
+}
+
+template <int MODE>
+medusa_status_t launch_gemm_nb(int nb, const CUtensorMap& a, const CUtensorMap& b,
+                               const GemmParams& p, cudaStream_t s) {
+  switch (nb) {
+    case 16: return launch_gemm<16, 8, MODE>(a, b, p, s);
+    case 32: return launch_gemm<32, 8, MODE>(a, b, p, s);
+    case 64: return launch_gemm<64, 6, MODE>(a, b, p, s);
+    case 128: return launch_gemm<128, 4, MODE>(a, b, p, s);
+    case 256: return launch_gemm<256, 3, MODE>(a, b, p, s);
+  }
+  return fail(MEDUSA_ERR_UNSUPPORTED, "heads: unsupported MMA width");
+}
+
+int round_nb(int cols) {
+  int nb = 16;
+  while (nb < cols) nb *= 2;
+  return nb;
+}
+
+struct HeadsWs {
+  size_t y_bytes, part_bytes, total;
+};
+
+HeadsWs heads_ws_layout(int B, int d, int V, int K, int kmax, medusa_dtype_t dt) {
+  HeadsWs w{};
+  if (dt == MEDUSA_BF16) {
+    const size_t tph = (size_t)(V + kTileM - 1) / kTileM;
+    w.y_bytes = align256((size_t)K * 2 * B * d * 2);
+    w.part_bytes = align256((size_t)B * K * tph * 4 * kmax * 4);
+    w.total = w.y_bytes + 2 * w.part_bytes;
+  } else {
+    w.y_bytes = align256((size_t)B * K * d * 4);
+    w.part_bytes = align256((size_t)B * K * V * 4);
+    w.total = w.y_bytes + w.part_bytes;
+  }
+  return w;
+}
+
+}  // namespace
+
+size_t heads_topk_workspace_size(int B, int d, int V, int K, int kmax, medusa_dtype_t dt) {
+  return heads_ws_layout(B, d, V, K, kmax, dt).total;
+}
+
+medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const void* W2,
+                           medusa_dtype_t dt, int B, int d, int V, int K, int kmax,
+                           int32_t* topk_ids, float* topk_vals, float* logits, void* ws,
+                           int32_t* status, cudaStream_t stream) {
+  const HeadsWs w = heads_ws_layout(B, d, V, K, kmax, dt);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  if (dt == MEDUSA_F32) {
+    float* y = reinterpret_cast<float*>(wsb);
+    float* z = logits != nullptr ? logits : reinterpret_cast<float*>(wsb + w.y_bytes);
+    heads_f32_w1_kernel<<<dim3((d + 7) / 8, K), 256, 0, stream>>>(
+        static_cast<const float*>(h), static_cast<const float*>(W1),
+        static_cast<const float*>(b1), B, d, K, y);
+    medusa_status_t st = check_launch("heads_f32_w1");
+    if (st != MEDUSA_OK) return st;
+    heads_f32_w2_kernel<<<dim3((V + 7) / 8, K), 256, 0, stream>>>(
+        y, static_cast<const float*>(W2), B, d, V, K, z);
+    st = check_launch("heads_f32_w2");
+    if (st != MEDUSA_OK) return st;
+    topk_merge_kernel<<<B * K, kMergeWarps * 32, 0, stream>>>(z, nullptr, V, kmax, topk_ids,
+                                                              topk_vals);
+    return check_launch("topk_merge");
+  }
+
+  __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(wsb);
+  float* part_vals = reinterpret_cast<float*>(wsb + w.y_bytes);
+  int32_t* part_ids = reinterpret_cast<int32_t*>(wsb + w.y_bytes + w.part_bytes);
+
+  CUtensorMap mA1, mB1, mA2, mB2;
+  const int nb1 = round_nb(B);
+  const int nb2 = round_nb(2 * B);
+  if (!make_map_3d(&mA1, W1, d, d, K, kTileM) || !make_map_3d(&mB1, h, d, B, 1, nb1) ||
+      !make_map_3d(&mA2, W2, d, V, K, kTileM) || !make_map_3d(&mB2, Y, d, 2 * B, K, nb2))
+    return fail(MEDUSA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+
+  GemmParams p1{};
+  p1.rows_per_head = d;
+  p1.n_heads = K;
+  p1.d = d;
+  p1.B = B;
+  p1.tiles_per_head = (d + kTileM - 1) / kTileM;
+  p1.n_tiles = p1.tiles_per_head * K;
+  p1.b_head_stride = 0;
+  p1.kmax = kmax;
+  p1.h = static_cast<const __nv_bfloat16*>(h);
+  p1.b1 = static_cast<const __nv_bfloat16*>(b1);
+  p1.Y = Y;
+  p1.status = status;
+  medusa_status_t st = launch_gemm_nb<kModeW1>(nb1, mA1, mB1, p1, stream);
+  if (st != MEDUSA_OK) return st;
+
+  GemmParams p2 = p1;
+  p2.rows_per_head = V;
+  p2.tiles_per_head = (V + kTileM - 1) / kTileM;
+  p2.n_tiles = p2.tiles_per_head * K;
+  p2.b_head_stride = 1;
+  p2.logits = logits;
+  p2.part_vals = part_vals;
+  p2.part_ids = part_ids;
+  st = launch_gemm_nb<kModeW2>(nb2, mA2, mB2, p2, stream);
+  if (st != MEDUSA_OK) return st;
+
+  topk_merge_kernel<<<B * K, kMergeWarps * 32, 0, stream>>>(
+      part_vals, part_ids, (long long)p2.tiles_per_head * 4 * kmax, kmax, topk_ids, topk_vals);
+  return check_launch("topk_merge");
+}
+
+}  // namespace medusa

@@ -1,0 +1,338 @@
+// Verification and acceptance of the candidate tree.
+//
+// "Medusa Heads" glossary, "Attention arborescente et acceptation": the
+// longest branch the model agrees with is kept.  Greedy: a candidate is
+// accepted when it equals the model's first choice.  Typical: a candidate is
+// kept when its base-model probability exceeds a threshold tied to the
+// entropy of the distribution, here min(eps, delta * exp(-H)).
+// "Medusa no contexto de LLMs": on rejection the model's own token is used.
+//
+// Two launches.  verify_rows streams the [B*N, V] logits (the only large
+// input) once, in chunks of kVChunk tokens per CTA, and leaves per chunk the
+// max logit, its lowest index and, for typical acceptance, the partial sums
+// sum exp(z/T - m) and sum exp(z/T - m) * z/T.  verify_path, one CTA per
+// sequence, merges the chunks per node and runs the integer path selection.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "abi_internal.h"
+#include "common.cuh"
+
+namespace medusa {
+
+constexpr int kVChunk = 8192;
+constexpr int kRowThreads = 256;
+constexpr int kPer = kVChunk / kRowThreads;  // 32 logits per thread
+
+struct RowPart {
+  float maxz;
+  int idx;
+  float s;  // sum exp(z/T - maxz/T)
+  float t;  // sum exp(z/T - maxz/T) * z/T
+};
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    v[2 * e] = __uint_as_float(w[e] << 16);
+    v[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+template <typename T>
+__device__ __forceinline__ float load1(const T* p);
+template <>
+__device__ __forceinline__ float load1<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+template <>
+__device__ __forceinline__ float load1<float>(const float* p) {
+  return *p;
+}
+
+template <typename T, bool TYPICAL>
+__global__ void __launch_bounds__(kRowThreads)
+    verify_rows_kernel(const T* __restrict__ logits, int V, int n_chunks, float inv_T,
+                       RowPart* __restrict__ part, int32_t* status) {
+  const int c = blockIdx.x;
+  const size_t row = blockIdx.y;
+  const T* base = logits + row * V;
+  const int v0 = c * kVChunk;
+  const int tid = threadIdx.x;
+  float vals[kPer];
+  // contiguous runs of 8 per thread, coalesced across the block
+  const bool vec_ok = (V % 8) == 0;
+#pragma unroll
+  for (int r = 0; r < kPer / 8; ++r) {
+    const int e0 = v0 + (r * kRowThreads + tid) * 8;
+    float v8[8];
+    if (vec_ok && e0 + 8 <= V) {
+      load8(base + e0, v8);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v8[e] = (e0 + e < V) ? load1<T>(base + e0 + e) : -INFINITY;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) vals[r * 8 + e] = v8[e];
+  }
+  // best (largest, lowest index) of this thread; indices ascend within a run
+  float bv = -INFINITY;
+  int bi = 0x7fffffff;
+  bool nan = false;
+#pragma unroll
+  for (int r = 0; r < kPer / 8; ++r) {
+    const int e0 = v0 + (r * kRowThreads + tid) * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x = vals[r * 8 + e];
+      nan |= (x != x);
+      if (e0 + e < V && better(x, e0 + e, bv, bi)) {
+        bv = x;
+        bi = e0 + e;
+      }
+    }
+  }
+  if (nan) report(status, MEDUSA_ERR_DEVICE_CHECK);
+  // block reduction of (bv, bi)
+  __shared__ float s_v[kRowThreads / 32];
+  __shared__ int s_i[kRowThreads / 32];
+  __shared__ float s_m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (better(ov, oi, bv, bi)) {
+      bv = ov;
+      bi = oi;
+    }
+  }
+  const int warp = tid >> 5, lane = tid & 31;
+  if (lane == 0) {
+    s_v[warp] = bv;
+    s_i[warp] = bi;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float v = s_v[0];
+    int i = s_i[0];
+    for (int w = 1; w < kRowThreads / 32; ++w)
+      if (better(s_v[w], s_i[w], v, i)) {
+        v = s_v[w];
+        i = s_i[w];
+      }
+    s_m = v;
+    part[row * n_chunks + c].maxz = v;
+    part[row * n_chunks + c].idx = i;
+    if (!TYPICAL) {
+      part[row * n_chunks + c].s = 0.f;
+      part[row * n_chunks + c].t = 0.f;
+    }
+  }
+  if (!TYPICAL) return;
+  __syncthreads();
+  const float m = s_m * inv_T;
+  float ss = 0.f, tt = 0.f;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    if (vals[e] != -INFINITY) {
+      const float zt = vals[e] * inv_T;
+      const float w = expf(zt - m);
+      ss += w;
+      tt += w * zt;
+    }
+  }
+  __shared__ float s_s[kRowThreads / 32], s_t[kRowThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    tt += __shfl_xor_sync(0xffffffffu, tt, o);
+  }
+  if (lane == 0) {
+    s_s[warp] = ss;
+    s_t[warp] = tt;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float a = 0.f, bsum = 0.f;
+    for (int w = 0; w < kRowThreads / 32; ++w) {
+      a += s_s[w];
+      bsum += s_t[w];
+    }
+    part[row * n_chunks + c].s = a;
+    part[row * n_chunks + c].t = bsum;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(MEDUSA_MAX_NODES)
+    verify_path_kernel(const T* __restrict__ logits, const RowPart* __restrict__ part,
+                       int n_chunks, const int32_t* __restrict__ cand_ids,
+                       const int32_t* __restrict__ parent, const int32_t* __restrict__ depth,
+                       int N, int max_depth, int V, int typical, float inv_T, float eps,
+                       float delta, int32_t* __restrict__ accept_len,
+                       int32_t* __restrict__ accepted_nodes, int32_t* __restrict__ accepted_tokens,
+                       int32_t* __restrict__ bonus, int32_t* status) {
+  __shared__ int s_g[MEDUSA_MAX_NODES];
+  __shared__ float s_lse[MEDUSA_MAX_NODES];
+  __shared__ float s_logthr[MEDUSA_MAX_NODES];
+  __shared__ int s_parent[MEDUSA_MAX_NODES];
+  __shared__ int s_depth[MEDUSA_MAX_NODES];
+  __shared__ int s_pass[MEDUSA_MAX_NODES];
+  __shared__ int s_best;
+  __shared__ int s_bad;
+  const int b = blockIdx.x;
+  const int i = threadIdx.x;
+  if (i == 0) {
+    s_best = 0xFFFF;  // the root: depth 0, node 0
+    s_bad = 0;
+  }
+  if (i < N) {
+    s_parent[i] = parent[i];
+    s_depth[i] = depth[i];
+  }
+  __syncthreads();
+  if (i < N) {
+    const int pa = s_parent[i];
+    const int dp = s_depth[i];
+    const bool ok = (i == 0) ? (pa == -1 && dp == 0)
+                             : (pa >= 0 && pa < i && dp == s_depth[pa] + 1 && dp <= max_depth);
+    // merge the chunks of row (b, i)
+    const RowPart* rp = part + ((size_t)b * N + i) * n_chunks;
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    float M = -INFINITY;
+    for (int c = 0; c < n_chunks; ++c) {
+      const RowPart q = rp[c];
+      if (better(q.maxz, q.idx, bv, bi)) {
+        bv = q.maxz;
+        bi = q.idx;
+      }
+    }
+    s_g[i] = bi;
+    if (typical) {
+      M = bv * inv_T;
+      float S = 0.f, Tt = 0.f;
+      for (int c = 0; c < n_chunks; ++c) {
+        const RowPart q = rp[c];
+        const float w = expf(q.maxz * inv_T - M);
+        S += q.s * w;
+        Tt += q.t * w;
+      }
+      const float lse = M + logf(S);
+      const float H = lse - Tt / S;
+      const float thr = fminf(eps, delta * expf(-H));
+      s_lse[i] = lse;
+      s_logthr[i] = thr > 0.f ? logf(thr) : -INFINITY;
+    }
+    if (!ok) atomicOr(&s_bad, 1);
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (i == 0) {
+      report(status, MEDUSA_ERR_DEVICE_CHECK);
+      accept_len[b] = 0;
+    }
+    return;
+  }
+  if (i < N) {
+    int pass = 1;
+    if (i > 0) {
+      const int tok = cand_ids[(size_t)b * N + i];
+      const int pa = s_parent[i];
+      if (tok < 0 || tok >= V) {
+        report(status, MEDUSA_ERR_DEVICE_CHECK);
+        pass = 0;
+      } else if (!typical) {
+        pass = s_g[pa] == tok;
+      } else {
+        const float lp = load1<T>(logits + ((size_t)b * N + pa) * V + tok) * inv_T - s_lse[pa];
+        pass = lp > s_logthr[pa];
+      }
+    }
+    s_pass[i] = pass;
+  }
+  __syncthreads();
+  if (i < N) {
+    bool acc = true;
+    for (int j = i; j > 0 && acc; j = s_parent[j]) acc = s_pass[j] != 0;
+    if (acc) atomicMax(&s_best, (s_depth[i] << 16) | (0xFFFF - i));
+  }
+  __syncthreads();
+  if (i == 0) {
+    const int best = 0xFFFF - (s_best & 0xFFFF);
+    const int L = s_depth[best];
+    const size_t o = (size_t)b * (max_depth + 1);
+    for (int t = L + 1; t <= max_depth; ++t) {
+      accepted_nodes[o + t] = -1;
+      accepted_tokens[o + t] = -1;
+    }
+    for (int j = best; j >= 0; j = s_parent[j]) {
+      accepted_nodes[o + s_depth[j]] = j;
+      if (j > 0) accepted_tokens[o + s_depth[j] - 1] = cand_ids[(size_t)b * N + j];
+    }
+    accepted_tokens[o + L] = s_g[best];
+    accept_len[b] = L;
+    bonus[b] = s_g[best];
+  }
+}
+
+size_t verify_accept_workspace_size(int B, int N, int V) {
+  const size_t n_chunks = (size_t)(V + kVChunk - 1) / kVChunk;
+  return align256((size_t)B * N * n_chunks * sizeof(RowPart));
+}
+
+medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32_t* cand_ids,
+                              const medusa_tree_t& tree, int B, int V, medusa_accept_t mode,
+                              float temperature, float eps, float delta, int32_t* accept_len,
+                              int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
+                              void* ws, int32_t* status, cudaStream_t stream) {
+  const int N = tree.n_nodes;
+  const int n_chunks = (V + kVChunk - 1) / kVChunk;
+  RowPart* part = static_cast<RowPart*>(ws);
+  const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
+  const float inv_T = typical ? 1.0f / temperature : 1.0f;
+  dim3 grid(n_chunks, B * N);
+  if (dt == MEDUSA_BF16) {
+    const __nv_bfloat16* lg = static_cast<const __nv_bfloat16*>(logits);
+    if (typical)
+      verify_rows_kernel<__nv_bfloat16, true><<<grid, kRowThreads, 0, stream>>>(lg, V, n_chunks,
+                                                                                 inv_T, part, status);
+    else
+      verify_rows_kernel<__nv_bfloat16, false><<<grid, kRowThreads, 0, stream>>>(
+          lg, V, n_chunks, inv_T, part, status);
+    medusa_status_t st = check_launch("verify_rows");
+    if (st != MEDUSA_OK) return st;
+    verify_path_kernel<__nv_bfloat16><<<B, MEDUSA_MAX_NODES, 0, stream>>>(
+        lg, part, n_chunks, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
+        typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
+        status);
+    return check_launch("verify_path");
+  }
+  const float* lg = static_cast<const float*>(logits);
+  if (typical)
+    verify_rows_kernel<float, true><<<grid, kRowThreads, 0, stream>>>(lg, V, n_chunks, inv_T, part,
+                                                                      status);
+  else
+    verify_rows_kernel<float, false><<<grid, kRowThreads, 0, stream>>>(lg, V, n_chunks, inv_T,
+                                                                       part, status);
+  medusa_status_t st = check_launch("verify_rows");
+  if (st != MEDUSA_OK) return st;
+  verify_path_kernel<float><<<B, MEDUSA_MAX_NODES, 0, stream>>>(
+      lg, part, n_chunks, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
+      typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
+      status);
+  return check_launch("verify_path");
+}
+
+}  // namespace medusa

@@ -1,0 +1,63 @@
+"""One decode-verify step through the C ABI: buffers plus the five calls in
+order (heads + top-k, tree build, tree attention, verify/accept, KV compaction).
+Argument marshalling only; all arithmetic runs in libmedusa_b200.so."""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib as M
+
+
+class DecodeVerifyStep:
+    def __init__(self, *, B: int, d: int, V: int, K: int, kmax: int, tree: M.Tree, Hq: int,
+                 Hkv: int, dh: int, cap: int, max_prefix: int, dtype: torch.dtype,
+                 accept: str = "greedy", temperature: float = 1.0, eps: float = 0.09,
+                 delta: float = 0.3, head_logits: bool = False,
+                 attn_out_dtype: Optional[torch.dtype] = None, device="cuda"):
+        self.B, self.d, self.V, self.K, self.kmax = B, d, V, K, kmax
+        self.tree, self.Hq, self.Hkv, self.dh, self.cap = tree, Hq, Hkv, dh, cap
+        self.max_prefix = max_prefix
+        self.mode = M.MEDUSA_ACCEPT_TYPICAL if accept == "typical" else M.MEDUSA_ACCEPT_GREEDY
+        self.temperature, self.eps, self.delta = temperature, eps, delta
+        dt = M.MEDUSA_BF16 if dtype == torch.bfloat16 else M.MEDUSA_F32
+        N, W = tree.n_nodes, tree.max_depth + 1
+        i32 = dict(dtype=torch.int32, device=device)
+        self.topk_ids = torch.empty(B, K, kmax, **i32)
+        self.topk_vals = torch.empty(B, K, kmax, dtype=torch.float32, device=device)
+        self.head_logits = (torch.empty(B, K, V, dtype=torch.float32, device=device)
+                            if head_logits else None)
+        self.cand_ids = torch.empty(B, N, **i32)
+        self.pos_ids = torch.empty(B, N, **i32)
+        self.anc_mask = torch.empty(N, (N + 31) // 32, **i32)
+        self.retrieve = torch.empty(tree.n_leaves, W, **i32)
+        self.attn_out = torch.empty(B, N, Hq, dh, dtype=attn_out_dtype or dtype, device=device)
+        self.accept_len = torch.empty(B, **i32)
+        self.accepted_nodes = torch.empty(B, W, **i32)
+        self.accepted_tokens = torch.empty(B, W, **i32)
+        self.bonus = torch.empty(B, **i32)
+        self.compact_src = torch.empty(B, W, **i32)
+        self.status = torch.zeros(1, **i32)
+        self.ws_heads = M.workspace(M.medusa_heads_topk_workspace_size(B, d, V, K, kmax, dt), device)
+        self.ws_attn = M.workspace(M.medusa_tree_attention_workspace_size(
+            B, N, Hq, Hkv, dh, max_prefix, dt), device)
+        self.ws_verify = M.workspace(M.medusa_verify_accept_workspace_size(B, N, V), device)
+
+    def run(self, h, W1, b1, W2, root_tok, q, k_new, v_new, Kc, Vc, prefix_len, verify_logits,
+            stream=None) -> None:
+        """Enqueue one step on ``stream``.  Kc/Vc/prefix_len are updated in place
+        (tree K/V written, then the kept branch compacted, prefix advanced)."""
+        M.medusa_heads_topk(h, W1, b1, W2, self.kmax, self.topk_ids, self.topk_vals,
+                            self.head_logits, self.ws_heads, self.status, stream)
+        M.medusa_tree_build(self.tree, root_tok, self.topk_ids, prefix_len, self.cand_ids,
+                            self.pos_ids, self.anc_mask, self.retrieve, self.status, stream)
+        M.medusa_tree_attention(q, k_new, v_new, Kc, Vc, prefix_len, self.anc_mask,
+                                self.max_prefix, self.attn_out, None, self.ws_attn, self.status,
+                                stream)
+        M.medusa_verify_accept(verify_logits, self.cand_ids, self.tree, self.accept_len,
+                               self.accepted_nodes, self.accepted_tokens, self.bonus, self.mode,
+                               self.temperature, self.eps, self.delta, self.ws_verify,
+                               self.status, stream)
+        M.medusa_kv_compact(Kc, Vc, prefix_len, self.accepted_nodes, self.accept_len,
+                            self.compact_src, self.status, stream)

@@ -1,0 +1,119 @@
+"""GPU parity: medusa_tree_attention against the oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import speculative_decoding_medusa_b200 as M
+from oracle import medusa_oracle as O
+from speculative_decoding_medusa_b200 import workloads as W
+from tests.helpers import ATTN_REL_L2, LOGIT_MAX_ABS, f64, i64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _mask(spec, B):
+    tb = O.tree_build(spec.parent, spec.depth, spec.rank, np.zeros(B, np.int64),
+                      np.zeros((B, max(1, spec.max_depth), 32), np.int64), np.zeros(B, np.int64))
+    return tb["mask"]
+
+
+def _run_gpu(inp, mask, max_prefix, out_dtype):
+    dev = "cuda"
+    q, kn, vn, Kc, Vc = (inp[k].to(dev) for k in ("q", "k_new", "v_new", "Kc", "Vc"))
+    pl = inp["prefix_len"].to(dev)
+    B, N, Hq, dh = q.shape
+    out = torch.full((B, N, Hq, dh), float("nan"), dtype=out_dtype, device=dev)
+    m = torch.from_numpy(mask.view(np.int32).copy()).to(dev)
+    status = M.new_status()
+    M.medusa_tree_attention(q, kn, vn, Kc, Vc, pl, m, max_prefix, out, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return f64(out), Kc.cpu(), Vc.cpu()
+
+
+def _compare(inp, spec, max_prefix, out_dtype=torch.float32, rows=None):
+    mask = _mask(spec, inp["q"].shape[0])
+    got, Kg, Vg = _run_gpu(inp, mask, max_prefix, out_dtype)
+    dh = inp["q"].shape[-1]
+    P = i64(inp["prefix_len"])
+    if rows is None:
+        ref = O.tree_attention(f64(inp["q"]), f64(inp["k_new"]), f64(inp["v_new"]), f64(inp["Kc"]),
+                               f64(inp["Vc"]), P, mask, 1.0 / math.sqrt(dh))
+        out_ref, Kr, Vr = ref["out"], ref["Kc"], ref["Vc"]
+        g = got
+    else:  # sampled (sequence, node) rows, all heads, the oracle one row at a time
+        out_ref = np.stack([_oracle_row(inp, mask, b, i, P[b], dh) for b, i in rows])
+        g = np.stack([got[b, i] for b, i in rows])
+        Kr = Vr = None
+    err = np.abs(g - out_ref).max()
+    assert err < LOGIT_MAX_ABS, err
+    if out_dtype == torch.float32:
+        assert rel_l2(g, out_ref) < ATTN_REL_L2, rel_l2(g, out_ref)
+    else:  # bf16 output adds its own rounding (relative 2^-9)
+        assert rel_l2(g, out_ref) < 4e-3
+    if Kr is not None:  # the tree K/V landed in their cache slots, bit for bit
+        np.testing.assert_array_equal(Kg.double().numpy(), Kr)
+        np.testing.assert_array_equal(Vg.double().numpy(), Vr)
+
+
+def _oracle_row(inp, mask, b, i, P, dh):
+    """Oracle tree attention for node i of sequence b only (all query heads):
+    the oracle is run on a one-node query whose mask row is node i's."""
+    N = inp["q"].shape[1]
+    # the oracle is given only node i's visible tree nodes (ancestors and
+    # itself, in node order) as its tree, every one of them visible
+    vis = [j for j in range(N) if O.mask_bit(mask, i, j)]
+    kn = f64(inp["k_new"][b:b + 1, vis])
+    vn = f64(inp["v_new"][b:b + 1, vis])
+    nvis = len(vis)
+    mm = np.zeros((nvis, (nvis + 31) // 32), dtype=np.uint32)
+    for r in range(nvis):
+        for j in range(nvis):
+            mm[r, j // 32] |= np.uint32(1 << (j % 32))
+    q = np.repeat(f64(inp["q"][b:b + 1, i:i + 1]), nvis, axis=1)
+    res = O.tree_attention(q, kn, vn, f64(inp["Kc"][b:b + 1]), f64(inp["Vc"][b:b + 1]),
+                           np.array([P]), mm, 1.0 / math.sqrt(dh))
+    return res["out"][0, 0]
+
+
+def test_tiny_fp32():
+    w = W.WORKLOADS["tiny"]
+    spec = W.tree_for(w)
+    inp = W.attention_inputs(w, seed=0)
+    _compare(inp, spec, w.ctx_hi)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,dh,ctx,tree,seed", [
+    (2, 8, 2, 128, (100, 700), "sparse64", 0),     # ragged, split boundaries, GQA 4
+    (1, 4, 4, 64, (64, 64), "cart23", 1),          # dh 64, prefix = one tile
+    (3, 8, 1, 128, (1, 200), "sparse16", 2),       # MQA, tiny prefixes
+    (2, 16, 2, 128, (0, 0), "sparse64", 3),        # empty prefix: tree only
+    (1, 8, 8, 128, (1500, 1500), "dense256", 4),   # 256 nodes, 8 mask words
+])
+def test_bf16_small(B, Hq, Hkv, dh, ctx, tree, seed):
+    if tree == "sparse64":
+        spec = W.sparse_tree(64, 4, 10, seed, max_depth=4)
+    elif tree == "sparse16":
+        spec = W.sparse_tree(16, 4, 10, seed, max_depth=4)
+    elif tree == "dense256":
+        spec = W.cartesian_tree([4, 4, 4, 4], n_nodes=256)
+    else:
+        spec = W.cartesian_tree([2, 3])
+    w = W.scaled(W.WORKLOADS["llama3_8b"], B=B, Hq=Hq, Hkv=Hkv, dh=dh, ctx_lo=ctx[0],
+                 ctx_hi=ctx[1], N=spec.n_nodes)
+    inp = W.attention_inputs(w, seed=seed)
+    _compare(inp, spec, w.ctx_hi)
+    _compare(W.attention_inputs(w, seed=seed), spec, w.ctx_hi, out_dtype=torch.bfloat16)
+
+
+@pytest.mark.slow
+def test_llama3_8b_full_size_sampled_rows():
+    w = W.WORKLOADS["llama3_8b"]
+    spec = W.tree_for(w)
+    inp = W.attention_inputs(w, seed=0)
+    rng = np.random.default_rng(0)
+    rows = [(int(rng.integers(w.B)), int(rng.integers(w.N))) for _ in range(24)]
+    rows += [(0, 0), (w.B - 1, w.N - 1)]
+    _compare(inp, spec, w.ctx_hi, rows=rows)
