@@ -286,6 +286,32 @@ MEDUSA_API medusa_status_t medusa_kv_compact(void* Kc, void* Vc, medusa_dtype_t 
                                   int B, int Hkv, int dh, int cap, int max_depth,
                                   int32_t* compact_src, int32_t* dev_status, void* stream);
 
+/* ------------------------------------------------------------------------
+ * medusa_verify_accept_noalloc
+ *
+ * No counterpart on the Medusa pages: a service of this library for callers
+ * that cannot provide device memory per call - a host framework that reserves
+ * all device memory up front and forbids allocating more at run time, or hot
+ * paths that must avoid cudaMalloc/cudaFree because those calls can
+ * synchronise the device.
+ *
+ * Same arguments, results, checks and errors as medusa_verify_accept, without
+ * ws/ws_bytes: the row statistics go to a 4 MiB array compiled into the
+ * library (every GPU that loads the library holds it until the process
+ * exits).  Requests needing more, i.e. B * n_nodes * ceil(V / 8192) * 16 bytes
+ * > 4 MiB, are rejected with MEDUSA_ERR_WORKSPACE before any launch.  Nothing
+ * is allocated.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  All calls share the one array and it keeps
+ * the last call's contents: calls whose kernels overlap on the GPU (e.g. on
+ * two streams at once) race and give wrong results.
+ * ---------------------------------------------------------------------- */
+MEDUSA_API medusa_status_t medusa_verify_accept_noalloc(
+    const void* logits, medusa_dtype_t dt, const int32_t* cand_ids, const medusa_tree_t* tree,
+    int B, int V, medusa_accept_t mode, float temperature, float eps, float delta,
+    int32_t* accept_len, int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
+    int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

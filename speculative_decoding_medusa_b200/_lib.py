@@ -35,7 +35,7 @@ EXPORTS = (
     "medusa_tree_build",
     "medusa_tree_attention_workspace_size", "medusa_tree_attention",
     "medusa_verify_accept_workspace_size", "medusa_verify_accept",
-    "medusa_kv_compact",
+    "medusa_kv_compact", "medusa_verify_accept_noalloc",
 )
 
 
@@ -86,6 +86,9 @@ def lib() -> ctypes.CDLL:
     L.medusa_verify_accept.restype = _I
     L.medusa_verify_accept.argtypes = [_V, _I, _V, ctypes.POINTER(medusa_tree_t), _I, _I, _I, _F, _F,
                                        _F, _V, _V, _V, _V, _V, _Z, _V, _V]
+    L.medusa_verify_accept_noalloc.restype = _I
+    L.medusa_verify_accept_noalloc.argtypes = [_V, _I, _V, ctypes.POINTER(medusa_tree_t), _I, _I, _I,
+                                               _F, _F, _F, _V, _V, _V, _V, _V, _V]
     L.medusa_kv_compact.restype = _I
     L.medusa_kv_compact.argtypes = [_V, _V, _I, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V, _V]
     _lib = L
@@ -242,3 +245,21 @@ def medusa_kv_compact(Kc, Vc, prefix_len, accepted_nodes, accept_len, compact_sr
     _check(lib().medusa_kv_compact(_p(Kc), _p(Vc), _dt(Kc), _p(prefix_len), _p(accepted_nodes),
                                    _p(accept_len), B, Hkv, dh, cap, max_depth, _p(compact_src),
                                    _p(dev_status), _stream(stream)))
+
+
+def medusa_verify_accept_noalloc(logits, cand_ids, tree: Tree, accept_len, accepted_nodes,
+                                 accepted_tokens, bonus, mode: int = MEDUSA_ACCEPT_GREEDY,
+                                 temperature: float = 1.0, eps: float = 0.09, delta: float = 0.3,
+                                 dev_status=None, stream=None) -> None:
+    """medusa_verify_accept without a workspace argument, for callers that
+    cannot hand the library device memory per call: the library keeps its
+    own fixed 4 MiB scratch on each device.  Calls that overlap on the GPU
+    share that scratch and race."""
+    _req(logits, "logits")
+    B, N, V = logits.shape
+    ct = tree.c()
+    _check(lib().medusa_verify_accept_noalloc(_p(logits), _dt(logits), _p(cand_ids),
+                                              ctypes.byref(ct), B, V, mode, float(temperature),
+                                              float(eps), float(delta), _p(accept_len),
+                                              _p(accepted_nodes), _p(accepted_tokens), _p(bonus),
+                                              _p(dev_status), _stream(stream)))

@@ -17,6 +17,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "abi_internal.h"
 #include "common.cuh"
 
@@ -336,3 +338,60 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
 }
 
 }  // namespace medusa
+
+// ---------------------------------------------------------------------------
+// medusa_verify_accept_noalloc: the same verification with no caller-supplied
+// workspace.  Some callers cannot hand this library device memory per call:
+// a host framework that owns and pre-reserves all device memory and forbids
+// growing it at run time, or code that must not call cudaMalloc/cudaFree on
+// the hot path because those calls can synchronise the device.  For them the
+// per-chunk row statistics live in a fixed array compiled into the library.
+// ---------------------------------------------------------------------------
+namespace {
+
+// 4 MiB holds B * N * ceil(V / 8192) 16-byte row records up to 262144 records
+// (for example B = 32, N = 128, V = 128256).  Every GPU that loads the library
+// keeps this array until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_verify_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::atomic<void*> g_verify_noalloc_ptr[kNoAllocMaxDevices];
+
+}  // namespace
+
+extern "C" medusa_status_t medusa_verify_accept_noalloc(
+    const void* logits, medusa_dtype_t dt, const int32_t* cand_ids, const medusa_tree_t* tree,
+    int B, int V, medusa_accept_t mode, float temperature, float eps, float delta,
+    int32_t* accept_len, int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
+    int32_t* dev_status, void* stream) {
+  if (tree == nullptr)
+    return medusa::fail(MEDUSA_ERR_INVALID_ARG, "verify_accept_noalloc: null tree");
+  if (B >= 1 && V >= 1 && tree->n_nodes >= 1 &&
+      medusa::verify_accept_workspace_size(B, tree->n_nodes, V) > kNoAllocScratchBytes)
+    return medusa::fail(MEDUSA_ERR_WORKSPACE,
+                        "verify_accept_noalloc: B * n_nodes * ceil(V / 8192) * 16 bytes exceeds "
+                        "the 4 MiB static scratch; use medusa_verify_accept with a workspace");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
+    return medusa::fail(MEDUSA_ERR_CUDA, "verify_accept_noalloc: cudaGetDevice failed");
+  if (dev >= kNoAllocMaxDevices)
+    return medusa::fail(MEDUSA_ERR_UNSUPPORTED, "verify_accept_noalloc: device index >= 64");
+  // host code sees only a stand-in for the device array: its device address
+  // is looked up once per device, with that device current
+  void* scratch = g_verify_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (scratch == nullptr) {
+    const cudaError_t e = cudaGetSymbolAddress(&scratch, g_verify_noalloc_scratch);
+    if (e != cudaSuccess || scratch == nullptr) {
+      cudaGetLastError();
+      return medusa::fail(MEDUSA_ERR_CUDA,
+                          "verify_accept_noalloc: cudaGetSymbolAddress of the scratch failed");
+    }
+    g_verify_noalloc_ptr[dev].store(scratch, std::memory_order_release);
+  }
+  // every row record is written by the row kernel before the path kernel
+  // reads it, so the scratch needs no clearing between calls
+  return medusa_verify_accept(logits, dt, cand_ids, tree, B, V, mode, temperature, eps, delta,
+                              accept_len, accepted_nodes, accepted_tokens, bonus, scratch,
+                              kNoAllocScratchBytes, dev_status, stream);
+}
