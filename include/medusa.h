@@ -298,7 +298,7 @@ MEDUSA_API medusa_status_t medusa_kv_compact(void* Kc, void* Vc, medusa_dtype_t 
  * Same arguments, results, checks and errors as medusa_verify_accept, without
  * ws/ws_bytes: the row statistics go to a 4 MiB array compiled into the
  * library (every GPU that loads the library holds it until the process
- * exits).  Requests needing more, i.e. B * n_nodes * ceil(V / 8192) * 16 bytes
+ * exits).  Requests needing more, i.e. B * n_nodes * ceil(V / 4096) * 16 bytes
  * > 4 MiB, are rejected with MEDUSA_ERR_WORKSPACE before any launch.  Nothing
  * is allocated.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress) with that device current; make that first

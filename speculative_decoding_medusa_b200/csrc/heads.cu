@@ -51,7 +51,7 @@ struct GemmParams {
   const __nv_bfloat16* b1;    // [K, d] (W1 epilogue)
   __nv_bfloat16* Y;           // [K, 2B, d] (W1 epilogue output)
   float* logits;              // [B, K, V] or null (W2 epilogue)
-  float* part_vals;           // [B*K, tiles_per_head*4, kmax] (W2)
+  float* part_vals;           // [B*K, tiles_per_head, kmax] (W2)
   int32_t* part_ids;
   int32_t* status;
 };
@@ -64,10 +64,13 @@ struct GemmSmem {
   static constexpr int kAOff = 0;
   static constexpr int kBOff = S * kABytes;
   static constexpr int kBarOff = kBOff + S * kBBytes;
-  // full[S], empty[S], tfull[2], tempty[2], drain
-  static constexpr int kNumBars = 2 * S + 5;
+  // full[S], empty[S], tfull[2], tempty[2], drain, epilogue
+  static constexpr int kNumBars = 2 * S + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16;
+  // per-warp sorted lists of the W2 epilogue: [4 quads][8 sequences][32] (value, index)
+  static constexpr int kListOff = kMiscOff + 16;
+  static constexpr int kListBytes = 4 * 8 * 32 * 8;
+  static constexpr int kBytes = kListOff + kListBytes;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base
 };
 
@@ -89,6 +92,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = bars + 2 * S;
   uint64_t* tempty = bars + 2 * S + 2;
   uint64_t* drain = bars + 2 * S + 4;
+  uint64_t* epi = bars + 2 * S + 5;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -106,6 +110,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    mbar_init(epi, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -191,8 +196,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------- epilogue (warps 2..5) ----------------
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;
+    // the four epilogue warps synchronise on an mbarrier with a bounded wait,
+    // so that one warp giving up cannot leave the others blocked
+    uint32_t epi_phase = 0;
+    bool epi_ok = true;
+    auto epi_sync = [&]() {
+      mbar_arrive(epi);
+      epi_ok = mbar_wait_bounded(epi, epi_phase, abort_flag, p.status);
+      epi_phase ^= 1u;
+      return epi_ok;
+    };
     int it = 0;
-    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
+    for (int tile = blockIdx.x; epi_ok && tile < p.n_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       if (!mbar_wait_bounded(&tfull[acc], aph, abort_flag, p.status)) break;
@@ -203,7 +218,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const bool valid = r < p.rows_per_head;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * NB;
 #pragma unroll 1
-      for (int c0 = 0; c0 < NB; c0 += 16) {
+      for (int c0 = 0; epi_ok && c0 < NB; c0 += 16) {
         float v[16];
         tmem_ld16(taddr + c0, v);
         tmem_ld_wait();
@@ -225,6 +240,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         } else {
+          float* lv = reinterpret_cast<float*>(smem + L::kListOff);
+          int* li = reinterpret_cast<int*>(smem + L::kListOff + 4 * 8 * 32 * 4);
+          // each warp sorts its 32 rows per sequence ...
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
             const int b = (c0 >> 1) + t;
@@ -235,12 +253,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float sv = valid ? z : -INFINITY;
             int si = valid ? r : 0x7fffffff;
             warp_sort_desc(sv, si);
+            lv[(quad * 8 + t) * 32 + lane] = sv;
+            li[(quad * 8 + t) * 32 + lane] = si;
+          }
+          if (!epi_sync()) break;
+          // ... then warp `quad` merges the four lists of sequences quad, quad+4
+#pragma unroll
+          for (int t = quad; t < 8; t += 4) {
+            const int b = (c0 >> 1) + t;
+            if (b >= p.B) continue;
+            float rv = lv[t * 32 + lane];
+            int ri = li[t * 32 + lane];
+#pragma unroll
+            for (int q2 = 1; q2 < 4; ++q2)
+              warp_merge_top32(rv, ri, lv[(q2 * 8 + t) * 32 + lane], li[(q2 * 8 + t) * 32 + lane]);
             if (lane < p.kmax) {
-              const size_t o = ((row_bk * p.tiles_per_head + tile_in_head) * 4 + quad) * p.kmax + lane;
-              p.part_vals[o] = sv;
-              p.part_ids[o] = si;
+              const size_t row_bk = (size_t)b * p.n_heads + head;
+              const size_t o = (row_bk * p.tiles_per_head + tile_in_head) * p.kmax + lane;
+              p.part_vals[o] = rv;
+              p.part_ids[o] = ri;
             }
           }
+          if (!epi_sync()) break;
         }
       }
       tc_fence_before();
@@ -259,7 +293,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ----------------------------------------------------------------------------
 // top-k merge: best kmax of C candidates per row
 // ----------------------------------------------------------------------------
-constexpr int kMergeWarps = 8;
+constexpr int kMergeWarps = 32;
+constexpr int kMergeUnroll = 4;  // 32-candidate chunks each warp has in flight
 
 __global__ void __launch_bounds__(kMergeWarps * 32)
     topk_merge_kernel(const float* __restrict__ vals, const int32_t* __restrict__ ids, long long C,
@@ -269,23 +304,33 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const size_t base = (size_t)blockIdx.x * C;
+  // running best-32 of this warp, sorted, and its kmax-th entry as a filter
   float rv = -INFINITY;
   int ri = 0x7fffffff;
   float tv = -INFINITY;
   int ti = 0x7fffffff;
-  for (long long c = (long long)warp * 32; c < C; c += kMergeWarps * 32) {
-    const long long e = c + lane;
-    float v = -INFINITY;
-    int i = 0x7fffffff;
-    if (e < C) {
-      v = vals[base + e];
-      i = ids != nullptr ? ids[base + e] : static_cast<int>(e);
+  for (long long c = (long long)warp * 32 * kMergeUnroll; c < C;
+       c += (long long)kMergeWarps * 32 * kMergeUnroll) {
+    float v[kMergeUnroll];
+    int i[kMergeUnroll];
+#pragma unroll
+    for (int u = 0; u < kMergeUnroll; ++u) {
+      const long long e = c + u * 32 + lane;
+      v[u] = -INFINITY;
+      i[u] = 0x7fffffff;
+      if (e < C) {
+        v[u] = vals[base + e];
+        i[u] = ids != nullptr ? ids[base + e] : static_cast<int>(e);
+      }
     }
-    if (__any_sync(0xffffffffu, better(v, i, tv, ti))) {
-      warp_sort_desc(v, i);
-      warp_merge_top32(rv, ri, v, i);
-      tv = __shfl_sync(0xffffffffu, rv, kmax - 1);
-      ti = __shfl_sync(0xffffffffu, ri, kmax - 1);
+#pragma unroll
+    for (int u = 0; u < kMergeUnroll; ++u) {
+      if (__any_sync(0xffffffffu, better(v[u], i[u], tv, ti))) {
+        warp_sort_desc(v[u], i[u]);
+        warp_merge_top32(rv, ri, v[u], i[u]);
+        tv = __shfl_sync(0xffffffffu, rv, kmax - 1);
+        ti = __shfl_sync(0xffffffffu, ri, kmax - 1);
+      }
     }
   }
   sv[warp][lane] = rv;
@@ -435,7 +480,7 @@ HeadsWs heads_ws_layout(int B, int d, int V, int K, int kmax, medusa_dtype_t dt)
   if (dt == MEDUSA_BF16) {
     const size_t tph = (size_t)(V + kTileM - 1) / kTileM;
     w.y_bytes = align256((size_t)K * 2 * B * d * 2);
-    w.part_bytes = align256((size_t)B * K * tph * 4 * kmax * 4);
+    w.part_bytes = align256((size_t)B * K * tph * kmax * 4);
     w.total = w.y_bytes + 2 * w.part_bytes;
   } else {
     w.y_bytes = align256((size_t)B * K * d * 4);
@@ -513,7 +558,7 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
   if (st != MEDUSA_OK) return st;
 
   topk_merge_kernel<<<B * K, kMergeWarps * 32, 0, stream>>>(
-      part_vals, part_ids, (long long)p2.tiles_per_head * 4 * kmax, kmax, topk_ids, topk_vals);
+      part_vals, part_ids, (long long)p2.tiles_per_head * kmax, kmax, topk_ids, topk_vals);
   return check_launch("topk_merge");
 }
 

@@ -23,8 +23,10 @@ __global__ void __launch_bounds__(kCompactThreads)
     kv_compact_kernel(uint8_t* Kc, uint8_t* Vc, int row_bytes, int32_t* prefix_len,
                       const int32_t* __restrict__ accepted_nodes,
                       const int32_t* __restrict__ accept_len, int Hkv, int cap, int max_depth,
-                      int32_t* __restrict__ compact_src, int32_t* status) {
-  extern __shared__ __align__(16) uint8_t stage[];  // [2][max_depth+1][row_bytes]
+                      int heads_at_once, int32_t* __restrict__ compact_src, int32_t* status) {
+  // [2][max_depth+1][row_bytes], or [2][Hkv][max_depth+1][row_bytes] when
+  // every head is staged at once
+  extern __shared__ __align__(16) uint8_t stage[];
   __shared__ int s_src[MEDUSA_MAX_HEADS + 1];
   __shared__ int s_ok;
   const int b = blockIdx.x;
@@ -47,8 +49,33 @@ __global__ void __launch_bounds__(kCompactThreads)
   if (!s_ok) return;
 
   const int vec_per_row = row_bytes / 16;
-  const int n_vec = (L + 1) * vec_per_row;
   uint4* sk = reinterpret_cast<uint4*>(stage);
+  if (heads_at_once > 1) {
+    // every kv head staged in one round trip: [Hkv][L+1][row] for K then V
+    const int n_vec = Hkv * (L + 1) * vec_per_row;
+    uint4* sv = sk + (size_t)Hkv * W * vec_per_row;
+    for (int e = tid; e < n_vec; e += kCompactThreads) {
+      const int c = e % vec_per_row;
+      const int j = (e / vec_per_row) % (L + 1);
+      const int h = e / (vec_per_row * (L + 1));
+      const size_t src = (((size_t)b * Hkv + h) * cap + s_src[j]) * row_bytes;
+      sk[e] = reinterpret_cast<const uint4*>(Kc + src)[c];
+      sv[e] = reinterpret_cast<const uint4*>(Vc + src)[c];
+    }
+    __syncthreads();
+    for (int e = tid; e < n_vec; e += kCompactThreads) {
+      const int c = e % vec_per_row;
+      const int j = (e / vec_per_row) % (L + 1);
+      const int h = e / (vec_per_row * (L + 1));
+      const size_t dst = (((size_t)b * Hkv + h) * cap + P + j) * row_bytes;
+      reinterpret_cast<uint4*>(Kc + dst)[c] = sk[e];
+      reinterpret_cast<uint4*>(Vc + dst)[c] = sv[e];
+    }
+    if (tid < W) compact_src[(size_t)b * W + tid] = tid <= L ? s_src[tid] : -1;
+    if (tid == 0) prefix_len[b] = P + L + 1;
+    return;
+  }
+  const int n_vec = (L + 1) * vec_per_row;
   uint4* sv = reinterpret_cast<uint4*>(stage + (size_t)W * row_bytes);
   for (int h = 0; h < Hkv; ++h) {
     const size_t head_base = ((size_t)b * Hkv + h) * cap;  // in rows
@@ -76,12 +103,13 @@ medusa_status_t kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefi
                            int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,
                            int32_t* status, cudaStream_t stream) {
   const int row_bytes = dh * (dt == MEDUSA_BF16 ? 2 : 4);
-  const size_t smem = 2 * (size_t)(max_depth + 1) * row_bytes;
-  if (smem > 48 * 1024)
+  const size_t per_head = 2 * (size_t)(max_depth + 1) * row_bytes;
+  if (per_head > 48 * 1024)
     return fail(MEDUSA_ERR_UNSUPPORTED, "kv_compact: (max_depth+1) * row too large");
-  kv_compact_kernel<<<B, kCompactThreads, smem, stream>>>(
+  const bool all_heads = per_head * Hkv <= 48 * 1024;
+  kv_compact_kernel<<<B, kCompactThreads, all_heads ? per_head * Hkv : per_head, stream>>>(
       static_cast<uint8_t*>(Kc), static_cast<uint8_t*>(Vc), row_bytes, prefix_len, accepted_nodes,
-      accept_len, Hkv, cap, max_depth, compact_src, status);
+      accept_len, Hkv, cap, max_depth, all_heads ? Hkv : 1, compact_src, status);
   return check_launch("kv_compact");
 }
 

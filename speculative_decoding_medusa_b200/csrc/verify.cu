@@ -24,9 +24,8 @@
 
 namespace medusa {
 
-constexpr int kVChunk = 8192;
-constexpr int kRowThreads = 256;
-constexpr int kPer = kVChunk / kRowThreads;  // 32 logits per thread
+constexpr int kVChunk = 4096;   // tokens per warp work item
+constexpr int kRowWarps = 8;    // work items per CTA
 
 struct RowPart {
   float maxz;
@@ -35,21 +34,47 @@ struct RowPart {
   float t;  // sum exp(z/T - maxz/T) * z/T
 };
 
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(p);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    v[2 * e] = __uint_as_float(w[e] << 16);
-    v[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+template <typename T>
+struct Elt;
+template <>
+struct Elt<__nv_bfloat16> {
+  static constexpr int kPerVec = 8;  // elements per 16-byte load
+  static constexpr uint32_t kNegInf = 0xFF80u;
+  __device__ static float get(const uint4& r, int e) {
+    const uint32_t w = (&r.x)[e >> 1];
+    return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
   }
-}
+  __device__ static uint4 load_scalar(const __nv_bfloat16* p, int n) {
+    uint16_t h[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) h[e] = e < n ? reinterpret_cast<const uint16_t*>(p)[e] : 0xFF80u;
+    uint4 r;
+    r.x = h[0] | (uint32_t(h[1]) << 16);
+    r.y = h[2] | (uint32_t(h[3]) << 16);
+    r.z = h[4] | (uint32_t(h[5]) << 16);
+    r.w = h[6] | (uint32_t(h[7]) << 16);
+    return r;
+  }
+};
+template <>
+struct Elt<float> {
+  static constexpr int kPerVec = 4;
+  __device__ static float get(const uint4& r, int e) { return __uint_as_float((&r.x)[e]); }
+  __device__ static uint4 load_scalar(const float* p, int n) {
+    uint4 r;
+    uint32_t* w = &r.x;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w[e] = e < n ? __float_as_uint(p[e]) : 0xFF800000u;
+    return r;
+  }
+};
 
-__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
-  const float4 a = *reinterpret_cast<const float4*>(p);
-  const float4 b = *reinterpret_cast<const float4*>(p + 4);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
 }
 
 template <typename T>
@@ -63,41 +88,43 @@ __device__ __forceinline__ float load1<float>(const float* p) {
   return *p;
 }
 
+// One warp per (row, 4096-token chunk): every lane issues all its 16-byte
+// loads at once, then the warp reduces with shuffles only.
 template <typename T, bool TYPICAL>
-__global__ void __launch_bounds__(kRowThreads)
-    verify_rows_kernel(const T* __restrict__ logits, int V, int n_chunks, float inv_T,
-                       RowPart* __restrict__ part, int32_t* status) {
-  const int c = blockIdx.x;
-  const size_t row = blockIdx.y;
+__global__ void __launch_bounds__(kRowWarps * 32)
+    verify_rows_kernel(const T* __restrict__ logits, int V, int n_chunks, long long n_items,
+                       float inv_T, RowPart* __restrict__ part, int32_t* status) {
+  using E = Elt<T>;
+  constexpr int EV = E::kPerVec;
+  constexpr int NL = kVChunk / (32 * EV);  // loads per lane
+  const int lane = threadIdx.x & 31;
+  const long long item = (long long)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  if (item >= n_items) return;  // whole warp
+  const long long row = item / n_chunks;
+  const int c = static_cast<int>(item - row * n_chunks);
   const T* base = logits + row * V;
   const int v0 = c * kVChunk;
-  const int tid = threadIdx.x;
-  float vals[kPer];
-  // contiguous runs of 8 per thread, coalesced across the block
-  const bool vec_ok = (V % 8) == 0;
+  const bool vec = (V % EV) == 0;
+  uint4 raw[NL];
 #pragma unroll
-  for (int r = 0; r < kPer / 8; ++r) {
-    const int e0 = v0 + (r * kRowThreads + tid) * 8;
-    float v8[8];
-    if (vec_ok && e0 + 8 <= V) {
-      load8(base + e0, v8);
+  for (int r = 0; r < NL; ++r) {
+    const int e0 = v0 + (r * 32 + lane) * EV;
+    if (vec && e0 + EV <= V) {
+      raw[r] = ld_stream16(base + e0);
     } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v8[e] = (e0 + e < V) ? load1<T>(base + e0 + e) : -INFINITY;
+      raw[r] = E::load_scalar(base + e0, e0 < V ? min(EV, V - e0) : 0);
     }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) vals[r * 8 + e] = v8[e];
   }
-  // best (largest, lowest index) of this thread; indices ascend within a run
+  // best (largest, lowest index) of this lane: indices ascend in (r, e) order
   float bv = -INFINITY;
   int bi = 0x7fffffff;
   bool nan = false;
 #pragma unroll
-  for (int r = 0; r < kPer / 8; ++r) {
-    const int e0 = v0 + (r * kRowThreads + tid) * 8;
+  for (int r = 0; r < NL; ++r) {
+    const int e0 = v0 + (r * 32 + lane) * EV;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float x = vals[r * 8 + e];
+    for (int e = 0; e < EV; ++e) {
+      const float x = E::get(raw[r], e);
       nan |= (x != x);
       if (e0 + e < V && better(x, e0 + e, bv, bi)) {
         bv = x;
@@ -106,10 +133,6 @@ __global__ void __launch_bounds__(kRowThreads)
     }
   }
   if (nan) report(status, MEDUSA_ERR_DEVICE_CHECK);
-  // block reduction of (bv, bi)
-  __shared__ float s_v[kRowThreads / 32];
-  __shared__ int s_i[kRowThreads / 32];
-  __shared__ float s_m;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -119,60 +142,35 @@ __global__ void __launch_bounds__(kRowThreads)
       bi = oi;
     }
   }
-  const int warp = tid >> 5, lane = tid & 31;
-  if (lane == 0) {
-    s_v[warp] = bv;
-    s_i[warp] = bi;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    float v = s_v[0];
-    int i = s_i[0];
-    for (int w = 1; w < kRowThreads / 32; ++w)
-      if (better(s_v[w], s_i[w], v, i)) {
-        v = s_v[w];
-        i = s_i[w];
-      }
-    s_m = v;
-    part[row * n_chunks + c].maxz = v;
-    part[row * n_chunks + c].idx = i;
-    if (!TYPICAL) {
-      part[row * n_chunks + c].s = 0.f;
-      part[row * n_chunks + c].t = 0.f;
-    }
-  }
-  if (!TYPICAL) return;
-  __syncthreads();
-  const float m = s_m * inv_T;
   float ss = 0.f, tt = 0.f;
+  if (TYPICAL) {
+    const float m = bv * inv_T;
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) {
-    if (vals[e] != -INFINITY) {
-      const float zt = vals[e] * inv_T;
-      const float w = expf(zt - m);
-      ss += w;
-      tt += w * zt;
+    for (int r = 0; r < NL; ++r) {
+#pragma unroll
+      for (int e = 0; e < EV; ++e) {
+        const float x = E::get(raw[r], e);
+        if (x != -INFINITY) {
+          const float zt = x * inv_T;
+          const float w = expf(zt - m);
+          ss += w;
+          tt += w * zt;
+        }
+      }
     }
-  }
-  __shared__ float s_s[kRowThreads / 32], s_t[kRowThreads / 32];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    tt += __shfl_xor_sync(0xffffffffu, tt, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      tt += __shfl_xor_sync(0xffffffffu, tt, o);
+    }
   }
   if (lane == 0) {
-    s_s[warp] = ss;
-    s_t[warp] = tt;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    float a = 0.f, bsum = 0.f;
-    for (int w = 0; w < kRowThreads / 32; ++w) {
-      a += s_s[w];
-      bsum += s_t[w];
-    }
-    part[row * n_chunks + c].s = a;
-    part[row * n_chunks + c].t = bsum;
+    RowPart rp;
+    rp.maxz = bv;
+    rp.idx = bi;
+    rp.s = ss;
+    rp.t = tt;
+    part[row * n_chunks + c] = rp;
   }
 }
 
@@ -214,6 +212,7 @@ __global__ void __launch_bounds__(MEDUSA_MAX_NODES)
     float bv = -INFINITY;
     int bi = 0x7fffffff;
     float M = -INFINITY;
+#pragma unroll 4
     for (int c = 0; c < n_chunks; ++c) {
       const RowPart q = rp[c];
       if (better(q.maxz, q.idx, bv, bi)) {
@@ -304,15 +303,16 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
   RowPart* part = static_cast<RowPart*>(ws);
   const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
   const float inv_T = typical ? 1.0f / temperature : 1.0f;
-  dim3 grid(n_chunks, B * N);
+  const long long n_items = (long long)B * N * n_chunks;
+  const unsigned grid = (unsigned)((n_items + kRowWarps - 1) / kRowWarps);
   if (dt == MEDUSA_BF16) {
     const __nv_bfloat16* lg = static_cast<const __nv_bfloat16*>(logits);
     if (typical)
-      verify_rows_kernel<__nv_bfloat16, true><<<grid, kRowThreads, 0, stream>>>(lg, V, n_chunks,
+      verify_rows_kernel<__nv_bfloat16, true><<<grid, kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items,
                                                                                  inv_T, part, status);
     else
-      verify_rows_kernel<__nv_bfloat16, false><<<grid, kRowThreads, 0, stream>>>(
-          lg, V, n_chunks, inv_T, part, status);
+      verify_rows_kernel<__nv_bfloat16, false><<<grid, kRowWarps * 32, 0, stream>>>(
+          lg, V, n_chunks, n_items, inv_T, part, status);
     medusa_status_t st = check_launch("verify_rows");
     if (st != MEDUSA_OK) return st;
     verify_path_kernel<__nv_bfloat16><<<B, MEDUSA_MAX_NODES, 0, stream>>>(
@@ -323,10 +323,10 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
   }
   const float* lg = static_cast<const float*>(logits);
   if (typical)
-    verify_rows_kernel<float, true><<<grid, kRowThreads, 0, stream>>>(lg, V, n_chunks, inv_T, part,
+    verify_rows_kernel<float, true><<<grid, kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T, part,
                                                                       status);
   else
-    verify_rows_kernel<float, false><<<grid, kRowThreads, 0, stream>>>(lg, V, n_chunks, inv_T,
+    verify_rows_kernel<float, false><<<grid, kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T,
                                                                        part, status);
   medusa_status_t st = check_launch("verify_rows");
   if (st != MEDUSA_OK) return st;
@@ -349,8 +349,8 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
 // ---------------------------------------------------------------------------
 namespace {
 
-// 4 MiB holds B * N * ceil(V / 8192) 16-byte row records up to 262144 records
-// (for example B = 32, N = 128, V = 128256).  Every GPU that loads the library
+// 4 MiB holds B * N * ceil(V / 4096) 16-byte row records up to 262144 records
+// (for example B = 32, N = 128, V = 128256 needs 131072).  Every GPU that loads the library
 // keeps this array until the process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) unsigned char g_verify_noalloc_scratch[kNoAllocScratchBytes];
@@ -370,7 +370,7 @@ extern "C" medusa_status_t medusa_verify_accept_noalloc(
   if (B >= 1 && V >= 1 && tree->n_nodes >= 1 &&
       medusa::verify_accept_workspace_size(B, tree->n_nodes, V) > kNoAllocScratchBytes)
     return medusa::fail(MEDUSA_ERR_WORKSPACE,
-                        "verify_accept_noalloc: B * n_nodes * ceil(V / 8192) * 16 bytes exceeds "
+                        "verify_accept_noalloc: B * n_nodes * ceil(V / 4096) * 16 bytes exceeds "
                         "the 4 MiB static scratch; use medusa_verify_accept with a workspace");
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
