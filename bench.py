@@ -213,7 +213,77 @@ def parse():
     ap.add_argument("--nodes", type=int, default=None, help="tree size override (long: 16/64/128)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--stage", choices=["all", "attention", "verify"], default="all",
+                    help="time one stage alone (profiling aid; prints a stage line, not the metric)")
     return ap.parse_args()
+
+
+def run_stage(args):
+    """One stage in a loop on the workload's inputs (for per-kernel timing
+    and profiling): tree attention or verify/accept."""
+    import speculative_decoding_medusa_b200 as M
+    from speculative_decoding_medusa_b200 import workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = W.WORKLOADS[args.workload]
+    N = args.nodes or w.N
+    if args.nodes:
+        w = W.scaled(w, N=N)
+    spec = W.tree_for(w, n_nodes=N)
+    tree = M.Tree.from_spec(spec, dev)
+    att = W.attention_inputs(w, seed=0, device=dev, n_nodes=N)
+    root = W.random_root_tokens(w, 0, device=dev)
+    topk = W.random_topk_ids(w, 0, device=dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+    cand = torch.empty(w.B, N, **i32)
+    pos = torch.empty(w.B, N, **i32)
+    mask = torch.empty(N, (N + 31) // 32, **i32)
+    retrieve = torch.empty(spec.n_leaves, spec.max_depth + 1, **i32)
+    status = M.new_status(dev)
+    M.medusa_tree_build(tree, root, topk, att["prefix_len"], cand, pos, mask, retrieve, status)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    if args.stage == "attention":
+        out = torch.empty(w.B, N, w.Hq, w.dh, dtype=dt, device=dev)
+        ws = M.workspace(M.medusa_tree_attention_workspace_size(
+            w.B, N, w.Hq, w.Hkv, w.dh, w.ctx_hi, M.MEDUSA_BF16 if dt == torch.bfloat16 else M.MEDUSA_F32), dev)
+        fn = lambda: M.medusa_tree_attention(att["q"], att["k_new"], att["v_new"], att["Kc"], att["Vc"],
+                                             att["prefix_len"], mask, w.ctx_hi, out, None, ws, status)
+        e = 2 if dt == torch.bfloat16 else 4
+        P = att["prefix_len"].tolist()
+        nbytes = (sum(P) * w.Hkv * w.dh * 2 + w.B * N * (2 * w.Hq + 4 * w.Hkv) * w.dh) * e
+        flops = 4.0 * w.Hq * w.dh * N * sum(p + N for p in P)
+    else:
+        torch.cuda.synchronize()
+        logits = W.verify_logits(w, spec, cand, seed=0, device=dev)
+        Wd = spec.max_depth + 1
+        outs = [torch.empty(w.B, **i32), torch.empty(w.B, Wd, **i32), torch.empty(w.B, Wd, **i32),
+                torch.empty(w.B, **i32)]
+        ws = M.workspace(M.medusa_verify_accept_workspace_size(w.B, N, w.V), dev)
+        mode = M.MEDUSA_ACCEPT_TYPICAL if w.accept == "typical" else M.MEDUSA_ACCEPT_GREEDY
+        fn = lambda: M.medusa_verify_accept(logits, cand, tree, *outs, mode, w.temperature, w.eps,
+                                            w.delta, ws, status)
+        nbytes = logits.numel() * logits.element_size()
+        flops = 0.0
+    for _ in range(max(args.warmup, 3)):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, int(status.item())
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    hbm, tflops, kind = _peaks()
+    line = {"stage": args.stage, "workload": args.workload, "n_nodes": N, "us_per_call": us,
+            "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / us / 1e3,
+            "hbm_frac": nbytes / us / 1e3 / hbm, "tflops": flops / us / 1e6,
+            "tensor_frac": flops / us / 1e6 / tflops if flops else None, "peaks": kind}
+    print(json.dumps(line))
+    return 0
 
 
 def run_reference(args):
@@ -250,6 +320,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.stage != "all":
+        return run_stage(args)
 
     import speculative_decoding_medusa_b200 as M
     from speculative_decoding_medusa_b200 import workloads as W

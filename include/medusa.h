@@ -204,13 +204,13 @@ MEDUSA_API medusa_status_t medusa_tree_build(const medusa_tree_t* tree, const in
  *   prefix_len[b] + N <= cap; anc_mask from medusa_tree_build.
  * Output (device): out [B, N, Hq, dh] of dtype out_dt (bf16 or f32).
  * max_prefix: host-side upper bound on every prefix_len[b]; sizes the launch.
- * Workspace: medusa_tree_attention_workspace_size(...) bytes (split-KV
- *   partial results), 256-byte aligned.
+ * Workspace: medusa_tree_attention_workspace_size(...) bytes (partial
+ *   results of key ranges, merged at the end), 256-byte aligned.
  * Precision: bf16 q/k/v, fp32 scores, fp32 softmax statistics; the softmax
  *   weights enter the value product as two bf16 terms (hi + lo).
  *   dt = MEDUSA_F32 runs an fp32 CUDA-core path.
- * Limits: Hq % Hkv == 0; bf16: dh in {64, 128}, pointers 16-byte aligned;
- *   f32: dh <= 256 and dh % 32 == 0; N <= MEDUSA_MAX_NODES.
+ * Limits: Hq % Hkv == 0; bf16: dh in {64, 128}, B <= 256, pointers 16-byte
+ *   aligned; f32: dh <= 256 and dh % 32 == 0; N <= MEDUSA_MAX_NODES.
  * ---------------------------------------------------------------------- */
 MEDUSA_API size_t medusa_tree_attention_workspace_size(int B, int N, int Hq, int Hkv, int dh,
                                             int max_prefix, medusa_dtype_t dt);

@@ -138,6 +138,7 @@ medusa_status_t medusa_tree_attention(const void* q, const void* k_new, const vo
     return fail(MEDUSA_ERR_SHAPE, "tree_attention: cache too large");
   if (dt == MEDUSA_BF16) {
     if (dh != 64 && dh != 128) return fail(MEDUSA_ERR_SHAPE, "tree_attention: bf16 dh must be 64 or 128");
+    if (B > 256) return fail(MEDUSA_ERR_SHAPE, "tree_attention: bf16 path takes at most 256 sequences");
     if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(Kc) ||
         !aligned16(Vc) || !aligned16(out))
       return fail(MEDUSA_ERR_ALIGNMENT, "tree_attention: pointers must be 16-byte aligned");

@@ -2,6 +2,7 @@
 // per-stage launchers.  Every launcher assumes its arguments were validated.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -16,6 +17,13 @@ medusa_status_t fail(medusa_status_t code, const char* msg);
 medusa_status_t check_launch(const char* what);
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// bf16 tensor of `rank` dims (dims[0] contiguous; byte_strides[i] is the
+// stride of dims[i+1]), tile `box`, 128-byte swizzle, zero fill outside
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* byte_strides, const uint32_t* box);
+// multiprocessors of the current device
+int device_sm_count();
 
 size_t heads_topk_workspace_size(int B, int d, int V, int K, int kmax, medusa_dtype_t dt);
 medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const void* W2,

@@ -5,15 +5,21 @@
 // candidate tokens are appended to the input at once; a mask lets each one see
 // only its ancestors, so one forward pass scores every branch.
 //
-// bf16 path: split-KV.  For each (sequence b, kv head) the N*G query rows
-// (G = Hq/Hkv grouped query heads per kv head) form tiles of 64 rows; the
-// prefix is cut into chunks of `chunk` keys, plus one more split for the N
-// tree keys (read from k_new/v_new, masked by the ancestor bitmask).  Each CTA
-// keeps an online softmax and writes a normalised partial output and its
-// log2-sum-exp; a combine kernel merges the splits.  The tree split with query
-// tile 0 also writes the tree K/V into cache slots P + i.
-// QK^T and PV run on mma.sync m16n8k16 (bf16, fp32 accumulate); the softmax
-// weights enter PV as two bf16 terms (hi + lo) to keep ~16 mantissa bits.
+// bf16 path (tcgen05): split-KV.  A CTA takes 256 query rows of one (sequence,
+// kv head) - the N nodes x G grouped query heads, as two M = 128 tiles - and
+// one split of the keys: a chunk of the cached prefix, or the N tree keys (read
+// from k_new/v_new and masked by the ancestor bitmask).  Roles:
+//   warp 0      TMA producer: 64-key K and V tiles into a 3-stage ring;
+//   warp 1      MMA issuer: S = Q K^T into TMEM (double-buffered per M tile),
+//               then O += P V with P = P_hi + P_lo (two bf16 terms) from
+//               shared memory and V as an M/N-major operand;
+//   warps 2..9  two softmax warpgroups, one query row per thread: the row's
+//               scores come out of TMEM, max and sum stay in the thread,
+//               O is rescaled in TMEM only when the row maximum grows by more
+//               than 2^8 (the stale maximum cancels in the final O / l).
+// Each CTA writes its normalised partial output and log2-sum-exp; a combine
+// kernel merges the splits.  The tree split of query group 0 also writes the
+// tree K/V into cache slots P + i.
 //
 // fp32 path: one warp per query row on CUDA cores (small shapes).
 #include <cuda_bf16.h>
@@ -26,9 +32,22 @@
 
 namespace medusa {
 
-constexpr int kBM = 64;  // query rows per CTA (4 warps x 16)
-constexpr int kBN = 64;  // keys per tile
-constexpr int kAttnThreads = 128;
+constexpr int kAttnBN = 64;          // keys per tile
+constexpr int kAttnMT = 128;         // query rows per M tile (UMMA M)
+constexpr int kAttnRows = 256;       // query rows per segment (two M tiles)
+constexpr int kAttnStages = 3;       // K/V ring depth
+constexpr int kAttnThreads = 320;    // producer, MMA, two softmax warpgroups
+constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold, log2 units
+constexpr uint32_t kAttnTmemCols = 512;
+constexpr int kAttnMaxB = 256;       // sequences per call (schedule table in shared memory)
+constexpr int kAttnMinTiles = 16;    // smallest tile range a CTA takes
+
+// 2^x with the SFU instruction (ex2.approx; relative error about 2^-22, -inf -> 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 struct AttnParams {
   const __nv_bfloat16* q;
@@ -38,329 +57,561 @@ struct AttnParams {
   __nv_bfloat16* Vc;
   const int32_t* prefix_len;
   const uint32_t* anc_mask;
-  float* o_part;   // [B*Hkv, n_qt, S, kBM, DH]
-  float* lse_part; // [B*Hkv, n_qt, S, kBM]
-  int B, N, Hq, Hkv, G, R, n_qt, S, chunk, cap, max_prefix, words;
+  float* o_part;    // [n_seg, slots, 256, DH]
+  float* lse_part;  // [n_seg, slots, 256]
+  int B, N, Hq, Hkv, G, R, n_qg, T_tree, slots, cap, max_prefix, words, grid;
   float scale_log2;
   int32_t* status;
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                          uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// split x into bf16 hi + bf16 lo (x ~= hi + lo)
-__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-  const float r0 = x0 - __low2float(h);
-  const float r1 = x1 - __high2float(h);
-  hi = *reinterpret_cast<uint32_t*>(&h);
-  lo = pack_bf16(r0, r1);
-}
-
-// byte offset of 16-byte chunk `c` of row `r` in a [rows][DH] bf16 tile whose
-// chunks are XOR-swizzled by the row (conflict-free ldmatrix)
 template <int DH>
-__device__ __forceinline__ uint32_t swz(int r, int c) {
-  return static_cast<uint32_t>(r * (DH * 2) + ((c ^ (r & 7)) << 4));
+struct AttnSmem {
+  static constexpr int kPanels = DH / 64;                  // 64-element (128 B) panels
+  static constexpr int kQBytes = kAttnMT * DH * 2;         // one M tile of Q
+  static constexpr int kKVBytes = kAttnBN * DH * 2;        // one K (or V) tile
+  static constexpr int kPBytes = kAttnMT * kAttnBN * 2;    // one of P_hi / P_lo
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + 2 * kQBytes;
+  static constexpr int kVOff = kKOff + kAttnStages * kKVBytes;
+  static constexpr int kPOff = kVOff + kAttnStages * kKVBytes;
+  static constexpr int kBarOff = kPOff + 4 * kPBytes;
+  // kv_full[S], kv_empty[S], q_full[2], s_full[2][2], s_free[2][2], p_full[2],
+  // p_empty[2], drain
+  static constexpr int kNumBars = 2 * kAttnStages + 2 + 4 + 4 + 2 + 2 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kCumOff = kMiscOff + 16;            // int cumT[kAttnMaxB + 1]
+  static constexpr int kBytes = kCumOff + (kAttnMaxB + 1) * 4;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+// ----------------------------------------------------------------------------
+// Schedule.  Segment = (sequence b, kv head, query group of 256 rows); its
+// tiles are the ceil(P_b / 64) prefix tiles followed by the ceil(N / 64) tree
+// tiles.  Segments are laid end to end (b-major) and every CTA takes an equal
+// contiguous range of `per` tiles; a range cut at segment ends gives pieces,
+// each written as one partial result (slot k = CTA - first CTA of the segment).
+// ----------------------------------------------------------------------------
+struct TileInfo {
+  int b, kvh, qg, lt, tpre, ntiles, seg, slot, P, n_mt;
+  bool first, last;
+};
+
+__device__ __forceinline__ void decode_tile(int t, const int* cumT, const AttnParams& p, int per,
+                                            int t0, int t1, TileInfo& x) {
+  int lo = 0, hi = p.B;  // cumT[lo] <= t < cumT[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cumT[mid] <= t) lo = mid;
+    else hi = mid;
+  }
+  x.b = lo;
+  x.P = p.prefix_len[lo];
+  x.tpre = (x.P + kAttnBN - 1) / kAttnBN;
+  x.ntiles = x.tpre + p.T_tree;
+  const int rem = t - cumT[lo];
+  const int sib = rem / x.ntiles;
+  x.lt = rem - sib * x.ntiles;
+  x.kvh = sib / p.n_qg;
+  x.qg = sib - x.kvh * p.n_qg;
+  x.seg = (x.b * p.Hkv + x.kvh) * p.n_qg + x.qg;
+  const int seg_start = t - x.lt;
+  x.slot = (t0 / per) - seg_start / per;
+  x.first = (t == t0) || (x.lt == 0);
+  x.last = (t == t1 - 1) || (x.lt == x.ntiles - 1);
+  x.n_mt = min(2, (p.R - x.qg * kAttnRows + kAttnMT - 1) / kAttnMT);
+}
+
+// cumT[b] = tiles of all segments of sequences < b; returns false if some
+// prefix length is out of range.  Called by one full warp.
+__device__ __forceinline__ bool build_schedule(const AttnParams& p, int* cumT) {
+  const int lane = threadIdx.x & 31;
+  int run = 0;
+  bool ok = true;
+  if (lane == 0) cumT[0] = 0;
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int b = b0 + lane;
+    int v = 0;
+    if (b < p.B) {
+      const int P = p.prefix_len[b];
+      if (P < 0 || P > p.max_prefix || P + p.N > p.cap) ok = false;
+      v = ((max(P, 0) + kAttnBN - 1) / kAttnBN + p.T_tree) * p.Hkv * p.n_qg;
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    if (b < p.B) cumT[b + 1] = run + v;
+    run += __shfl_sync(0xffffffffu, v, 31);
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ int tiles_per_cta(int total, int grid) {
+  const int per = (total + grid - 1) / grid;
+  return per < kAttnMinTiles ? kAttnMinTiles : per;
 }
 
 template <int DH>
-__global__ void __launch_bounds__(kAttnThreads, 2) tree_attn_bf16_kernel(AttnParams p) {
-  constexpr int CH = DH / 8;  // 16-byte chunks per row
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kBM * DH * 2;
-  uint8_t* sV = sK + 2 * kBN * DH * 2;
-  uint32_t* sMask = reinterpret_cast<uint32_t*>(sV + 2 * kBN * DH * 2);  // [kBM][8]
-
-  const int s = blockIdx.x;
-  const int qt = blockIdx.y;
-  const int bh = blockIdx.z;
-  const int b = bh / p.Hkv;
-  const int kvh = bh - b * p.Hkv;
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
-
-  const int P = p.prefix_len[b];
-  if (P < 0 || P > p.max_prefix || P + p.N > p.cap) {
-    if (tid == 0) report(p.status, MEDUSA_ERR_DEVICE_CHECK);
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmKn,
+                        const __grid_constant__ CUtensorMap tmVn, AttnParams p) {
+  using L = AttnSmem<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  int* cumT = reinterpret_cast<int*>(smem + L::kCumOff);
+  volatile int* sched_ok = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp == 0) {
+    const bool ok = build_schedule(p, cumT);
+    if (lane == 0) *sched_ok = ok ? 1 : 0;
+  }
+  __syncthreads();
+  if (!*sched_ok) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, MEDUSA_ERR_DEVICE_CHECK);
     return;
   }
-  const int n_pre = (P + p.chunk - 1) / p.chunk;
-  if (s > n_pre) return;
-  const bool tree_split = (s == n_pre);
-  const int key0 = tree_split ? 0 : s * p.chunk;
-  const int key_end = tree_split ? p.N : min(P, key0 + p.chunk);
-  const int n_tiles = (key_end - key0 + kBN - 1) / kBN;
+  const int total = cumT[p.B];
+  const int per = tiles_per_cta(total, gridDim.x);
+  const int t0 = blockIdx.x * per;
+  const int t1 = min(t0 + per, total);
+  if (t0 >= total) return;
+  const int n = t1 - t0;
 
-  const size_t kv_head_base = ((size_t)b * p.Hkv + kvh) * p.cap;  // in rows of DH
-  // ---- tree split, tile 0: write the tree K/V into the cache ----
-  if (tree_split && qt == 0) {
-    for (int e = tid; e < p.N * CH; e += kAttnThreads) {
-      const int j = e / CH, c = e - j * CH;
-      const size_t src = (((size_t)b * p.N + j) * p.Hkv + kvh) * DH + c * 8;
-      const size_t dst = (kv_head_base + P + j) * DH + c * 8;
-      *reinterpret_cast<uint4*>(p.Kc + dst) = *reinterpret_cast<const uint4*>(p.k_new + src);
-      *reinterpret_cast<uint4*>(p.Vc + dst) = *reinterpret_cast<const uint4*>(p.v_new + src);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + kAttnStages;
+  uint64_t* q_full = bars + 2 * kAttnStages;
+  uint64_t* s_full = q_full + 2;   // [m * 2 + buf]
+  uint64_t* s_free = s_full + 4;   // [m * 2 + buf]
+  uint64_t* p_full = s_free + 4;   // [m]
+  uint64_t* p_empty = p_full + 2;  // [m]
+  uint64_t* drain = p_empty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kAttnStages; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
-  }
-
-  // ---- Q tile (rows r = qt*kBM + row; node r / G, head kvh*G + r % G) ----
-  const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-  for (int e = tid; e < kBM * CH; e += kAttnThreads) {
-    const int row = e / CH, c = e - row * CH;
-    const int r = qt * kBM + row;
-    const bool valid = r < p.R;
-    const int node = valid ? r / p.G : 0;
-    const int g = valid ? r - node * p.G : 0;
-    const __nv_bfloat16* src = p.q + (((size_t)b * p.N + node) * p.Hq + kvh * p.G + g) * DH + c * 8;
-    cp_async16(sQa + swz<DH>(row, c), valid ? src : p.q, valid);
-  }
-  if (tree_split) {
-    for (int e = tid; e < kBM * 8; e += kAttnThreads) {
-      const int row = e >> 3, w = e & 7;
-      const int r = qt * kBM + row;
-      uint32_t m = 0xffffffffu;
-      if (r < p.R && w < p.words) m = p.anc_mask[(size_t)(r / p.G) * p.words + w];
-      sMask[e] = m;
+    for (int m = 0; m < 2; ++m) {
+      mbar_init(&q_full[m], 128);
+      mbar_init(&p_full[m], 128);
+      mbar_init(&p_empty[m], 1);
+      for (int bf = 0; bf < 2; ++bf) {
+        mbar_init(&s_full[m * 2 + bf], 1);
+        mbar_init(&s_free[m * 2 + bf], 128);
+      }
     }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kAttnTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint32_t tmem_o = tmem_base;             // O[m]: columns m*DH .. m*DH+DH-1
+  const uint32_t tmem_s = tmem_base + 2 * DH;    // S[m][buf]: 64 columns each
 
-  auto load_tile = [&](int t, int stage) {
-    const int k0 = key0 + t * kBN;
-    for (int e = tid; e < kBN * CH; e += kAttnThreads) {
-      const int row = e / CH, c = e - row * CH;
-      const int key = k0 + row;
-      const bool valid = key < key_end;
-      const __nv_bfloat16 *ks, *vs;
-      if (tree_split) {
-        const size_t off = (((size_t)b * p.N + key) * p.Hkv + kvh) * DH + c * 8;
-        ks = valid ? p.k_new + off : p.k_new;
-        vs = valid ? p.v_new + off : p.v_new;
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmKn);
+      tma_prefetch_desc(&tmVn);
+      const uint64_t pol = p.n_qg > 1 ? l2_policy_evict_last() : l2_policy_evict_first();
+      int j = 0;
+      for (; j < n; ++j) {
+        TileInfo x;
+        decode_tile(t0 + j, cumT, p, per, t0, t1, x);
+        const int st = j % kAttnStages;
+        if (!mbar_wait_bounded(&kv_empty[st], ((j / kAttnStages) & 1) ^ 1u, abort_flag, p.status))
+          break;
+        mbar_arrive_expect_tx(&kv_full[st], 2 * L::kKVBytes);
+        uint8_t* kdst = smem + L::kKOff + st * L::kKVBytes;
+        uint8_t* vdst = smem + L::kVOff + st * L::kKVBytes;
+        const int bh = x.b * p.Hkv + x.kvh;
+#pragma unroll
+        for (int pn = 0; pn < L::kPanels; ++pn) {
+          if (x.lt < x.tpre) {
+            const int key = x.lt * kAttnBN;
+            tma_load_3d(kdst + pn * kAttnBN * 128, &tmK, &kv_full[st], pn * 64, key, bh, pol);
+            tma_load_3d(vdst + pn * kAttnBN * 128, &tmV, &kv_full[st], pn * 64, key, bh, pol);
+          } else {
+            const int node = (x.lt - x.tpre) * kAttnBN;
+            tma_load_4d(kdst + pn * kAttnBN * 128, &tmKn, &kv_full[st], pn * 64, x.kvh, node, x.b,
+                        pol);
+            tma_load_4d(vdst + pn * kAttnBN * 128, &tmVn, &kv_full[st], pn * 64, x.kvh, node, x.b,
+                        pol);
+          }
+        }
+      }
+      const int first = j > kAttnStages ? j - kAttnStages : 0;
+      for (int x = first; x < j; ++x) {
+        int dummy_abort = 0;
+        mbar_wait_bounded(&kv_full[x % kAttnStages], (x / kAttnStages) & 1, &dummy_abort, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = umma_idesc_bf16(kAttnMT, kAttnBN, 0);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(kAttnMT, DH, 1);
+      int tq[2] = {0, 0}, pq[2] = {0, 0}, tp[2] = {0, 0};
+      auto issue_qk = [&](int j) -> bool {
+        TileInfo x;
+        decode_tile(t0 + j, cumT, p, per, t0, t1, x);
+        const int st = j % kAttnStages;
+        if (!mbar_wait_bounded(&kv_full[st], (j / kAttnStages) & 1, abort_flag, p.status))
+          return false;
+        const uint32_t kaddr = smem_u32(smem + L::kKOff + st * L::kKVBytes);
+        for (int m = 0; m < x.n_mt; ++m) {
+          if (x.first) {
+            if (!mbar_wait_bounded(&q_full[m], pq[m] & 1, abort_flag, p.status)) return false;
+            ++pq[m];
+          }
+          const int bf = tq[m] & 1;
+          if (!mbar_wait_bounded(&s_free[m * 2 + bf], ((tq[m] >> 1) & 1) ^ 1u, abort_flag,
+                                 p.status))
+            return false;
+          tc_fence_after();
+          const uint32_t qaddr = smem_u32(smem + L::kQOff + m * L::kQBytes);
+          const uint32_t d = tmem_s + (m * 2 + bf) * kAttnBN;
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            const uint32_t a = qaddr + (kk >> 2) * (kAttnMT * 128) + (kk & 3) * 32;
+            const uint32_t bb = kaddr + (kk >> 2) * (kAttnBN * 128) + (kk & 3) * 32;
+            umma_bf16(d, umma_desc_sw128(a), umma_desc_sw128(bb), idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[m * 2 + bf]);
+          ++tq[m];
+        }
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        TileInfo x;
+        decode_tile(t0 + j, cumT, p, per, t0, t1, x);
+        const int st = j % kAttnStages;
+        const uint32_t vaddr = smem_u32(smem + L::kVOff + st * L::kKVBytes);
+        for (int m = 0; m < x.n_mt; ++m) {
+          if (!mbar_wait_bounded(&p_full[m], tp[m] & 1, abort_flag, p.status)) return false;
+          tc_fence_after();
+          const uint32_t d = tmem_o + m * DH;
+#pragma unroll
+          for (int hl = 0; hl < 2; ++hl) {
+            const uint32_t paddr = smem_u32(smem + L::kPOff + (m * 2 + hl) * L::kPBytes);
+#pragma unroll
+            for (int kk = 0; kk < kAttnBN / 16; ++kk) {
+              // P: K-major, 16 keys = 32 bytes along the swizzled row.
+              // V: M/N-major, 16 keys = two 8-row groups of 1024 bytes; the
+              // second 64-element head-dimension panel sits one tile-panel on.
+              umma_bf16(d, umma_desc_sw128(paddr + kk * 32),
+                        umma_desc_sw128_lbo(vaddr + kk * 16 * 128, kAttnBN * 128, 1024), idesc_pv,
+                        (!x.first || hl > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&p_empty[m]);
+          ++tp[m];
+        }
+        umma_commit(&kv_empty[st]);
+        return true;
+      };
+      // order: QK(0), QK(1), then PV(j) followed by QK(j+2), so that PV(j)
+      // never waits for a K/V tile that is still loading
+      bool ok = issue_qk(0);
+      if (ok && n > 1) ok = issue_qk(1);
+      for (int j = 0; ok && j < n; ++j) {
+        ok = issue_pv(j);
+        if (ok && j + 2 < n) ok = issue_qk(j + 2);
+      }
+      umma_commit(drain);
+      int dummy_abort = 0;
+      mbar_wait_bounded(drain, 0, &dummy_abort, p.status);
+    }
+  } else {
+    // ---------------- softmax warpgroups ----------------
+    const int m = (warp - 2) >> 2;
+    const int quad = warp & 3;
+    const int rl = quad * 32 + lane;  // row within the M tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    uint8_t* qtile = smem + L::kQOff + m * L::kQBytes;
+    uint8_t* phi = smem + L::kPOff + (m * 2 + 0) * L::kPBytes + rl * 128;
+    uint8_t* plo = smem + L::kPOff + (m * 2 + 1) * L::kPBytes + rl * 128;
+
+    // Q rows of a segment into the swizzled K-major tile (zeros past R)
+    auto load_q = [&](const TileInfo& x) {
+      const int r = x.qg * kAttnRows + m * kAttnMT + rl;
+      const bool valid = r < p.R;
+      const int node = valid ? r / p.G : 0;
+      const int g = valid ? r - node * p.G : 0;
+      const uint4* qsrc = reinterpret_cast<const uint4*>(
+          p.q + (((size_t)x.b * p.N + node) * p.Hq + x.kvh * p.G + g) * DH);
+#pragma unroll
+      for (int c = 0; c < DH / 8; ++c) {
+        const uint4 v = valid ? qsrc[c] : make_uint4(0u, 0u, 0u, 0u);
+        const int pn = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4*>(qtile + pn * (kAttnMT * 128) + rl * 128 + ((cc ^ (rl & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&q_full[m]);
+    };
+
+    int tcount = 0;
+    bool q_ready = false;
+    bool ok = true;
+    float m_used = -INFINITY, l_run = 0.f;
+    uint32_t mw[8];
+    int jj = 0;
+    for (int j = 0; ok && j < n; ++j) {
+      TileInfo x;
+      decode_tile(t0 + j, cumT, p, per, t0, t1, x);
+      if (m >= x.n_mt) continue;
+      const int r = x.qg * kAttnRows + m * kAttnMT + rl;
+      const bool valid = r < p.R;
+      if (x.first) {
+        if (!q_ready) load_q(x);
+        q_ready = false;
+        const int node = valid ? r / p.G : 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+          mw[w] = (valid && w < p.words) ? p.anc_mask[(size_t)node * p.words + w] : 0xffffffffu;
+        m_used = -INFINITY;
+        l_run = 0.f;
+        jj = 0;
+      }
+      if (m == 0 && x.lt == x.tpre && x.qg == 0) {
+        // first tree tile of (b, kvh): the tree K/V into cache slots P + i
+        constexpr int CH = DH / 8;
+        const size_t kv_head_base = ((size_t)x.b * p.Hkv + x.kvh) * p.cap;
+        for (int e = rl; e < p.N * CH; e += 128) {
+          const int jn = e / CH, c = e - jn * CH;
+          const size_t src = (((size_t)x.b * p.N + jn) * p.Hkv + x.kvh) * DH + c * 8;
+          const size_t dst = (kv_head_base + x.P + jn) * DH + c * 8;
+          *reinterpret_cast<uint4*>(p.Kc + dst) = *reinterpret_cast<const uint4*>(p.k_new + src);
+          *reinterpret_cast<uint4*>(p.Vc + dst) = *reinterpret_cast<const uint4*>(p.v_new + src);
+        }
+      }
+      const int bf = tcount & 1;
+      if (!mbar_wait_bounded(&s_full[m * 2 + bf], (tcount >> 1) & 1, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[kAttnBN];
+      {
+        uint32_t r0[32], r1[32];
+        const uint32_t ta = tmem_s + lane_off + (m * 2 + bf) * kAttnBN;
+        tmem_ld32_raw(ta, r0);
+        tmem_ld32_raw(ta + 32, r1);
+        tmem_ld_wait();
+        tmem_regs_after_wait(r0);
+        tmem_regs_after_wait(r1);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          sv[c] = __uint_as_float(r0[c]);
+          sv[32 + c] = __uint_as_float(r1[c]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[m * 2 + bf]);
+      if (x.last && j + 1 < n) {
+        // every QK of this piece is done: load the next piece's Q now, so the
+        // MMA warp can run ahead into it
+        TileInfo y;
+        decode_tile(t0 + j + 1, cumT, p, per, t0, t1, y);
+        if (m < y.n_mt) {
+          load_q(y);
+          q_ready = true;
+        }
+      }
+      const bool tree_tile = x.lt >= x.tpre;
+      const int kbase = tree_tile ? (x.lt - x.tpre) * kAttnBN : x.lt * kAttnBN;
+      const int key_end = tree_tile ? p.N : x.P;
+      if (m == 0 && !tree_tile && kbase + kAttnBN > key_end) {
+        // V rows past the prefix end hold whatever the cache holds there;
+        // their weights are zero, but 0 * NaN is not, so clear them (the
+        // tile has landed: its scores were computed from the same stage)
+        uint8_t* vt = smem + L::kVOff + (j % kAttnStages) * L::kKVBytes;
+        const int from = key_end - kbase;
+        const int n16 = (kAttnBN - from) * 8 * L::kPanels;
+        for (int e = rl; e < n16; e += 128) {
+          const int pn = e / ((kAttnBN - from) * 8);
+          const int rem = e - pn * ((kAttnBN - from) * 8);
+          const int row = from + (rem >> 3);
+          *reinterpret_cast<uint4*>(vt + pn * (kAttnBN * 128) + row * 128 + ((rem & 7) << 4)) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      // row maximum of the raw scores (the scale is positive); full prefix
+      // tiles need no mask
+      float mx = -INFINITY;
+      if (!tree_tile && kbase + kAttnBN <= key_end) {
+#pragma unroll
+        for (int c = 0; c < kAttnBN; ++c) mx = fmaxf(mx, sv[c]);
       } else {
-        const size_t off = (kv_head_base + key) * DH + c * 8;
-        ks = valid ? p.Kc + off : p.Kc;
-        vs = valid ? p.Vc + off : p.Vc;
+        // the tile's two mask words, picked without dynamic register indexing
+        uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
+        if (tree_tile) {
+          const int tw = 2 * (x.lt - x.tpre);
+#pragma unroll
+          for (int w = 0; w < 8; ++w) {
+            if (w == tw) w0 = mw[w];
+            if (w == tw + 1) w1 = mw[w];
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < kAttnBN; ++c) {
+          const uint32_t word = c < 32 ? w0 : w1;
+          const bool vis = (kbase + c < key_end) && ((word >> (c & 31)) & 1u);
+          sv[c] = vis ? sv[c] : -INFINITY;
+          mx = fmaxf(mx, sv[c]);
+        }
       }
-      const uint32_t so = stage * kBN * DH * 2 + swz<DH>(row, c);
-      cp_async16(sKa + so, ks, valid);
-      cp_async16(sVa + so, vs, valid);
-    }
-  };
-
-  load_tile(0, 0);
-  cp_async_commit();  // group 0: Q + tile 0
-
-  // per-thread state: rows r_lo = 16*warp + lane/4 and r_hi = r_lo + 8
-  float o[DH / 8][4];
-#pragma unroll
-  for (int n = 0; n < DH / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
-  uint32_t qf[DH / 16][4];
-  const int row_lo = warp * 16 + (lane >> 2);
-
-  for (int t = 0; t < n_tiles; ++t) {
-    if (t + 1 < n_tiles) load_tile(t + 1, (t + 1) & 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    if (t == 0) {
-#pragma unroll
-      for (int kk = 0; kk < DH / 16; ++kk) {
-        const int row = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int c = 2 * kk + (lane >> 4);
-        ldsm_x4(sQa + swz<DH>(row, c), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+      mx *= p.scale_log2;
+      float corr = 1.f;
+      bool resc = false;
+      if (jj == 0) {
+        m_used = mx;
+      } else if (mx > m_used + kRescaleLog2) {
+        corr = exp2f(m_used - mx);
+        m_used = mx;
+        resc = true;
       }
-    }
-    const uint32_t kst = sKa + (t & 1) * kBN * DH * 2;
-    const uint32_t vst = sVa + (t & 1) * kBN * DH * 2;
-
-    // S = Q K^T : 16 rows x 64 keys per warp
-    float sc[kBN / 8][4];
+      const float nbase = m_used == -INFINITY ? 0.f : -m_used;
+      float sum = 0.f;
 #pragma unroll
-    for (int n = 0; n < kBN / 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < DH / 16; ++kk) {
-#pragma unroll
-      for (int np = 0; np < kBN / 16; ++np) {
-        uint32_t b0, b1, b2, b3;
-        const int key = np * 16 + (lane & 7) + (lane >> 4) * 8;
-        const int c = 2 * kk + ((lane >> 3) & 1);
-        ldsm_x4(kst + swz<DH>(key, c), b0, b1, b2, b3);
-        mma_bf16(sc[2 * np], qf[kk], b0, b1);
-        mma_bf16(sc[2 * np + 1], qf[kk], b2, b3);
+      for (int c = 0; c < kAttnBN; ++c) {
+        sv[c] = ex2_approx(fmaf(sv[c], p.scale_log2, nbase));
+        sum += sv[c];
       }
-    }
-
-    // scale, mask, row max
-    const int kbase = key0 + t * kBN;
-    float mx_lo = -INFINITY, mx_hi = -INFINITY;
-#pragma unroll
-    for (int n = 0; n < kBN / 8; ++n) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kl = n * 8 + (lane & 3) * 2 + (e & 1);  // key within tile
-        const int key = kbase + kl;
-        const int row = row_lo + (e >> 1) * 8;
-        bool vis = key < key_end;
-        if (tree_split && vis) vis = (sMask[row * 8 + (key >> 5)] >> (key & 31)) & 1u;
-        const float v = vis ? sc[n][e] * p.scale_log2 : -INFINITY;
-        sc[n][e] = v;
-        if (e < 2) mx_lo = fmaxf(mx_lo, v);
-        else mx_hi = fmaxf(mx_hi, v);
+      l_run = l_run * corr + sum;
+      // PV of the previous tile must be done: P buffer free, O stable
+      if (!mbar_wait_bounded(&p_empty[m], (tcount & 1) ^ 1u, abort_flag, p.status)) {
+        ok = false;
+        break;
       }
-    }
-    mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
-    mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
-    mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
-    mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
-    const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
-    const float base_lo = mn_lo == -INFINITY ? 0.f : mn_lo;
-    const float base_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
-    const float corr_lo = exp2f(m_lo - base_lo), corr_hi = exp2f(m_hi - base_hi);
-    m_lo = mn_lo;
-    m_hi = mn_hi;
-    float sum_lo = 0.f, sum_hi = 0.f;
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+        for (int ch = 0; ch < DH / 32; ++ch) {
+          float o[32];
+          const uint32_t ta = tmem_o + lane_off + m * DH + ch * 32;
+          tmem_ld32(ta, o);
 #pragma unroll
-    for (int n = 0; n < kBN / 8; ++n) {
-      sc[n][0] = exp2f(sc[n][0] - base_lo);
-      sc[n][1] = exp2f(sc[n][1] - base_lo);
-      sc[n][2] = exp2f(sc[n][2] - base_hi);
-      sc[n][3] = exp2f(sc[n][3] - base_hi);
-      sum_lo += sc[n][0] + sc[n][1];
-      sum_hi += sc[n][2] + sc[n][3];
-    }
-    l_lo = l_lo * corr_lo + sum_lo;  // quad-partial sums; reduced at the end
-    l_hi = l_hi * corr_hi + sum_hi;
-#pragma unroll
-    for (int n = 0; n < DH / 8; ++n) {
-      o[n][0] *= corr_lo;
-      o[n][1] *= corr_lo;
-      o[n][2] *= corr_hi;
-      o[n][3] *= corr_hi;
-    }
-
-    // O += P V with P = P_hi + P_lo
-#pragma unroll
-    for (int kk = 0; kk < kBN / 16; ++kk) {
-      uint32_t ah[4], al[4];
-      split_pair(sc[2 * kk][0], sc[2 * kk][1], ah[0], al[0]);
-      split_pair(sc[2 * kk][2], sc[2 * kk][3], ah[1], al[1]);
-      split_pair(sc[2 * kk + 1][0], sc[2 * kk + 1][1], ah[2], al[2]);
-      split_pair(sc[2 * kk + 1][2], sc[2 * kk + 1][3], ah[3], al[3]);
-#pragma unroll
-      for (int np = 0; np < DH / 16; ++np) {
-        uint32_t b0, b1, b2, b3;
-        const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int c = 2 * np + (lane >> 4);
-        ldsm_x4_t(vst + swz<DH>(key, c), b0, b1, b2, b3);
-        mma_bf16(o[2 * np], ah, b0, b1);
-        mma_bf16(o[2 * np + 1], ah, b2, b3);
-        mma_bf16(o[2 * np], al, b0, b1);
-        mma_bf16(o[2 * np + 1], al, b2, b3);
+          for (int c = 0; c < 32; ++c) o[c] *= corr;
+          tmem_st32(ta, o);
+        }
+        tmem_st_wait();
       }
+      // P = P_hi + P_lo as bf16, swizzled 128-byte rows: P_hi keeps the top
+      // 16 bits of each fp32 weight, P_lo the rounded remainder
+#pragma unroll
+      for (int cc = 0; cc < kAttnBN / 8; ++cc) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t b0 = __float_as_uint(sv[cc * 8 + 2 * e]);
+          const uint32_t b1 = __float_as_uint(sv[cc * 8 + 2 * e + 1]);
+          hi[e] = __byte_perm(b0, b1, 0x7632);
+          const float r0 = sv[cc * 8 + 2 * e] - __uint_as_float(b0 & 0xffff0000u);
+          const float r1 = sv[cc * 8 + 2 * e + 1] - __uint_as_float(b1 & 0xffff0000u);
+          const __nv_bfloat162 l2 = __floats2bfloat162_rn(r0, r1);
+          lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
+        }
+        const int off = (cc ^ (rl & 7)) << 4;
+        *reinterpret_cast<uint4*>(phi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(plo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[m]);
+      if (x.last) {
+        // the piece ends: wait for its last PV, then write the partial
+        if (!mbar_wait_bounded(&p_empty[m], tcount & 1, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const size_t prow = ((size_t)x.seg * p.slots + x.slot) * kAttnRows + m * kAttnMT + rl;
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll 1
+        for (int ch = 0; ch < DH / 32; ++ch) {
+          float o[32];
+          tmem_ld32(tmem_o + lane_off + m * DH + ch * 32, o);
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(p.o_part + prow * DH + ch * 32);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              dst[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv,
+                                   o[4 * c + 3] * inv);
+          }
+        }
+        if (valid) p.lse_part[prow] = l_run > 0.f ? m_used + log2f(l_run) : -INFINITY;
+        tc_fence_before();
+      }
+      ++tcount;
+      ++jj;
     }
-    __syncthreads();
   }
-  cp_async_wait<0>();
 
-  l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
-  l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
-  l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
-  l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
-
-  const size_t prow = ((size_t)bh * p.n_qt + qt) * p.S + s;  // partial block
-  const float inv_lo = l_lo > 0.f ? 1.f / l_lo : 0.f;
-  const float inv_hi = l_hi > 0.f ? 1.f / l_hi : 0.f;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int row = row_lo + half * 8;
-    if (qt * kBM + row >= p.R) continue;
-    const float inv = half ? inv_hi : inv_lo;
-    float* dst = p.o_part + (prow * kBM + row) * DH;
-#pragma unroll
-    for (int n = 0; n < DH / 8; ++n) {
-      const int col = n * 8 + (lane & 3) * 2;
-      float2 v;
-      v.x = o[n][2 * half] * inv;
-      v.y = o[n][2 * half + 1] * inv;
-      *reinterpret_cast<float2*>(dst + col) = v;
-    }
-    if ((lane & 3) == 0) {
-      const float m = half ? m_hi : m_lo;
-      const float l = half ? l_hi : l_lo;
-      p.lse_part[prow * kBM + row] = l > 0.f ? m + log2f(l) : -INFINITY;
-    }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kAttnTmemCols);
   }
 }
 
-// merge the splits of every query row; one warp per row
+// merge the pieces of every query row; one warp per row
 template <int DH>
 __global__ void __launch_bounds__(256)
     attn_combine_kernel(AttnParams p, void* __restrict__ out, int out_f32) {
+  __shared__ int cumT[kAttnMaxB + 1];
+  __shared__ int sched_ok;
+  if (threadIdx.x < 32) {
+    const bool ok = build_schedule(p, cumT);
+    if (threadIdx.x == 0) sched_ok = ok ? 1 : 0;
+  }
+  __syncthreads();
+  if (!sched_ok) return;  // reported by the attention kernel
+  const int per = tiles_per_cta(cumT[p.B], p.grid);
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  const int total = p.B * p.Hkv * p.R;
-  if (gw >= total) return;
+  const int total_rows = p.B * p.Hkv * p.R;
+  if (gw >= total_rows) return;
   const int bh = gw / p.R;
   const int r = gw - bh * p.R;
   const int b = bh / p.Hkv;
   const int kvh = bh - b * p.Hkv;
+  const int qg = r / kAttnRows, row = r - qg * kAttnRows;
   const int P = p.prefix_len[b];
-  if (P < 0 || P > p.max_prefix || P + p.N > p.cap) return;  // reported by the attention kernel
-  const int n_split = (P + p.chunk - 1) / p.chunk + 1;
-  const int qt = r / kBM, row = r - qt * kBM;
-  const size_t pbase = ((size_t)bh * p.n_qt + qt) * p.S;
+  const int ntiles = (P + kAttnBN - 1) / kAttnBN + p.T_tree;
+  const int seg_start = cumT[b] + (kvh * p.n_qg + qg) * ntiles;
+  const int n_pieces = (seg_start + ntiles - 1) / per - seg_start / per + 1;
+  const int seg = bh * p.n_qg + qg;
+  const size_t pbase = (size_t)seg * p.slots;
   float M = -INFINITY;
-  for (int s = 0; s < n_split; ++s) M = fmaxf(M, p.lse_part[(pbase + s) * kBM + row]);
+  for (int k = 0; k < n_pieces; ++k) M = fmaxf(M, p.lse_part[(pbase + k) * kAttnRows + row]);
   constexpr int PER = DH / 32;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float wsum = 0.f;
-  for (int s = 0; s < n_split; ++s) {
-    const float lse = p.lse_part[(pbase + s) * kBM + row];
+  for (int k = 0; k < n_pieces; ++k) {
+    const float lse = p.lse_part[(pbase + k) * kAttnRows + row];
     const float w = lse == -INFINITY ? 0.f : exp2f(lse - M);
     wsum += w;
-    const float* src = p.o_part + ((pbase + s) * kBM + row) * DH + lane * PER;
+    const float* src = p.o_part + ((pbase + k) * kAttnRows + row) * DH + lane * PER;
 #pragma unroll
     for (int e = 0; e < PER; ++e) acc[e] += w * src[e];
   }
@@ -475,31 +726,18 @@ __global__ void __launch_bounds__(256)
 // ----------------------------------------------------------------------------
 namespace {
 
-struct Split {
-  int n_qt, S, chunk;
+struct Plan {
+  int n_qg, T_tree, slots;
 };
 
-Split plan_split(int B, int N, int Hq, int Hkv, int max_prefix) {
-  Split sp{};
+Plan plan(int N, int Hq, int Hkv, int max_prefix) {
+  Plan pl{};
   const int R = N * (Hq / Hkv);
-  sp.n_qt = (R + kBM - 1) / kBM;
-  const long long groups = (long long)B * Hkv * sp.n_qt;
-  // about eight CTAs per SM of a 148-SM B200 (a fixed number, so that the
-  // workspace size does not depend on the device queried)
-  const long long target = 8LL * 148;
-  long long splits = target / (groups > 0 ? groups : 1);
-  if (splits < 1) splits = 1;
-  int chunk = (int)((max_prefix + splits - 1) / splits);
-  chunk = ((chunk + kBN - 1) / kBN) * kBN;
-  if (chunk < 4 * kBN) chunk = 4 * kBN;
-  sp.chunk = chunk;
-  sp.S = (max_prefix + chunk - 1) / chunk + 1;
-  return sp;
-}
-
-template <int DH>
-size_t attn_smem() {
-  return (size_t)kBM * DH * 2 + 4 * (size_t)kBN * DH * 2 + kBM * 8 * 4;
+  pl.n_qg = (R + kAttnRows - 1) / kAttnRows;
+  pl.T_tree = (N + kAttnBN - 1) / kAttnBN;
+  const int max_seg_tiles = (max_prefix + kAttnBN - 1) / kAttnBN + pl.T_tree;
+  pl.slots = (max_seg_tiles + kAttnMinTiles - 1) / kAttnMinTiles + 1;
+  return pl;
 }
 
 }  // namespace
@@ -507,19 +745,30 @@ size_t attn_smem() {
 size_t tree_attention_workspace_size(int B, int N, int Hq, int Hkv, int dh, int max_prefix,
                                      medusa_dtype_t dt) {
   if (dt == MEDUSA_F32) return 0;
-  const Split sp = plan_split(B, N, Hq, Hkv, max_prefix);
-  const size_t rows = (size_t)B * Hkv * sp.n_qt * sp.S * kBM;
+  const Plan pl = plan(N, Hq, Hkv, max_prefix);
+  const size_t rows = (size_t)B * Hkv * pl.n_qg * pl.slots * kAttnRows;
   return align256(rows * dh * 4) + align256(rows * 4);
 }
 
 template <int DH>
 static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaStream_t stream) {
-  const size_t smem = attn_smem<DH>();
-  if (cudaFuncSetAttribute(tree_attn_bf16_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  using L = AttnSmem<DH>;
+  // caches [B*Hkv][cap][DH]; tree K/V [B][N][Hkv][DH]; tiles of 64 keys x 64
+  CUtensorMap mK, mV, mKn, mVn;
+  const uint64_t dc[3] = {DH, (uint64_t)p.cap, (uint64_t)p.B * p.Hkv};
+  const uint64_t sc[2] = {DH * 2, (uint64_t)p.cap * DH * 2};
+  const uint32_t bc[3] = {64, kAttnBN, 1};
+  const uint64_t dn[4] = {DH, (uint64_t)p.Hkv, (uint64_t)p.N, (uint64_t)p.B};
+  const uint64_t sn[3] = {DH * 2, (uint64_t)p.Hkv * DH * 2, (uint64_t)p.N * p.Hkv * DH * 2};
+  const uint32_t bn[4] = {64, 1, kAttnBN, 1};
+  if (!make_tmap_bf16(&mK, p.Kc, 3, dc, sc, bc) || !make_tmap_bf16(&mV, p.Vc, 3, dc, sc, bc) ||
+      !make_tmap_bf16(&mKn, p.k_new, 4, dn, sn, bn) || !make_tmap_bf16(&mVn, p.v_new, 4, dn, sn, bn))
+    return fail(MEDUSA_ERR_CUDA, "tree_attention: cuTensorMapEncodeTiled failed");
+  if (cudaFuncSetAttribute(tree_attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           L::kAlloc) != cudaSuccess)
     return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(tree_attention) failed");
-  dim3 grid(p.S, p.n_qt, p.B * p.Hkv);
-  tree_attn_bf16_kernel<DH><<<grid, kAttnThreads, smem, stream>>>(p);
+  p.grid = device_sm_count();  // persistent: one CTA per SM
+  tree_attn_tc_kernel<DH><<<p.grid, kAttnThreads, L::kAlloc, stream>>>(mK, mV, mKn, mVn, p);
   medusa_status_t st = check_launch("tree_attention");
   if (st != MEDUSA_OK) return st;
   const int rows = p.B * p.Hkv * p.R;
@@ -551,7 +800,7 @@ medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_n
         words, scale, out, out_f32);
     return check_launch("tree_attention_f32");
   }
-  const Split sp = plan_split(B, N, Hq, Hkv, max_prefix);
+  const Plan pl = plan(N, Hq, Hkv, max_prefix);
   AttnParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_new = static_cast<const __nv_bfloat16*>(k_new);
@@ -560,7 +809,7 @@ medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_n
   p.Vc = static_cast<__nv_bfloat16*>(Vc);
   p.prefix_len = prefix_len;
   p.anc_mask = anc_mask;
-  const size_t rows = (size_t)B * Hkv * sp.n_qt * sp.S * kBM;
+  const size_t rows = (size_t)B * Hkv * pl.n_qg * pl.slots * kAttnRows;
   p.o_part = static_cast<float*>(ws);
   p.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(rows * dh * 4));
   p.B = B;
@@ -569,9 +818,9 @@ medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_n
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
   p.R = N * p.G;
-  p.n_qt = sp.n_qt;
-  p.S = sp.S;
-  p.chunk = sp.chunk;
+  p.n_qg = pl.n_qg;
+  p.T_tree = pl.T_tree;
+  p.slots = pl.slots;
   p.cap = cap;
   p.max_prefix = max_prefix;
   p.words = words;

@@ -221,7 +221,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int c0 = 0; epi_ok && c0 < NB; c0 += 16) {
         float v[16];
         tmem_ld16(taddr + c0, v);
-        tmem_ld_wait();
         if (MODE == kModeW1) {
           if (valid) {
             const float bias = __bfloat162float(p.b1[(size_t)head * p.d + r]);
@@ -397,47 +396,16 @@ __global__ void __launch_bounds__(256)
 // ----------------------------------------------------------------------------
 namespace {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess) {
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-  }
-  return fn;
-}
-
-// bf16 tensor [dim2][dim1][dim0] (dim0 contiguous), box {64, box1, 1},
-// 128-byte swizzle, zero fill outside the tensor.
+// bf16 tensor [dim2][dim1][dim0] (dim0 contiguous), box {64, box1, 1}
 bool make_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
                  uint32_t box1) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[3] = {dim0, dim1, dim2};
-  cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(kTileK), box1, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  const uint64_t dims[3] = {dim0, dim1, dim2};
+  const uint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
+  const uint32_t box[3] = {static_cast<uint32_t>(kTileK), box1, 1};
+  return make_tmap_bf16(map, base, 3, dims, strides, box);
 }
 
-int num_sms() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
+int num_sms() { return device_sm_count(); }
 
 template <int NB, int S, int MODE>
 medusa_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
