@@ -23,6 +23,7 @@
 //
 // fp32 path: one warp per query row on CUDA cores (small shapes).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -32,15 +33,15 @@
 
 namespace medusa {
 
-constexpr int kAttnBN = 64;          // keys per tile
+constexpr int kAttnBN = 128;         // keys per tile (UMMA N of S = Q K^T)
 constexpr int kAttnMT = 128;         // query rows per M tile (UMMA M)
 constexpr int kAttnRows = 256;       // query rows per segment (two M tiles)
-constexpr int kAttnStages = 3;       // K/V ring depth
-constexpr int kAttnThreads = 320;    // producer, MMA, two softmax warpgroups
+constexpr int kAttnStages = 2;       // K/V ring depth (64 KB per stage)
+constexpr int kAttnThreads = 384;    // producer, MMA, two softmax warpgroups, two V converters
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold, log2 units
 constexpr uint32_t kAttnTmemCols = 512;
 constexpr int kAttnMaxB = 256;       // sequences per call (schedule table in shared memory)
-constexpr int kAttnMinTiles = 16;    // smallest tile range a CTA takes
+constexpr int kAttnMinTiles = 8;     // smallest tile range a CTA takes
 
 // 2^x with the SFU instruction (ex2.approx; relative error about 2^-22, -inf -> 0)
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -69,25 +70,24 @@ struct AttnSmem {
   static constexpr int kPanels = DH / 64;                  // 64-element (128 B) panels
   static constexpr int kQBytes = kAttnMT * DH * 2;         // one M tile of Q
   static constexpr int kKVBytes = kAttnBN * DH * 2;        // one K (or V) tile
-  static constexpr int kPBytes = kAttnMT * kAttnBN * 2;    // one of P_hi / P_lo
+  static constexpr int kPanelBytes = kAttnBN * 128;        // one 64-element panel of a tile
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + 2 * kQBytes;
   static constexpr int kVOff = kKOff + kAttnStages * kKVBytes;
-  static constexpr int kPOff = kVOff + kAttnStages * kKVBytes;
-  static constexpr int kBarOff = kPOff + 4 * kPBytes;
-  // kv_full[S], kv_empty[S], q_full[2], s_full[2][2], s_free[2][2], p_full[2],
-  // p_empty[2], drain
-  static constexpr int kNumBars = 2 * kAttnStages + 2 + 4 + 4 + 2 + 2 + 1;
+  static constexpr int kBarOff = kVOff + kAttnStages * kKVBytes;
+  // kv_full[S], kv_empty[S], v_ready[S], q_full[2], s_full[2], p_full[2], p_empty[2], drain
+  static constexpr int kNumBars = 3 * kAttnStages + 2 + 2 + 2 + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kCumOff = kMiscOff + 16;            // int cumT[kAttnMaxB + 1]
-  static constexpr int kBytes = kCumOff + (kAttnMaxB + 1) * 4;
+  static constexpr int kPrefOff = kCumOff + (kAttnMaxB + 1) * 4;  // int P[kAttnMaxB]
+  static constexpr int kBytes = kPrefOff + kAttnMaxB * 4;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
 // ----------------------------------------------------------------------------
 // Schedule.  Segment = (sequence b, kv head, query group of 256 rows); its
-// tiles are the ceil(P_b / 64) prefix tiles followed by the ceil(N / 64) tree
-// tiles.  Segments are laid end to end (b-major) and every CTA takes an equal
+// tiles are the ceil(P_b / 128) prefix tiles followed by the ceil(N / 128)
+// tree tiles.  Segments are laid end to end (b-major) and every CTA takes an equal
 // contiguous range of `per` tiles; a range cut at segment ends gives pieces,
 // each written as one partial result (slot k = CTA - first CTA of the segment).
 // ----------------------------------------------------------------------------
@@ -96,8 +96,9 @@ struct TileInfo {
   bool first, last;
 };
 
-__device__ __forceinline__ void decode_tile(int t, const int* cumT, const AttnParams& p, int per,
-                                            int t0, int t1, TileInfo& x) {
+__device__ __forceinline__ void decode_tile(int t, const int* cumT, const int* pref,
+                                            const AttnParams& p, int per, int t0, int t1,
+                                            TileInfo& x) {
   int lo = 0, hi = p.B;  // cumT[lo] <= t < cumT[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -105,7 +106,7 @@ __device__ __forceinline__ void decode_tile(int t, const int* cumT, const AttnPa
     else hi = mid;
   }
   x.b = lo;
-  x.P = p.prefix_len[lo];
+  x.P = pref[lo];
   x.tpre = (x.P + kAttnBN - 1) / kAttnBN;
   x.ntiles = x.tpre + p.T_tree;
   const int rem = t - cumT[lo];
@@ -121,9 +122,56 @@ __device__ __forceinline__ void decode_tile(int t, const int* cumT, const AttnPa
   x.n_mt = min(2, (p.R - x.qg * kAttnRows + kAttnMT - 1) / kAttnMT);
 }
 
+// Walks a CTA's tile range one tile at a time: decode_tile once, then only
+// increments (the single-thread roles cannot afford a division per tile).
+struct TileCursor {
+  TileInfo x;
+  int t, t0, t1, per, sib;
+  const int* pref;
+  const AttnParams* p;
+
+  __device__ __forceinline__ void init(int t_, int t0_, int t1_, int per_, const int* cumT,
+                                       const int* pref_, const AttnParams& pp) {
+    t = t_;
+    t0 = t0_;
+    t1 = t1_;
+    per = per_;
+    pref = pref_;
+    p = &pp;
+    if (t < t1) {
+      decode_tile(t, cumT, pref, pp, per, t0, t1, x);
+      sib = x.kvh * pp.n_qg + x.qg;
+    }
+  }
+
+  __device__ __forceinline__ void advance() {
+    ++t;
+    if (t >= t1) return;
+    if (++x.lt == x.ntiles) {
+      // next segment: next (kv head, query group) of this sequence, or the
+      // next sequence
+      x.lt = 0;
+      if (++sib == p->Hkv * p->n_qg) {
+        sib = 0;
+        ++x.b;
+        x.P = pref[x.b];
+        x.tpre = (x.P + kAttnBN - 1) / kAttnBN;
+        x.ntiles = x.tpre + p->T_tree;
+      }
+      x.kvh = sib / p->n_qg;
+      x.qg = sib - x.kvh * p->n_qg;
+      x.seg = (x.b * p->Hkv + x.kvh) * p->n_qg + x.qg;
+      x.slot = t0 / per - t / per;
+      x.n_mt = min(2, (p->R - x.qg * kAttnRows + kAttnMT - 1) / kAttnMT);
+    }
+    x.first = (x.lt == 0);
+    x.last = (t == t1 - 1) || (x.lt == x.ntiles - 1);
+  }
+};
+
 // cumT[b] = tiles of all segments of sequences < b; returns false if some
 // prefix length is out of range.  Called by one full warp.
-__device__ __forceinline__ bool build_schedule(const AttnParams& p, int* cumT) {
+__device__ __forceinline__ bool build_schedule(const AttnParams& p, int* cumT, int* pref) {
   const int lane = threadIdx.x & 31;
   int run = 0;
   bool ok = true;
@@ -133,6 +181,7 @@ __device__ __forceinline__ bool build_schedule(const AttnParams& p, int* cumT) {
     int v = 0;
     if (b < p.B) {
       const int P = p.prefix_len[b];
+      if (pref != nullptr) pref[b] = P;
       if (P < 0 || P > p.max_prefix || P + p.N > p.cap) ok = false;
       v = ((max(P, 0) + kAttnBN - 1) / kAttnBN + p.T_tree) * p.Hkv * p.n_qg;
     }
@@ -162,11 +211,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   int* cumT = reinterpret_cast<int*>(smem + L::kCumOff);
+  int* pref = reinterpret_cast<int*>(smem + L::kPrefOff);
   volatile int* sched_ok = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (warp == 0) {
-    const bool ok = build_schedule(p, cumT);
+    const bool ok = build_schedule(p, cumT, pref);
     if (lane == 0) *sched_ok = ok ? 1 : 0;
   }
   __syncthreads();
@@ -184,11 +234,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + kAttnStages;
-  uint64_t* q_full = bars + 2 * kAttnStages;
-  uint64_t* s_full = q_full + 2;   // [m * 2 + buf]
-  uint64_t* s_free = s_full + 4;   // [m * 2 + buf]
-  uint64_t* p_full = s_free + 4;   // [m]
-  uint64_t* p_empty = p_full + 2;  // [m]
+  uint64_t* v_ready = bars + 2 * kAttnStages;  // V tile converted to fp16
+  uint64_t* q_full = bars + 3 * kAttnStages;  // [m]
+  uint64_t* s_full = q_full + 2;              // [m]
+  uint64_t* p_full = s_full + 2;              // [m]
+  uint64_t* p_empty = p_full + 2;             // [m]
   uint64_t* drain = p_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -197,15 +247,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < kAttnStages; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
+      mbar_init(&v_ready[i], 64);
     }
     for (int m = 0; m < 2; ++m) {
       mbar_init(&q_full[m], 128);
+      mbar_init(&s_full[m], 1);
       mbar_init(&p_full[m], 128);
       mbar_init(&p_empty[m], 1);
-      for (int bf = 0; bf < 2; ++bf) {
-        mbar_init(&s_full[m * 2 + bf], 1);
-        mbar_init(&s_free[m * 2 + bf], 128);
-      }
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -219,8 +267,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const uint32_t tmem_o = tmem_base;             // O[m]: columns m*DH .. m*DH+DH-1
-  const uint32_t tmem_s = tmem_base + 2 * DH;    // S[m][buf]: 64 columns each
+  const uint32_t tmem_o = tmem_base;           // O[m]: columns m*DH .. m*DH+DH-1
+  const uint32_t tmem_s = tmem_base + 2 * DH;  // S[m] then P[m]: 128 columns each
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -230,10 +278,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_prefetch_desc(&tmKn);
       tma_prefetch_desc(&tmVn);
       const uint64_t pol = p.n_qg > 1 ? l2_policy_evict_last() : l2_policy_evict_first();
+      TileCursor cur;
+      cur.init(t0, t0, t1, per, cumT, pref, p);
       int j = 0;
-      for (; j < n; ++j) {
-        TileInfo x;
-        decode_tile(t0 + j, cumT, p, per, t0, t1, x);
+      for (; j < n; ++j, cur.advance()) {
+        const TileInfo& x = cur.x;
         const int st = j % kAttnStages;
         if (!mbar_wait_bounded(&kv_empty[st], ((j / kAttnStages) & 1) ^ 1u, abort_flag, p.status))
           break;
@@ -245,13 +294,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int pn = 0; pn < L::kPanels; ++pn) {
           if (x.lt < x.tpre) {
             const int key = x.lt * kAttnBN;
-            tma_load_3d(kdst + pn * kAttnBN * 128, &tmK, &kv_full[st], pn * 64, key, bh, pol);
-            tma_load_3d(vdst + pn * kAttnBN * 128, &tmV, &kv_full[st], pn * 64, key, bh, pol);
+            tma_load_3d(kdst + pn * L::kPanelBytes, &tmK, &kv_full[st], pn * 64, key, bh, pol);
+            tma_load_3d(vdst + pn * L::kPanelBytes, &tmV, &kv_full[st], pn * 64, key, bh, pol);
           } else {
             const int node = (x.lt - x.tpre) * kAttnBN;
-            tma_load_4d(kdst + pn * kAttnBN * 128, &tmKn, &kv_full[st], pn * 64, x.kvh, node, x.b,
+            tma_load_4d(kdst + pn * L::kPanelBytes, &tmKn, &kv_full[st], pn * 64, x.kvh, node, x.b,
                         pol);
-            tma_load_4d(vdst + pn * kAttnBN * 128, &tmVn, &kv_full[st], pn * 64, x.kvh, node, x.b,
+            tma_load_4d(vdst + pn * L::kPanelBytes, &tmVn, &kv_full[st], pn * 64, x.kvh, node, x.b,
                         pol);
           }
         }
@@ -264,89 +313,159 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // Order per tile j: PV(0,j), QK(0,j+1), PV(1,j), QK(1,j+1): each M tile
+    // has one S/P buffer, and while one warpgroup computes its softmax the
+    // tensor core works on the other M tile.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(kAttnMT, kAttnBN, 0);
-      constexpr uint32_t idesc_pv = umma_idesc_bf16(kAttnMT, DH, 1);
-      int tq[2] = {0, 0}, pq[2] = {0, 0}, tp[2] = {0, 0};
-      auto issue_qk = [&](int j) -> bool {
-        TileInfo x;
-        decode_tile(t0 + j, cumT, p, per, t0, t1, x);
-        const int st = j % kAttnStages;
-        if (!mbar_wait_bounded(&kv_full[st], (j / kAttnStages) & 1, abort_flag, p.status))
+      constexpr uint32_t idesc_pv = umma_idesc_f16(kAttnMT, DH, 1);
+      int pq[2] = {0, 0}, tp[2] = {0, 0};
+      // shared-memory descriptors built once; advancing a descriptor only adds
+      // to its start-address field (16-byte units)
+      const uint64_t dq0 = umma_desc_sw128(smem_u32(smem + L::kQOff));
+      const uint64_t dk0 = umma_desc_sw128(smem_u32(smem + L::kKOff));
+      const uint64_t dv0 = umma_desc_sw128_lbo(smem_u32(smem + L::kVOff), L::kPanelBytes, 1024);
+      TileCursor cq, cp;
+      cq.init(t0, t0, t1, per, cumT, pref, p);
+      cp.init(t0, t0, t1, per, cumT, pref, p);
+      bool ok = true;
+      int kv_ready = -1;  // last tile whose K/V stage this thread has waited for
+      auto wait_kv = [&](int j) -> bool {
+        if (kv_ready >= j) return true;
+        if (!mbar_wait_bounded(&kv_full[j % kAttnStages], (j / kAttnStages) & 1, abort_flag,
+                               p.status))
           return false;
-        const uint32_t kaddr = smem_u32(smem + L::kKOff + st * L::kKVBytes);
-        for (int m = 0; m < x.n_mt; ++m) {
-          if (x.first) {
-            if (!mbar_wait_bounded(&q_full[m], pq[m] & 1, abort_flag, p.status)) return false;
-            ++pq[m];
-          }
-          const int bf = tq[m] & 1;
-          if (!mbar_wait_bounded(&s_free[m * 2 + bf], ((tq[m] >> 1) & 1) ^ 1u, abort_flag,
+        kv_ready = j;
+        return true;
+      };
+      // S[m] = Q[m] K^T for tile j (cursor cq at tile j)
+      auto issue_qk = [&](int m, int j, const TileInfo& x) -> bool {
+        if (!wait_kv(j)) return false;
+        if (x.first) {
+          if (!mbar_wait_bounded(&q_full[m], pq[m] & 1, abort_flag, p.status)) return false;
+          ++pq[m];
+        }
+        tc_fence_after();
+        const uint64_t dq = dq0 + (uint64_t)((m * L::kQBytes) >> 4);
+        const uint64_t dk = dk0 + (uint64_t)(((j % kAttnStages) * L::kKVBytes) >> 4);
+        const uint32_t d = tmem_s + m * kAttnBN;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          constexpr uint32_t qpanel = (kAttnMT * 128) >> 4, kpanel = L::kPanelBytes >> 4;
+          const uint32_t qo = (kk >> 2) * qpanel + (kk & 3) * 2;
+          const uint32_t ko = (kk >> 2) * kpanel + (kk & 3) * 2;
+          umma_bf16(d, dq + qo, dk + ko, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[m]);
+        return true;
+      };
+      int v_ok = -1;  // last tile whose converted V this thread has waited for
+      // O[m] (+)= P[m] V for tile j
+      auto issue_pv = [&](int m, int j, const TileInfo& x) -> bool {
+        if (v_ok < j) {
+          if (!mbar_wait_bounded(&v_ready[j % kAttnStages], (j / kAttnStages) & 1, abort_flag,
                                  p.status))
             return false;
-          tc_fence_after();
-          const uint32_t qaddr = smem_u32(smem + L::kQOff + m * L::kQBytes);
-          const uint32_t d = tmem_s + (m * 2 + bf) * kAttnBN;
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            const uint32_t a = qaddr + (kk >> 2) * (kAttnMT * 128) + (kk & 3) * 32;
-            const uint32_t bb = kaddr + (kk >> 2) * (kAttnBN * 128) + (kk & 3) * 32;
-            umma_bf16(d, umma_desc_sw128(a), umma_desc_sw128(bb), idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[m * 2 + bf]);
-          ++tq[m];
+          v_ok = j;
         }
+        if (!mbar_wait_bounded(&p_full[m], tp[m] & 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint64_t dv = dv0 + (uint64_t)(((j % kAttnStages) * L::kKVBytes) >> 4);
+        const uint32_t d = tmem_o + m * DH;
+        const uint32_t pcol = tmem_s + m * kAttnBN;
+        const uint32_t acc0 = x.first ? 0u : 1u;
+#pragma unroll
+        for (int kk = 0; kk < kAttnBN / 16; ++kk) {
+          // P in TMEM: 16 keys = 8 columns of packed fp16 pairs.
+          // V (fp16 after conversion): M/N-major, 16 keys = two 8-row groups
+          // of 1024 bytes; the second 64-element head-dimension panel sits
+          // one tile-panel on.
+          umma_bf16_ts(d, pcol + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
+                       kk > 0 ? 1u : acc0);
+        }
+        umma_commit(&p_empty[m]);
+        ++tp[m];
         return true;
       };
-      auto issue_pv = [&](int j) -> bool {
-        TileInfo x;
-        decode_tile(t0 + j, cumT, p, per, t0, t1, x);
-        const int st = j % kAttnStages;
-        const uint32_t vaddr = smem_u32(smem + L::kVOff + st * L::kKVBytes);
-        for (int m = 0; m < x.n_mt; ++m) {
-          if (!mbar_wait_bounded(&p_full[m], tp[m] & 1, abort_flag, p.status)) return false;
-          tc_fence_after();
-          const uint32_t d = tmem_o + m * DH;
-#pragma unroll
-          for (int hl = 0; hl < 2; ++hl) {
-            const uint32_t paddr = smem_u32(smem + L::kPOff + (m * 2 + hl) * L::kPBytes);
-#pragma unroll
-            for (int kk = 0; kk < kAttnBN / 16; ++kk) {
-              // P: K-major, 16 keys = 32 bytes along the swizzled row.
-              // V: M/N-major, 16 keys = two 8-row groups of 1024 bytes; the
-              // second 64-element head-dimension panel sits one tile-panel on.
-              umma_bf16(d, umma_desc_sw128(paddr + kk * 32),
-                        umma_desc_sw128_lbo(vaddr + kk * 16 * 128, kAttnBN * 128, 1024), idesc_pv,
-                        (!x.first || hl > 0 || kk > 0) ? 1u : 0u);
-            }
-          }
-          umma_commit(&p_empty[m]);
-          ++tp[m];
-        }
-        umma_commit(&kv_empty[st]);
-        return true;
-      };
-      // order: QK(0), QK(1), then PV(j) followed by QK(j+2), so that PV(j)
-      // never waits for a K/V tile that is still loading
-      bool ok = issue_qk(0);
-      if (ok && n > 1) ok = issue_qk(1);
+      for (int m = 0; ok && m < cq.x.n_mt; ++m) ok = issue_qk(m, 0, cq.x);
+      cq.advance();
       for (int j = 0; ok && j < n; ++j) {
-        ok = issue_pv(j);
-        if (ok && j + 2 < n) ok = issue_qk(j + 2);
+        const TileInfo x = cp.x;      // tile j
+        const TileInfo y = cq.x;      // tile j + 1 (valid when j + 1 < n)
+        const bool next = j + 1 < n;
+        for (int m = 0; ok && m < 2; ++m) {
+          if (m < x.n_mt) {
+            ok = issue_pv(m, j, x);
+            if (ok && m == x.n_mt - 1) umma_commit(&kv_empty[j % kAttnStages]);
+          }
+          if (ok && next && m < y.n_mt) ok = issue_qk(m, j + 1, y);
+        }
+        cp.advance();
+        cq.advance();
       }
       umma_commit(drain);
       int dummy_abort = 0;
       mbar_wait_bounded(drain, 0, &dummy_abort, p.status);
     }
+  } else if (warp >= 10) {
+    // ---------------- V converters (warps 10, 11) ----------------
+    // Each landed V tile is rewritten in place from bf16 to fp16 (the value
+    // product runs on fp16 P and V); rows past the prefix end of a partial
+    // tile are cleared (their weights are zero, but 0 * NaN is not).  A V
+    // entry of magnitude 65536 or more, inf or NaN is reported as a
+    // device-check error.
+    const int ct = (warp - 10) * 32 + lane;
+    TileCursor cur;
+    cur.init(t0, t0, t1, per, cumT, pref, p);
+    bool range_ok = true;
+    for (int j = 0; j < n; ++j, cur.advance()) {
+      const TileInfo& x = cur.x;
+      const int st = j % kAttnStages;
+      if (!mbar_wait_bounded(&kv_full[st], (j / kAttnStages) & 1, abort_flag, p.status)) break;
+      const bool tree_tile = x.lt >= x.tpre;
+      const int kbase = tree_tile ? (x.lt - x.tpre) * kAttnBN : x.lt * kAttnBN;
+      const int zero_from = tree_tile ? kAttnBN : min(kAttnBN, x.P - kbase);
+      uint4* vt = reinterpret_cast<uint4*>(smem + L::kVOff + st * L::kKVBytes);
+      constexpr int kChunks = L::kKVBytes / 16, kPanelChunks = L::kPanelBytes / 16;
+      constexpr int kUnroll = 8;
+      static_assert(kChunks % (64 * kUnroll) == 0, "V tile must split evenly over the converters");
+      uint32_t vmax = 0u;  // largest |v| bit pattern seen (bf16 halves)
+#pragma unroll 1
+      for (int e0 = ct; e0 < kChunks; e0 += 64 * kUnroll) {
+        uint4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) v[u] = vt[e0 + u * 64];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int row = ((e0 + u * 64) % kPanelChunks) >> 3;  // key within the tile
+          uint32_t* w = &v[u].x;
+          const bool keep = row < zero_from;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (keep) vmax = __vmaxu2(vmax, w[q] & 0x7FFF7FFFu);
+            const __half2 h2 = __floats2half2_rn(__uint_as_float(w[q] << 16),
+                                                 __uint_as_float(w[q] & 0xffff0000u));
+            w[q] = keep ? *reinterpret_cast<const uint32_t*>(&h2) : 0u;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) vt[e0 + u * 64] = v[u];
+      }
+      // |v| of 65536 and above (0x4780: the first bf16 past fp16's 65504),
+      // inf or NaN cannot be carried by the fp16 value product
+      if (__vcmpgtu2(vmax, 0x477F477Fu)) range_ok = false;
+      fence_proxy_async_smem();
+      mbar_arrive(&v_ready[st]);
+    }
+    if (!range_ok) report(p.status, MEDUSA_ERR_DEVICE_CHECK);
   } else {
     // ---------------- softmax warpgroups ----------------
     const int m = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int rl = quad * 32 + lane;  // row within the M tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t srow = tmem_s + lane_off + m * kAttnBN;
     uint8_t* qtile = smem + L::kQOff + m * L::kQBytes;
-    uint8_t* phi = smem + L::kPOff + (m * 2 + 0) * L::kPBytes + rl * 128;
-    uint8_t* plo = smem + L::kPOff + (m * 2 + 1) * L::kPBytes + rl * 128;
 
     // Q rows of a segment into the swizzled K-major tile (zeros past R)
     auto load_q = [&](const TileInfo& x) {
@@ -365,6 +484,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(&q_full[m]);
     };
+    // 64 scores of half h of the tile, waited
+    auto load_half = [&](int h, float (&sv)[64]) {
+      uint32_t r0[32], r1[32];
+      tmem_ld32_raw(srow + h * 64, r0);
+      tmem_ld32_raw(srow + h * 64 + 32, r1);
+      tmem_ld_wait();
+      tmem_regs_after_wait(r0);
+      tmem_regs_after_wait(r1);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        sv[c] = __uint_as_float(r0[c]);
+        sv[32 + c] = __uint_as_float(r1[c]);
+      }
+    };
 
     int tcount = 0;
     bool q_ready = false;
@@ -372,9 +505,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float m_used = -INFINITY, l_run = 0.f;
     uint32_t mw[8];
     int jj = 0;
-    for (int j = 0; ok && j < n; ++j) {
-      TileInfo x;
-      decode_tile(t0 + j, cumT, p, per, t0, t1, x);
+    TileCursor cur;
+    cur.init(t0, t0, t1, per, cumT, pref, p);
+    for (int j = 0; ok && j < n; ++j, cur.advance()) {
+      const TileInfo x = cur.x;
       if (m >= x.n_mt) continue;
       const int r = x.qg * kAttnRows + m * kAttnMT + rl;
       const bool valid = r < p.R;
@@ -401,138 +535,113 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           *reinterpret_cast<uint4*>(p.Vc + dst) = *reinterpret_cast<const uint4*>(p.v_new + src);
         }
       }
-      const int bf = tcount & 1;
-      if (!mbar_wait_bounded(&s_full[m * 2 + bf], (tcount >> 1) & 1, abort_flag, p.status)) {
+      if (!mbar_wait_bounded(&s_full[m], tcount & 1, abort_flag, p.status)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float sv[kAttnBN];
-      {
-        uint32_t r0[32], r1[32];
-        const uint32_t ta = tmem_s + lane_off + (m * 2 + bf) * kAttnBN;
-        tmem_ld32_raw(ta, r0);
-        tmem_ld32_raw(ta + 32, r1);
-        tmem_ld_wait();
-        tmem_regs_after_wait(r0);
-        tmem_regs_after_wait(r1);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          sv[c] = __uint_as_float(r0[c]);
-          sv[32 + c] = __uint_as_float(r1[c]);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&s_free[m * 2 + bf]);
       if (x.last && j + 1 < n) {
         // every QK of this piece is done: load the next piece's Q now, so the
         // MMA warp can run ahead into it
-        TileInfo y;
-        decode_tile(t0 + j + 1, cumT, p, per, t0, t1, y);
-        if (m < y.n_mt) {
-          load_q(y);
+        TileCursor nx = cur;
+        nx.advance();
+        if (m < nx.x.n_mt) {
+          load_q(nx.x);
           q_ready = true;
         }
       }
       const bool tree_tile = x.lt >= x.tpre;
       const int kbase = tree_tile ? (x.lt - x.tpre) * kAttnBN : x.lt * kAttnBN;
       const int key_end = tree_tile ? p.N : x.P;
-      if (m == 0 && !tree_tile && kbase + kAttnBN > key_end) {
-        // V rows past the prefix end hold whatever the cache holds there;
-        // their weights are zero, but 0 * NaN is not, so clear them (the
-        // tile has landed: its scores were computed from the same stage)
-        uint8_t* vt = smem + L::kVOff + (j % kAttnStages) * L::kKVBytes;
-        const int from = key_end - kbase;
-        const int n16 = (kAttnBN - from) * 8 * L::kPanels;
-        for (int e = rl; e < n16; e += 128) {
-          const int pn = e / ((kAttnBN - from) * 8);
-          const int rem = e - pn * ((kAttnBN - from) * 8);
-          const int row = from + (rem >> 3);
-          *reinterpret_cast<uint4*>(vt + pn * (kAttnBN * 128) + row * 128 + ((rem & 7) << 4)) =
-              make_uint4(0u, 0u, 0u, 0u);
+      const bool full_tile = !tree_tile && kbase + kAttnBN <= key_end;
+      // the tile's four mask words, picked without dynamic register indexing
+      uint32_t tw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+      if (tree_tile) {
+        const int w0 = 4 * (x.lt - x.tpre);
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (w == w0 + q) tw[q] = mw[w];
         }
       }
-      // row maximum of the raw scores (the scale is positive); full prefix
-      // tiles need no mask
-      float mx = -INFINITY;
-      if (!tree_tile && kbase + kAttnBN <= key_end) {
+      auto visible = [&](int c) -> bool {  // c: key within the tile
+        return (kbase + c < key_end) && ((tw[c >> 5] >> (c & 31)) & 1u);
+      };
+      // One pass over the tile, in two halves of 64 keys: the exponent base is
+      // the running maximum m_used (log2 units); a half whose maximum exceeds
+      // it by more than 2^8 (or the first half of a piece) moves the base,
+      // rescaling O, l and the half already written, so that every stored
+      // weight stays <= 2^8 (well inside fp16).
+      float sum_tile = 0.f;
+      bool moved = false;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float sv[64];
+        load_half(h, sv);
+        float mx = -INFINITY;
+        if (full_tile) {
 #pragma unroll
-        for (int c = 0; c < kAttnBN; ++c) mx = fmaxf(mx, sv[c]);
-      } else {
-        // the tile's two mask words, picked without dynamic register indexing
-        uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
-        if (tree_tile) {
-          const int tw = 2 * (x.lt - x.tpre);
+          for (int c = 0; c < 64; ++c) mx = fmaxf(mx, sv[c]);
+        } else {
 #pragma unroll
-          for (int w = 0; w < 8; ++w) {
-            if (w == tw) w0 = mw[w];
-            if (w == tw + 1) w1 = mw[w];
+          for (int c = 0; c < 64; ++c) {
+            if (!visible(h * 64 + c)) sv[c] = -INFINITY;
+            mx = fmaxf(mx, sv[c]);
           }
         }
-#pragma unroll
-        for (int c = 0; c < kAttnBN; ++c) {
-          const uint32_t word = c < 32 ? w0 : w1;
-          const bool vis = (kbase + c < key_end) && ((word >> (c & 31)) & 1u);
-          sv[c] = vis ? sv[c] : -INFINITY;
-          mx = fmaxf(mx, sv[c]);
-        }
-      }
-      mx *= p.scale_log2;
-      float corr = 1.f;
-      bool resc = false;
-      if (jj == 0) {
-        m_used = mx;
-      } else if (mx > m_used + kRescaleLog2) {
-        corr = exp2f(m_used - mx);
-        m_used = mx;
-        resc = true;
-      }
-      const float nbase = m_used == -INFINITY ? 0.f : -m_used;
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < kAttnBN; ++c) {
-        sv[c] = ex2_approx(fmaf(sv[c], p.scale_log2, nbase));
-        sum += sv[c];
-      }
-      l_run = l_run * corr + sum;
-      // PV of the previous tile must be done: P buffer free, O stable
-      if (!mbar_wait_bounded(&p_empty[m], (tcount & 1) ^ 1u, abort_flag, p.status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (__any_sync(0xffffffffu, resc)) {
+        mx *= p.scale_log2;
+        const bool need = (m_used == -INFINITY) ? (mx != -INFINITY) : (mx > m_used + kRescaleLog2);
+        if (__any_sync(0xffffffffu, need)) {
+          const float new_m = need ? mx : m_used;
+          const float corr = (need && m_used != -INFINITY) ? ex2_approx(m_used - new_m) : 1.f;
+          if (jj > 0) {
+            // O holds earlier tiles (their PV is done: this tile's QK was
+            // issued after it)
 #pragma unroll 1
-        for (int ch = 0; ch < DH / 32; ++ch) {
-          float o[32];
-          const uint32_t ta = tmem_o + lane_off + m * DH + ch * 32;
-          tmem_ld32(ta, o);
+            for (int ch = 0; ch < DH / 32; ++ch) {
+              float o[32];
+              const uint32_t ta = tmem_o + lane_off + m * DH + ch * 32;
+              tmem_ld32(ta, o);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] *= corr;
-          tmem_st32(ta, o);
+              for (int c = 0; c < 32; ++c) o[c] *= corr;
+              tmem_st32(ta, o);
+            }
+          }
+          if (h == 1) {
+            // half 0 of this tile is already stored as fp16 pairs
+            uint32_t r0[32];
+            tmem_ld32_raw(srow, r0);
+            tmem_ld_wait();
+            tmem_regs_after_wait(r0);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r0[c]));
+              const __half2 h2 = __floats2half2_rn(f.x * corr, f.y * corr);
+              r0[c] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            tmem_st32_u(srow, r0);
+          }
+          l_run *= corr;
+          sum_tile *= corr;
+          m_used = new_m;
+          moved = true;
         }
-        tmem_st_wait();
-      }
-      // P = P_hi + P_lo as bf16, swizzled 128-byte rows: P_hi keeps the top
-      // 16 bits of each fp32 weight, P_lo the rounded remainder
+        const float nbase = m_used == -INFINITY ? 0.f : -m_used;
+        uint32_t pk[32];
 #pragma unroll
-      for (int cc = 0; cc < kAttnBN / 8; ++cc) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t b0 = __float_as_uint(sv[cc * 8 + 2 * e]);
-          const uint32_t b1 = __float_as_uint(sv[cc * 8 + 2 * e + 1]);
-          hi[e] = __byte_perm(b0, b1, 0x7632);
-          const float r0 = sv[cc * 8 + 2 * e] - __uint_as_float(b0 & 0xffff0000u);
-          const float r1 = sv[cc * 8 + 2 * e + 1] - __uint_as_float(b1 & 0xffff0000u);
-          const __nv_bfloat162 l2 = __floats2bfloat162_rn(r0, r1);
-          lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
+        for (int e = 0; e < 32; ++e) {
+          const float a0 = ex2_approx(fmaf(sv[2 * e], p.scale_log2, nbase));
+          const float a1 = ex2_approx(fmaf(sv[2 * e + 1], p.scale_log2, nbase));
+          sum_tile += a0 + a1;
+          const __half2 h2 = __floats2half2_rn(a0, a1);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-        const int off = (cc ^ (rl & 7)) << 4;
-        *reinterpret_cast<uint4*>(phi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(plo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        tmem_st32_u(srow + h * 32, pk);
       }
-      fence_proxy_async_smem();
+      (void)moved;
+      l_run += sum_tile;
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[m]);
       if (x.last) {
@@ -579,7 +688,7 @@ __global__ void __launch_bounds__(256)
   __shared__ int cumT[kAttnMaxB + 1];
   __shared__ int sched_ok;
   if (threadIdx.x < 32) {
-    const bool ok = build_schedule(p, cumT);
+    const bool ok = build_schedule(p, cumT, nullptr);
     if (threadIdx.x == 0) sched_ok = ok ? 1 : 0;
   }
   __syncthreads();
@@ -753,11 +862,12 @@ size_t tree_attention_workspace_size(int B, int N, int Hq, int Hkv, int dh, int 
 template <int DH>
 static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaStream_t stream) {
   using L = AttnSmem<DH>;
-  // caches [B*Hkv][cap][DH]; tree K/V [B][N][Hkv][DH]; tiles of 64 keys x 64
+  // caches [B*Hkv][cap][DH]; tree K/V [B][N][Hkv][DH]; boxes of 128 keys x 64
+  // head dims (one 128-byte swizzled panel)
   CUtensorMap mK, mV, mKn, mVn;
   const uint64_t dc[3] = {DH, (uint64_t)p.cap, (uint64_t)p.B * p.Hkv};
   const uint64_t sc[2] = {DH * 2, (uint64_t)p.cap * DH * 2};
-  const uint32_t bc[3] = {64, kAttnBN, 1};
+  const uint32_t bc[3] = {64, kAttnBN, 1};  // 64 head dims x 128 keys
   const uint64_t dn[4] = {DH, (uint64_t)p.Hkv, (uint64_t)p.N, (uint64_t)p.B};
   const uint64_t sn[3] = {DH * 2, (uint64_t)p.Hkv * DH * 2, (uint64_t)p.N * p.Hkv * DH * 2};
   const uint32_t bn[4] = {64, 1, kAttnBN, 1};

@@ -18,6 +18,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "abi_internal.h"
 #include "common.cuh"
@@ -114,6 +115,54 @@ __global__ void __launch_bounds__(kRowWarps * 32)
     } else {
       raw[r] = E::load_scalar(base + e0, e0 < V ? min(EV, V - e0) : 0);
     }
+  }
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && !TYPICAL) {
+    // greedy on bf16: packed maximum (NaN propagates, so one check at the
+    // end catches a NaN anywhere), then the first index holding that value
+    __nv_bfloat162 m2 = __halves2bfloat162(__ushort_as_bfloat16(0xFF80u), __ushort_as_bfloat16(0xFF80u));
+#pragma unroll
+    for (int r = 0; r < NL; ++r) {
+      const uint32_t* w = &raw[r].x;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        m2 = __hmax2_nan(m2, *reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+    }
+    const float lo_f = __low2float(m2), hi_f = __high2float(m2);
+    bool nan = (lo_f != lo_f) || (hi_f != hi_f);
+    float M = fmaxf(lo_f, hi_f);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (__any_sync(0xffffffffu, nan)) {
+      if (lane == 0) report(status, MEDUSA_ERR_DEVICE_CHECK);
+    }
+    // bf16 bit pattern of M; +0 and -0 are equal values, so a zero maximum
+    // matches either sign
+    const uint32_t mb = __float_as_uint(M) >> 16;
+    const bool zero = (mb & 0x7FFFu) == 0u;
+    const uint32_t pat = zero ? 0u : (mb | (mb << 16));
+    const uint32_t msk = zero ? 0x7FFF7FFFu : 0xFFFFFFFFu;
+    int idx = 0x7fffffff;
+#pragma unroll
+    for (int r = 0; r < NL; ++r) {
+      const int e0 = v0 + (r * 32 + lane) * EV;
+      const uint32_t* w = &raw[r].x;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t eq = __vcmpeq2(w[q] & msk, pat);
+        if (idx == 0x7fffffff && eq != 0u) idx = e0 + 2 * q + ((eq & 0xFFFFu) ? 0 : 1);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) idx = min(idx, __shfl_xor_sync(0xffffffffu, idx, o));
+    if (lane == 0) {
+      RowPart rp;
+      rp.maxz = M;
+      rp.idx = idx;
+      rp.s = 0.f;
+      rp.t = 0.f;
+      part[row * n_chunks + c] = rp;
+    }
+    return;
   }
   // best (largest, lowest index) of this lane: indices ascend in (r, e) order
   float bv = -INFINITY;
