@@ -49,6 +49,25 @@ def _peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+def heads_traffic(algorithmic):
+    """DRAM bytes of one heads call, scaled from the profiled ratio; None when
+    the kernel sources changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "heads_topk_traffic.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        h = hashlib.sha256()
+        for name in j["source_files"]:
+            with open(os.path.join(ROOT, name), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != j["source_sha256"]:
+            return None, "kernel changed since the ncu capture"
+        return algorithmic * float(j["traffic_ratio"]), j["measured_on"]
+    except (OSError, KeyError, ValueError):
+        return None, "no ncu record"
+
+
 def algorithmic_bytes(w, prefix_lens, N):
     """Bytes the step must move at minimum (bf16 = 2 B)."""
     e = 2 if w.dtype == "bf16" else 4
@@ -468,6 +487,7 @@ def main():
     hbm_peak, _, peak_kind = _peaks()
     ab = algorithmic_bytes(w, prefix_list, N)
     heads_gbs = ab["heads"] / (stages["heads_topk"] * 1e-6) / 1e9
+    traffic, traffic_src = heads_traffic(ab["heads"])
     step_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
     value = world * args.steps / (ms_total / 1e3)
 
@@ -493,7 +513,8 @@ def main():
             "stages_us": stages,
             "roofline": {"bound": "hbm", "kernel": "medusa_heads_topk (W1 GEMM + W2 GEMM + top-k merge)",
                          "achieved": heads_gbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": heads_gbs / hbm_peak, "traffic": None,
+                         "frac": heads_gbs / hbm_peak, "traffic": traffic,
+                         "traffic_source": "ncu dram bytes ratio, " + traffic_src,
                          "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": ab["heads"]},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
