@@ -58,7 +58,7 @@ struct AttnParams {
   __nv_bfloat16* Vc;
   const int32_t* prefix_len;
   const uint32_t* anc_mask;
-  float* o_part;    // [n_seg, slots, 256, DH]
+  float* o_part;    // [n_seg, slots, DH / 4, 256] groups of 4 floats
   float* lse_part;  // [n_seg, slots, 256]
   int B, N, Hq, Hkv, G, R, n_qg, T_tree, slots, cap, max_prefix, words, grid;
   float scale_log2;
@@ -78,7 +78,8 @@ struct AttnSmem {
   // kv_full[S], kv_empty[S], v_ready[S], q_full[2], s_full[2], p_full[2], p_empty[2], drain
   static constexpr int kNumBars = 3 * kAttnStages + 2 + 2 + 2 + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kCumOff = kMiscOff + 16;            // int cumT[kAttnMaxB + 1]
+  static constexpr int kInfoOff = kMiscOff + 16;           // int info[kAttnStages]
+  static constexpr int kCumOff = kInfoOff + 16;            // int cumT[kAttnMaxB + 1]
   static constexpr int kPrefOff = kCumOff + (kAttnMaxB + 1) * 4;  // int P[kAttnMaxB]
   static constexpr int kBytes = kPrefOff + kAttnMaxB * 4;
   static constexpr int kAlloc = kBytes + 1024;
@@ -169,6 +170,19 @@ struct TileCursor {
   }
 };
 
+// What the MMA and converter warps need of a tile, packed into one word by the
+// producer: bit 0 first tile of a piece (the accumulator starts over, a new Q
+// tile is awaited), bit 1 both M tiles active, bits 8..15 keys of the tile
+// that are real (rows from there on are cleared in the converted V).
+__device__ __forceinline__ int pack_stage_info(const TileInfo& x) {
+  const bool tree_tile = x.lt >= x.tpre;
+  const int zero_from = tree_tile ? kAttnBN : min(kAttnBN, x.P - x.lt * kAttnBN);
+  return (x.first ? 1 : 0) | (x.n_mt > 1 ? 2 : 0) | (zero_from << 8);
+}
+__device__ __forceinline__ bool info_first(int w) { return (w & 1) != 0; }
+__device__ __forceinline__ bool info_two(int w) { return (w & 2) != 0; }
+__device__ __forceinline__ int info_zero_from(int w) { return (w >> 8) & 0xff; }
+
 // cumT[b] = tiles of all segments of sequences < b; returns false if some
 // prefix length is out of range.  Called by one full warp.
 __device__ __forceinline__ bool build_schedule(const AttnParams& p, int* cumT, int* pref) {
@@ -242,6 +256,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* drain = p_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  int* stage_info = reinterpret_cast<int*>(smem + L::kInfoOff);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kAttnStages; ++i) {
@@ -286,6 +301,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int st = j % kAttnStages;
         if (!mbar_wait_bounded(&kv_empty[st], ((j / kAttnStages) & 1) ^ 1u, abort_flag, p.status))
           break;
+        // published with the stage (the kv_full arrive releases it): the
+        // MMA and converter warps read it instead of walking the schedule
+        stage_info[st] = pack_stage_info(x);
         mbar_arrive_expect_tx(&kv_full[st], 2 * L::kKVBytes);
         uint8_t* kdst = smem + L::kKOff + st * L::kKVBytes;
         uint8_t* vdst = smem + L::kVOff + st * L::kKVBytes;
@@ -315,39 +333,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ---------------- MMA issuer ----------------
     // Order per tile j: PV(0,j), QK(0,j+1), PV(1,j), QK(1,j+1): each M tile
     // has one S/P buffer, and while one warpgroup computes its softmax the
-    // tensor core works on the other M tile.
+    // tensor core works on the other M tile.  The loop is kept lean (one
+    // thread, sharing its issue slots with two softmax warps): tile facts come
+    // from the producer's stage info, the two M tiles are unrolled, and the
+    // barrier phases are plain counters.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(kAttnMT, kAttnBN, 0);
       constexpr uint32_t idesc_pv = umma_idesc_f16(kAttnMT, DH, 1);
-      int pq[2] = {0, 0}, tp[2] = {0, 0};
       // shared-memory descriptors built once; advancing a descriptor only adds
       // to its start-address field (16-byte units)
       const uint64_t dq0 = umma_desc_sw128(smem_u32(smem + L::kQOff));
       const uint64_t dk0 = umma_desc_sw128(smem_u32(smem + L::kKOff));
       const uint64_t dv0 = umma_desc_sw128_lbo(smem_u32(smem + L::kVOff), L::kPanelBytes, 1024);
-      TileCursor cq, cp;
-      cq.init(t0, t0, t1, per, cumT, pref, p);
-      cp.init(t0, t0, t1, per, cumT, pref, p);
-      bool ok = true;
-      int kv_ready = -1;  // last tile whose K/V stage this thread has waited for
-      auto wait_kv = [&](int j) -> bool {
-        if (kv_ready >= j) return true;
-        if (!mbar_wait_bounded(&kv_full[j % kAttnStages], (j / kAttnStages) & 1, abort_flag,
-                               p.status))
-          return false;
-        kv_ready = j;
-        return true;
-      };
-      // S[m] = Q[m] K^T for tile j (cursor cq at tile j)
-      auto issue_qk = [&](int m, int j, const TileInfo& x) -> bool {
-        if (!wait_kv(j)) return false;
-        if (x.first) {
-          if (!mbar_wait_bounded(&q_full[m], pq[m] & 1, abort_flag, p.status)) return false;
-          ++pq[m];
-        }
-        tc_fence_after();
+      // S[m] = Q[m] K^T from stage st
+      auto issue_qk = [&](int m, int st) {
         const uint64_t dq = dq0 + (uint64_t)((m * L::kQBytes) >> 4);
-        const uint64_t dk = dk0 + (uint64_t)(((j % kAttnStages) * L::kKVBytes) >> 4);
+        const uint64_t dk = dk0 + (uint64_t)((st * L::kKVBytes) >> 4);
         const uint32_t d = tmem_s + m * kAttnBN;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
@@ -357,23 +358,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           umma_bf16(d, dq + qo, dk + ko, idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[m]);
-        return true;
       };
-      int v_ok = -1;  // last tile whose converted V this thread has waited for
-      // O[m] (+)= P[m] V for tile j
-      auto issue_pv = [&](int m, int j, const TileInfo& x) -> bool {
-        if (v_ok < j) {
-          if (!mbar_wait_bounded(&v_ready[j % kAttnStages], (j / kAttnStages) & 1, abort_flag,
-                                 p.status))
-            return false;
-          v_ok = j;
-        }
-        if (!mbar_wait_bounded(&p_full[m], tp[m] & 1, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint64_t dv = dv0 + (uint64_t)(((j % kAttnStages) * L::kKVBytes) >> 4);
+      // O[m] (+)= P[m] V from stage st
+      auto issue_pv = [&](int m, int st, uint32_t acc0) {
+        const uint64_t dv = dv0 + (uint64_t)((st * L::kKVBytes) >> 4);
         const uint32_t d = tmem_o + m * DH;
         const uint32_t pcol = tmem_s + m * kAttnBN;
-        const uint32_t acc0 = x.first ? 0u : 1u;
 #pragma unroll
         for (int kk = 0; kk < kAttnBN / 16; ++kk) {
           // P in TMEM: 16 keys = 8 columns of packed fp16 pairs.
@@ -384,24 +374,59 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                        kk > 0 ? 1u : acc0);
         }
         umma_commit(&p_empty[m]);
-        ++tp[m];
-        return true;
       };
-      for (int m = 0; ok && m < cq.x.n_mt; ++m) ok = issue_qk(m, 0, cq.x);
-      cq.advance();
-      for (int j = 0; ok && j < n; ++j) {
-        const TileInfo x = cp.x;      // tile j
-        const TileInfo y = cq.x;      // tile j + 1 (valid when j + 1 < n)
-        const bool next = j + 1 < n;
-        for (int m = 0; ok && m < 2; ++m) {
-          if (m < x.n_mt) {
-            ok = issue_pv(m, j, x);
-            if (ok && m == x.n_mt - 1) umma_commit(&kv_empty[j % kAttnStages]);
+      uint32_t nq0 = 0, nq1 = 0, np0 = 0, np1 = 0;  // completed waits per barrier
+      bool ok = mbar_wait_bounded(&kv_full[0], 0, abort_flag, p.status);
+      int cur = ok ? stage_info[0] : 0;
+      if (ok) ok = mbar_wait_bounded(&q_full[0], nq0++ & 1, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        if (info_two(cur)) {
+          ok = mbar_wait_bounded(&q_full[1], nq1++ & 1, abort_flag, p.status);
+          if (ok) {
+            tc_fence_after();
+            issue_qk(1, 0);
           }
-          if (ok && next && m < y.n_mt) ok = issue_qk(m, j + 1, y);
         }
-        cp.advance();
-        cq.advance();
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % kAttnStages;
+        const int sn = (j + 1) % kAttnStages;
+        const bool has_next = j + 1 < n;
+        const bool two = info_two(cur);
+        const uint32_t acc0 = info_first(cur) ? 0u : 1u;
+        if (!mbar_wait_bounded(&v_ready[st], (j / kAttnStages) & 1, abort_flag, p.status) ||
+            !mbar_wait_bounded(&p_full[0], np0++ & 1, abort_flag, p.status))
+          break;
+        tc_fence_after();
+        issue_pv(0, st, acc0);
+        if (!two) umma_commit(&kv_empty[st]);
+        int nxt = 0;
+        if (has_next) {
+          if (!mbar_wait_bounded(&kv_full[sn], ((j + 1) / kAttnStages) & 1, abort_flag, p.status))
+            break;
+          nxt = stage_info[sn];
+          if (info_first(nxt) &&
+              !mbar_wait_bounded(&q_full[0], nq0++ & 1, abort_flag, p.status))
+            break;
+          tc_fence_after();
+          issue_qk(0, sn);
+        }
+        if (two) {
+          if (!mbar_wait_bounded(&p_full[1], np1++ & 1, abort_flag, p.status)) break;
+          tc_fence_after();
+          issue_pv(1, st, acc0);
+          umma_commit(&kv_empty[st]);
+        }
+        if (has_next && info_two(nxt)) {
+          if (info_first(nxt) &&
+              !mbar_wait_bounded(&q_full[1], nq1++ & 1, abort_flag, p.status))
+            break;
+          tc_fence_after();
+          issue_qk(1, sn);
+        }
+        cur = nxt;
       }
       umma_commit(drain);
       int dummy_abort = 0;
@@ -415,16 +440,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // entry of magnitude 65536 or more, inf or NaN is reported as a
     // device-check error.
     const int ct = (warp - 10) * 32 + lane;
-    TileCursor cur;
-    cur.init(t0, t0, t1, per, cumT, pref, p);
     bool range_ok = true;
-    for (int j = 0; j < n; ++j, cur.advance()) {
-      const TileInfo& x = cur.x;
+    for (int j = 0; j < n; ++j) {
       const int st = j % kAttnStages;
       if (!mbar_wait_bounded(&kv_full[st], (j / kAttnStages) & 1, abort_flag, p.status)) break;
-      const bool tree_tile = x.lt >= x.tpre;
-      const int kbase = tree_tile ? (x.lt - x.tpre) * kAttnBN : x.lt * kAttnBN;
-      const int zero_from = tree_tile ? kAttnBN : min(kAttnBN, x.P - kbase);
+      const int zero_from = info_zero_from(stage_info[st]);
       uint4* vt = reinterpret_cast<uint4*>(smem + L::kVOff + st * L::kKVBytes);
       constexpr int kChunks = L::kKVBytes / 16, kPanelChunks = L::kPanelBytes / 16;
       constexpr int kUnroll = 8;
@@ -651,18 +671,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           break;
         }
         tc_fence_after();
-        const size_t prow = ((size_t)x.seg * p.slots + x.slot) * kAttnRows + m * kAttnMT + rl;
+        const size_t piece = (size_t)x.seg * p.slots + x.slot;
+        const size_t prow = piece * kAttnRows + m * kAttnMT + rl;
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        // column-group-major partial: a warp's 32 rows of one group of 4
+        // columns are 512 contiguous bytes
+        float4* dst = reinterpret_cast<float4*>(p.o_part) + piece * kAttnRows * (DH / 4) +
+                      m * kAttnMT + rl;
 #pragma unroll 1
         for (int ch = 0; ch < DH / 32; ++ch) {
           float o[32];
           tmem_ld32(tmem_o + lane_off + m * DH + ch * 32, o);
           if (valid) {
-            float4* dst = reinterpret_cast<float4*>(p.o_part + prow * DH + ch * 32);
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-              dst[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv,
-                                   o[4 * c + 3] * inv);
+              dst[(ch * 8 + c) * kAttnRows] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv,
+                                                          o[4 * c + 2] * inv, o[4 * c + 3] * inv);
           }
         }
         if (valid) p.lse_part[prow] = l_run > 0.f ? m_used + log2f(l_run) : -INFINITY;
@@ -681,12 +705,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-// merge the pieces of every query row; one warp per row
+// Merge the pieces of every query row.  A CTA takes 32 consecutive query rows
+// (global row = (b * Hkv + kvh) * R + r): lane = row while the partials are
+// read (each warp reads whole 512-byte runs of one column group), then the
+// rows go through shared memory so that each output row is written by 8
+// threads in contiguous pieces.
+constexpr int kCombineRows = 32;
+
 template <int DH>
 __global__ void __launch_bounds__(256)
     attn_combine_kernel(AttnParams p, void* __restrict__ out, int out_f32) {
+  constexpr int C4 = DH / 4;  // column groups of 4 floats
   __shared__ int cumT[kAttnMaxB + 1];
   __shared__ int sched_ok;
+  __shared__ float4 tile[kCombineRows][C4 + 1];
   if (threadIdx.x < 32) {
     const bool ok = build_schedule(p, cumT, nullptr);
     if (threadIdx.x == 0) sched_ok = ok ? 1 : 0;
@@ -694,47 +726,75 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   if (!sched_ok) return;  // reported by the attention kernel
   const int per = tiles_per_cta(cumT[p.B], p.grid);
-  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int total_rows = p.B * p.Hkv * p.R;
-  if (gw >= total_rows) return;
-  const int bh = gw / p.R;
-  const int r = gw - bh * p.R;
+  const int gr = blockIdx.x * kCombineRows + lane;
+  if (gr < total_rows) {
+    const int bh = gr / p.R;
+    const int r = gr - bh * p.R;
+    const int b = bh / p.Hkv;
+    const int kvh = bh - b * p.Hkv;
+    const int qg = r / kAttnRows, row = r - qg * kAttnRows;
+    const int P = p.prefix_len[b];
+    const int ntiles = (P + kAttnBN - 1) / kAttnBN + p.T_tree;
+    const int seg_start = cumT[b] + (kvh * p.n_qg + qg) * ntiles;
+    const int n_pieces = (seg_start + ntiles - 1) / per - seg_start / per + 1;
+    const size_t pbase = ((size_t)bh * p.n_qg + qg) * p.slots;
+    float M = -INFINITY;
+    for (int k = 0; k < n_pieces; ++k) M = fmaxf(M, p.lse_part[(pbase + k) * kAttnRows + row]);
+    constexpr int PER = C4 / 8;  // column groups per warp
+    float4 acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float wsum = 0.f;
+    for (int k = 0; k < n_pieces; ++k) {
+      const float lse = p.lse_part[(pbase + k) * kAttnRows + row];
+      const float w = lse == -INFINITY ? 0.f : exp2f(lse - M);
+      wsum += w;
+      const float4* src = reinterpret_cast<const float4*>(p.o_part) +
+                          (pbase + k) * kAttnRows * C4 + row;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const float4 v = src[(warp + 8 * e) * kAttnRows];
+        acc[e].x += w * v.x;
+        acc[e].y += w * v.y;
+        acc[e].z += w * v.z;
+        acc[e].w += w * v.w;
+      }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e)
+      tile[lane][warp + 8 * e] =
+          make_float4(acc[e].x * inv, acc[e].y * inv, acc[e].z * inv, acc[e].w * inv);
+  }
+  __syncthreads();
+  // writer: 8 threads per row, C4 / 8 consecutive column groups each
+  const int wr = threadIdx.x >> 3, part = threadIdx.x & 7;
+  const int ogr = blockIdx.x * kCombineRows + wr;
+  if (ogr >= total_rows) return;
+  const int bh = ogr / p.R;
+  const int r = ogr - bh * p.R;
   const int b = bh / p.Hkv;
   const int kvh = bh - b * p.Hkv;
-  const int qg = r / kAttnRows, row = r - qg * kAttnRows;
-  const int P = p.prefix_len[b];
-  const int ntiles = (P + kAttnBN - 1) / kAttnBN + p.T_tree;
-  const int seg_start = cumT[b] + (kvh * p.n_qg + qg) * ntiles;
-  const int n_pieces = (seg_start + ntiles - 1) / per - seg_start / per + 1;
-  const int seg = bh * p.n_qg + qg;
-  const size_t pbase = (size_t)seg * p.slots;
-  float M = -INFINITY;
-  for (int k = 0; k < n_pieces; ++k) M = fmaxf(M, p.lse_part[(pbase + k) * kAttnRows + row]);
-  constexpr int PER = DH / 32;
-  float acc[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  float wsum = 0.f;
-  for (int k = 0; k < n_pieces; ++k) {
-    const float lse = p.lse_part[(pbase + k) * kAttnRows + row];
-    const float w = lse == -INFINITY ? 0.f : exp2f(lse - M);
-    wsum += w;
-    const float* src = p.o_part + ((pbase + k) * kAttnRows + row) * DH + lane * PER;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] += w * src[e];
-  }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   const int node = r / p.G, g = r - node * p.G;
-  const size_t obase = (((size_t)b * p.N + node) * p.Hq + kvh * p.G + g) * DH + lane * PER;
+  constexpr int PER = C4 / 8;
+  const size_t obase = (((size_t)b * p.N + node) * p.Hq + kvh * p.G + g) * DH + part * PER * 4;
   if (out_f32) {
-    float* o = static_cast<float*>(out) + obase;
+    float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + obase);
 #pragma unroll
-    for (int e = 0; e < PER; ++e) o[e] = acc[e] * inv;
+    for (int e = 0; e < PER; ++e) o[e] = tile[wr][part * PER + e];
   } else {
-    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out) + obase;
+    uint2* o = reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + obase);
 #pragma unroll
-    for (int e = 0; e < PER; ++e) o[e] = __float2bfloat16_rn(acc[e] * inv);
+    for (int e = 0; e < PER; ++e) {
+      const float4 v = tile[wr][part * PER + e];
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+      o[e] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                        *reinterpret_cast<const uint32_t*>(&hi));
+    }
   }
 }
 
@@ -882,7 +942,8 @@ static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaSt
   medusa_status_t st = check_launch("tree_attention");
   if (st != MEDUSA_OK) return st;
   const int rows = p.B * p.Hkv * p.R;
-  attn_combine_kernel<DH><<<(rows + 7) / 8, 256, 0, stream>>>(p, out, out_f32);
+  attn_combine_kernel<DH>
+      <<<(rows + kCombineRows - 1) / kCombineRows, 256, 0, stream>>>(p, out, out_f32);
   return check_launch("tree_attention_combine");
 }
 
