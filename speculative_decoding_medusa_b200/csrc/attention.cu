@@ -577,17 +577,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // the tile's four mask words, picked without dynamic register indexing
       uint32_t tw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
       if (tree_tile) {
-        const int w0 = 4 * (x.lt - x.tpre);
+        const bool upper = x.lt > x.tpre;  // second tree tile: nodes 128..255
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (w == w0 + q) tw[q] = mw[w];
-        }
+        for (int q = 0; q < 4; ++q) tw[q] = upper ? mw[4 + q] : mw[q];
       }
-      auto visible = [&](int c) -> bool {  // c: key within the tile
-        return (kbase + c < key_end) && ((tw[c >> 5] >> (c & 31)) & 1u);
-      };
       // One pass over the tile, in two halves of 64 keys: the exponent base is
       // the running maximum m_used (log2 units); a half whose maximum exceeds
       // it by more than 2^8 (or the first half of a piece) moves the base,
@@ -604,9 +597,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int c = 0; c < 64; ++c) mx = fmaxf(mx, sv[c]);
         } else {
+          // visible keys of this half as a 64-bit mask: below the key end and
+          // set in the ancestor bitmask (the half's words are selected, not
+          // indexed, so the mask stays in registers)
+          const int nv = min(max(key_end - kbase - h * 64, 0), 64);
+          const uint64_t in_range = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
+          const uint32_t lo = h ? tw[2] : tw[0], hi = h ? tw[3] : tw[1];
+          const uint64_t vis = in_range & ((static_cast<uint64_t>(hi) << 32) | lo);
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
-            if (!visible(h * 64 + c)) sv[c] = -INFINITY;
+            if (!((vis >> c) & 1ull)) sv[c] = -INFINITY;
             mx = fmaxf(mx, sv[c]);
           }
         }
