@@ -50,6 +50,53 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 3-D tiled store from shared memory (bulk-group completion), c0 innermost
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0,
+                                             int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::
+                   "l"(reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the shared-memory sources of every committed store have been read
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// every committed store has been performed
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// paired fp32 arithmetic (two lanes in one 64-bit register, sm_100)
+__device__ __forceinline__ uint64_t f32x2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 struct AttnParams {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k_new;
@@ -75,11 +122,13 @@ struct AttnSmem {
   static constexpr int kKOff = kQOff + 2 * kQBytes;
   static constexpr int kVOff = kKOff + kAttnStages * kKVBytes;
   static constexpr int kBarOff = kVOff + kAttnStages * kKVBytes;
-  // kv_full[S], kv_empty[S], v_ready[S], q_full[2], s_full[2], p_full[2], p_empty[2], drain
-  static constexpr int kNumBars = 3 * kAttnStages + 2 + 2 + 2 + 2 + 1;
+  // kv_full[S], kv_empty[S], v_ready[S], q_full[2], s_full[2], p_full[2], p_empty[2], drain,
+  // copy_read[S]
+  static constexpr int kNumBars = 4 * kAttnStages + 2 + 2 + 2 + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kInfoOff = kMiscOff + 16;           // int info[kAttnStages]
-  static constexpr int kCumOff = kInfoOff + 16;            // int cumT[kAttnMaxB + 1]
+  static constexpr int kAuxOff = kInfoOff + 16;            // int {bh, row0}[kAttnStages]
+  static constexpr int kCumOff = kAuxOff + 32;             // int cumT[kAttnMaxB + 1]
   static constexpr int kPrefOff = kCumOff + (kAttnMaxB + 1) * 4;  // int P[kAttnMaxB]
   static constexpr int kBytes = kPrefOff + kAttnMaxB * 4;
   static constexpr int kAlloc = kBytes + 1024;
@@ -174,14 +223,20 @@ struct TileCursor {
 // producer: bit 0 first tile of a piece (the accumulator starts over, a new Q
 // tile is awaited), bit 1 both M tiles active, bits 8..15 keys of the tile
 // that are real (rows from there on are cleared in the converted V).
+// Bit 16: a tree tile of query group 0, whose K/V the converter also stores
+// into the caches (bit 17: the second tree tile, nodes 128..255).
 __device__ __forceinline__ int pack_stage_info(const TileInfo& x) {
   const bool tree_tile = x.lt >= x.tpre;
   const int zero_from = tree_tile ? kAttnBN : min(kAttnBN, x.P - x.lt * kAttnBN);
-  return (x.first ? 1 : 0) | (x.n_mt > 1 ? 2 : 0) | (zero_from << 8);
+  const bool copy = tree_tile && x.qg == 0;
+  return (x.first ? 1 : 0) | (x.n_mt > 1 ? 2 : 0) | (zero_from << 8) | (copy ? 1 << 16 : 0) |
+         (copy && x.lt > x.tpre ? 1 << 17 : 0);
 }
 __device__ __forceinline__ bool info_first(int w) { return (w & 1) != 0; }
 __device__ __forceinline__ bool info_two(int w) { return (w & 2) != 0; }
 __device__ __forceinline__ int info_zero_from(int w) { return (w >> 8) & 0xff; }
+__device__ __forceinline__ bool info_copy(int w) { return (w & (1 << 16)) != 0; }
+__device__ __forceinline__ bool info_second_tree(int w) { return (w & (1 << 17)) != 0; }
 
 // cumT[b] = tiles of all segments of sequences < b; returns false if some
 // prefix length is out of range.  Called by one full warp.
@@ -220,7 +275,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmKn,
-                        const __grid_constant__ CUtensorMap tmVn, AttnParams p) {
+                        const __grid_constant__ CUtensorMap tmVn,
+                        const __grid_constant__ CUtensorMap tmKs0,
+                        const __grid_constant__ CUtensorMap tmVs0,
+                        const __grid_constant__ CUtensorMap tmKs1,
+                        const __grid_constant__ CUtensorMap tmVs1, AttnParams p) {
   using L = AttnSmem<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -254,9 +313,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* p_full = s_full + 2;              // [m]
   uint64_t* p_empty = p_full + 2;             // [m]
   uint64_t* drain = p_empty + 2;
+  // [stage] a tree tile's cache stores have read the stage (one barrier per
+  // stage: the next copy from a stage needs every converter thread past this one)
+  uint64_t* copy_read = drain + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   int* stage_info = reinterpret_cast<int*>(smem + L::kInfoOff);
+  int* stage_aux = reinterpret_cast<int*>(smem + L::kAuxOff);  // tree copy: bh, first cache row
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kAttnStages; ++i) {
@@ -271,6 +334,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&p_empty[m], 1);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < kAttnStages; ++i) mbar_init(&copy_read[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -303,11 +367,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           break;
         // published with the stage (the kv_full arrive releases it): the
         // MMA and converter warps read it instead of walking the schedule
+        const int bh = x.b * p.Hkv + x.kvh;
         stage_info[st] = pack_stage_info(x);
+        stage_aux[2 * st] = bh;
+        stage_aux[2 * st + 1] = x.P + (x.lt - x.tpre) * kAttnBN;
         mbar_arrive_expect_tx(&kv_full[st], 2 * L::kKVBytes);
         uint8_t* kdst = smem + L::kKOff + st * L::kKVBytes;
         uint8_t* vdst = smem + L::kVOff + st * L::kKVBytes;
-        const int bh = x.b * p.Hkv + x.kvh;
 #pragma unroll
         for (int pn = 0; pn < L::kPanels; ++pn) {
           if (x.lt < x.tpre) {
@@ -441,11 +507,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // device-check error.
     const int ct = (warp - 10) * 32 + lane;
     bool range_ok = true;
+    uint32_t copy_par = 0;  // bit s: parity of the copies made from stage s
     for (int j = 0; j < n; ++j) {
       const int st = j % kAttnStages;
       if (!mbar_wait_bounded(&kv_full[st], (j / kAttnStages) & 1, abort_flag, p.status)) break;
-      const int zero_from = info_zero_from(stage_info[st]);
+      const int info = stage_info[st];
+      const int zero_from = info_zero_from(info);
       uint4* vt = reinterpret_cast<uint4*>(smem + L::kVOff + st * L::kKVBytes);
+      if (info_copy(info)) {
+        // tree tile of query group 0: its K/V (still bf16) go to cache rows
+        // P + node by bulk tensor stores, whose boxes hold exactly the
+        // tile's real nodes; V is converted once the stores have read it
+        if (ct == 0) {
+          const bool second = info_second_tree(info);
+          const CUtensorMap* mk = second ? &tmKs1 : &tmKs0;
+          const CUtensorMap* mv = second ? &tmVs1 : &tmVs0;
+          const int bh = stage_aux[2 * st], row0 = stage_aux[2 * st + 1];
+          const uint8_t* ks = smem + L::kKOff + st * L::kKVBytes;
+#pragma unroll
+          for (int pn = 0; pn < L::kPanels; ++pn) {
+            tma_store_3d(mk, ks + pn * L::kPanelBytes, pn * 64, row0, bh);
+            tma_store_3d(mv, reinterpret_cast<const uint8_t*>(vt) + pn * L::kPanelBytes, pn * 64,
+                         row0, bh);
+          }
+          bulk_commit_group();
+          bulk_wait_read_all();
+          mbar_arrive(&copy_read[st]);
+        } else if (!mbar_wait_bounded(&copy_read[st], (copy_par >> st) & 1u, abort_flag,
+                                      p.status)) {
+          break;
+        }
+        copy_par ^= 1u << st;
+      }
       constexpr int kChunks = L::kKVBytes / 16, kPanelChunks = L::kPanelBytes / 16;
       constexpr int kUnroll = 8;
       static_assert(kChunks % (64 * kUnroll) == 0, "V tile must split evenly over the converters");
@@ -477,6 +570,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(&v_ready[st]);
     }
+    if (ct == 0) bulk_wait_all();
     if (!range_ok) report(p.status, MEDUSA_ERR_DEVICE_CHECK);
   } else {
     // ---------------- softmax warpgroups ----------------
@@ -543,18 +637,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         l_run = 0.f;
         jj = 0;
       }
-      if (m == 0 && x.lt == x.tpre && x.qg == 0) {
-        // first tree tile of (b, kvh): the tree K/V into cache slots P + i
-        constexpr int CH = DH / 8;
-        const size_t kv_head_base = ((size_t)x.b * p.Hkv + x.kvh) * p.cap;
-        for (int e = rl; e < p.N * CH; e += 128) {
-          const int jn = e / CH, c = e - jn * CH;
-          const size_t src = (((size_t)x.b * p.N + jn) * p.Hkv + x.kvh) * DH + c * 8;
-          const size_t dst = (kv_head_base + x.P + jn) * DH + c * 8;
-          *reinterpret_cast<uint4*>(p.Kc + dst) = *reinterpret_cast<const uint4*>(p.k_new + src);
-          *reinterpret_cast<uint4*>(p.Vc + dst) = *reinterpret_cast<const uint4*>(p.v_new + src);
-        }
-      }
       if (!mbar_wait_bounded(&s_full[m], tcount & 1, abort_flag, p.status)) {
         ok = false;
         break;
@@ -592,11 +674,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int h = 0; h < 2; ++h) {
         float sv[64];
         load_half(h, sv);
-        float mx = -INFINITY;
-        if (full_tile) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) mx = fmaxf(mx, sv[c]);
-        } else {
+        if (!full_tile) {
           // visible keys of this half as a 64-bit mask: below the key end and
           // set in the ancestor bitmask (the half's words are selected, not
           // indexed, so the mask stays in registers)
@@ -605,12 +683,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t lo = h ? tw[2] : tw[0], hi = h ? tw[3] : tw[1];
           const uint64_t vis = in_range & ((static_cast<uint64_t>(hi) << 32) | lo);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
+          for (int c = 0; c < 64; ++c)
             if (!((vis >> c) & 1ull)) sv[c] = -INFINITY;
-            mx = fmaxf(mx, sv[c]);
-          }
         }
-        mx *= p.scale_log2;
+        // row maximum of the half: three-input max in four independent chains
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], sv[c], sv[c + 1]);
+        const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * p.scale_log2;
         const bool need = (m_used == -INFINITY) ? (mx != -INFINITY) : (mx > m_used + kRescaleLog2);
         if (__any_sync(0xffffffffu, need)) {
           const float new_m = need ? mx : m_used;
@@ -648,16 +728,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           moved = true;
         }
         const float nbase = m_used == -INFINITY ? 0.f : -m_used;
+        // weights 2^(s * scale - m) on key pairs: the exponent argument and the
+        // running sums use the paired fp32 instructions; four partial sums
+        const uint64_t scale2 = f32x2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nbase2 = f32x2_pack(nbase, nbase);
+        uint64_t part[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float a0 = ex2_approx(fmaf(sv[2 * e], p.scale_log2, nbase));
-          const float a1 = ex2_approx(fmaf(sv[2 * e + 1], p.scale_log2, nbase));
-          sum_tile += a0 + a1;
+          float x0, x1;
+          f32x2_unpack(f32x2_fma(f32x2_pack(sv[2 * e], sv[2 * e + 1]), scale2, nbase2), x0, x1);
+          const float a0 = ex2_approx(x0);
+          const float a1 = ex2_approx(x1);
+          part[e & 3] = f32x2_add(part[e & 3], f32x2_pack(a0, a1));
           const __half2 h2 = __floats2half2_rn(a0, a1);
           pk[e] = *reinterpret_cast<const uint32_t*>(&h2);
         }
         tmem_st32_u(srow + h * 32, pk);
+        float s0, s1;
+        f32x2_unpack(f32x2_add(f32x2_add(part[0], part[1]), f32x2_add(part[2], part[3])), s0, s1);
+        sum_tile += s0 + s1;
       }
       (void)moved;
       l_run += sum_tile;
@@ -931,14 +1021,23 @@ static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaSt
   const uint64_t dn[4] = {DH, (uint64_t)p.Hkv, (uint64_t)p.N, (uint64_t)p.B};
   const uint64_t sn[3] = {DH * 2, (uint64_t)p.Hkv * DH * 2, (uint64_t)p.N * p.Hkv * DH * 2};
   const uint32_t bn[4] = {64, 1, kAttnBN, 1};
+  // tree K/V stores into the caches: boxes of exactly the real nodes of the
+  // first and (N > 128) second tree tile
+  CUtensorMap mKs0, mVs0, mKs1, mVs1;
+  const uint32_t bs0[3] = {64, (uint32_t)(p.N < kAttnBN ? p.N : kAttnBN), 1};
+  const uint32_t bs1[3] = {64, (uint32_t)(p.N > kAttnBN ? p.N - kAttnBN : 1), 1};
   if (!make_tmap_bf16(&mK, p.Kc, 3, dc, sc, bc) || !make_tmap_bf16(&mV, p.Vc, 3, dc, sc, bc) ||
-      !make_tmap_bf16(&mKn, p.k_new, 4, dn, sn, bn) || !make_tmap_bf16(&mVn, p.v_new, 4, dn, sn, bn))
+      !make_tmap_bf16(&mKn, p.k_new, 4, dn, sn, bn) ||
+      !make_tmap_bf16(&mVn, p.v_new, 4, dn, sn, bn) ||
+      !make_tmap_bf16(&mKs0, p.Kc, 3, dc, sc, bs0) || !make_tmap_bf16(&mVs0, p.Vc, 3, dc, sc, bs0) ||
+      !make_tmap_bf16(&mKs1, p.Kc, 3, dc, sc, bs1) || !make_tmap_bf16(&mVs1, p.Vc, 3, dc, sc, bs1))
     return fail(MEDUSA_ERR_CUDA, "tree_attention: cuTensorMapEncodeTiled failed");
   if (cudaFuncSetAttribute(tree_attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            L::kAlloc) != cudaSuccess)
     return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(tree_attention) failed");
   p.grid = device_sm_count();  // persistent: one CTA per SM
-  tree_attn_tc_kernel<DH><<<p.grid, kAttnThreads, L::kAlloc, stream>>>(mK, mV, mKn, mVn, p);
+  tree_attn_tc_kernel<DH><<<p.grid, kAttnThreads, L::kAlloc, stream>>>(mK, mV, mKn, mVn, mKs0,
+                                                                        mVs0, mKs1, mVs1, p);
   medusa_status_t st = check_launch("tree_attention");
   if (st != MEDUSA_OK) return st;
   const int rows = p.B * p.Hkv * p.R;
