@@ -50,6 +50,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 5-D tiled load (no multicast), c0 innermost
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 3-D tiled store from shared memory (bulk-group completion), c0 innermost
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0,
                                              int c1, int c2) {
@@ -108,6 +119,7 @@ struct AttnParams {
   float* o_part;    // [n_seg, slots, DH / 4, 256] groups of 4 floats
   float* lse_part;  // [n_seg, slots, 256]
   int B, N, Hq, Hkv, G, R, n_qg, T_tree, slots, cap, max_prefix, words, grid;
+  int q_tma;  // Q tiles by bulk tensor loads (G divides 128)
   float scale_log2;
   int32_t* status;
 };
@@ -279,7 +291,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         const __grid_constant__ CUtensorMap tmKs0,
                         const __grid_constant__ CUtensorMap tmVs0,
                         const __grid_constant__ CUtensorMap tmKs1,
-                        const __grid_constant__ CUtensorMap tmVs1, AttnParams p) {
+                        const __grid_constant__ CUtensorMap tmVs1,
+                        const __grid_constant__ CUtensorMap tmQ, AttnParams p) {
   using L = AttnSmem<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -328,7 +341,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&v_ready[i], 64);
     }
     for (int m = 0; m < 2; ++m) {
-      mbar_init(&q_full[m], 128);
+      mbar_init(&q_full[m], p.q_tma ? 1 : 128);
       mbar_init(&s_full[m], 1);
       mbar_init(&p_full[m], 128);
       mbar_init(&p_empty[m], 1);
@@ -581,8 +594,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t srow = tmem_s + lane_off + m * kAttnBN;
     uint8_t* qtile = smem + L::kQOff + m * L::kQBytes;
 
-    // Q rows of a segment into the swizzled K-major tile (zeros past R)
+    // Q rows of a segment into the swizzled K-major tile (zeros past R).
+    // When G divides 128 the tile is one box of the query tensor seen as
+    // [B][N][Hkv][G][DH] (rows = node-major (node, g) pairs, nodes past N
+    // zero-filled), fetched by one bulk tensor load per 64-column panel.
     auto load_q = [&](const TileInfo& x) {
+      if (p.q_tma) {
+        if (rl == 0) {
+          const int node0 = (x.qg * kAttnRows + m * kAttnMT) / p.G;
+          mbar_arrive_expect_tx(&q_full[m], L::kQBytes);
+#pragma unroll
+          for (int pn = 0; pn < L::kPanels; ++pn)
+            tma_load_5d(qtile + pn * (kAttnMT * 128), &tmQ, &q_full[m], pn * 64, 0, x.kvh, node0,
+                        x.b);
+        }
+        return;
+      }
       const int r = x.qg * kAttnRows + m * kAttnMT + rl;
       const bool valid = r < p.R;
       const int node = valid ? r / p.G : 0;
@@ -1026,6 +1053,16 @@ static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaSt
   CUtensorMap mKs0, mVs0, mKs1, mVs1;
   const uint32_t bs0[3] = {64, (uint32_t)(p.N < kAttnBN ? p.N : kAttnBN), 1};
   const uint32_t bs1[3] = {64, (uint32_t)(p.N > kAttnBN ? p.N - kAttnBN : 1), 1};
+  // queries as [B][N][Hkv][G][DH]: a box of 64 columns x G heads x 128 / G nodes
+  CUtensorMap mQ;
+  p.q_tma = (kAttnMT % p.G == 0) ? 1 : 0;
+  const uint64_t dq[5] = {DH, (uint64_t)p.G, (uint64_t)p.Hkv, (uint64_t)p.N, (uint64_t)p.B};
+  const uint64_t sq[4] = {DH * 2, (uint64_t)p.G * DH * 2, (uint64_t)p.Hq * DH * 2,
+                          (uint64_t)p.N * p.Hq * DH * 2};
+  const uint32_t bq[5] = {64, (uint32_t)(p.q_tma ? p.G : 1), 1,
+                          (uint32_t)(p.q_tma ? kAttnMT / p.G : 1), 1};
+  if (!make_tmap_bf16(&mQ, p.q, 5, dq, sq, bq))
+    return fail(MEDUSA_ERR_CUDA, "tree_attention: cuTensorMapEncodeTiled failed");
   if (!make_tmap_bf16(&mK, p.Kc, 3, dc, sc, bc) || !make_tmap_bf16(&mV, p.Vc, 3, dc, sc, bc) ||
       !make_tmap_bf16(&mKn, p.k_new, 4, dn, sn, bn) ||
       !make_tmap_bf16(&mVn, p.v_new, 4, dn, sn, bn) ||
@@ -1037,7 +1074,7 @@ static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaSt
     return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(tree_attention) failed");
   p.grid = device_sm_count();  // persistent: one CTA per SM
   tree_attn_tc_kernel<DH><<<p.grid, kAttnThreads, L::kAlloc, stream>>>(mK, mV, mKn, mVn, mKs0,
-                                                                        mVs0, mKs1, mVs1, p);
+                                                                        mVs0, mKs1, mVs1, mQ, p);
   medusa_status_t st = check_launch("tree_attention");
   if (st != MEDUSA_OK) return st;
   const int rows = p.B * p.Hkv * p.R;

@@ -91,6 +91,8 @@ def test_tiny_fp32():
     (3, 8, 1, 128, (1, 200), "sparse16", 2),       # MQA, tiny prefixes
     (2, 16, 2, 128, (0, 0), "sparse64", 3),        # empty prefix: tree only
     (1, 8, 8, 128, (1500, 1500), "dense256", 4),   # 256 nodes, 8 mask words
+    (2, 6, 2, 128, (50, 300), "sparse16", 5),      # G 3: Q rows gathered by threads
+    (1, 16, 1, 64, (200, 200), "sparse64", 6),     # G 16: four query groups of 256 rows
 ])
 def test_bf16_small(B, Hq, Hkv, dh, ctx, tree, seed):
     if tree == "sparse64":
