@@ -89,18 +89,15 @@ __device__ __forceinline__ float load1<float>(const float* p) {
   return *p;
 }
 
-// One warp per (row, 4096-token chunk): every lane issues all its 16-byte
-// loads at once, then the warp reduces with shuffles only.
+// One warp per (row, 4096-token chunk) work item: every lane issues all its
+// 16-byte loads at once, then the warp reduces with shuffles only.
 template <typename T, bool TYPICAL>
-__global__ void __launch_bounds__(kRowWarps * 32)
-    verify_rows_kernel(const T* __restrict__ logits, int V, int n_chunks, long long n_items,
-                       float inv_T, RowPart* __restrict__ part, int32_t* status) {
+__device__ __forceinline__ void verify_item(const T* __restrict__ logits, int V, int n_chunks,
+                                            long long item, int lane, float inv_T,
+                                            RowPart* __restrict__ part, int32_t* status) {
   using E = Elt<T>;
   constexpr int EV = E::kPerVec;
   constexpr int NL = kVChunk / (32 * EV);  // loads per lane
-  const int lane = threadIdx.x & 31;
-  const long long item = (long long)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
-  if (item >= n_items) return;  // whole warp
   const long long row = item / n_chunks;
   const int c = static_cast<int>(item - row * n_chunks);
   const T* base = logits + row * V;
@@ -122,10 +119,8 @@ __global__ void __launch_bounds__(kRowWarps * 32)
     __nv_bfloat162 m2 = __halves2bfloat162(__ushort_as_bfloat16(0xFF80u), __ushort_as_bfloat16(0xFF80u));
 #pragma unroll
     for (int r = 0; r < NL; ++r) {
-      const uint32_t* w = &raw[r].x;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        m2 = __hmax2_nan(m2, *reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+      const __nv_bfloat162* w = reinterpret_cast<const __nv_bfloat162*>(&raw[r].x);
+      m2 = __hmax2_nan(m2, __hmax2_nan(__hmax2_nan(w[0], w[1]), __hmax2_nan(w[2], w[3])));
     }
     const float lo_f = __low2float(m2), hi_f = __high2float(m2);
     bool nan = (lo_f != lo_f) || (hi_f != hi_f);
@@ -135,21 +130,27 @@ __global__ void __launch_bounds__(kRowWarps * 32)
     if (__any_sync(0xffffffffu, nan)) {
       if (lane == 0) report(status, MEDUSA_ERR_DEVICE_CHECK);
     }
-    // bf16 bit pattern of M; +0 and -0 are equal values, so a zero maximum
-    // matches either sign
-    const uint32_t mb = __float_as_uint(M) >> 16;
-    const bool zero = (mb & 0x7FFFu) == 0u;
-    const uint32_t pat = zero ? 0u : (mb | (mb << 16));
-    const uint32_t msk = zero ? 0x7FFF7FFFu : 0xFFFFFFFFu;
+    // first index holding M: a floating equality (so +0 and -0 both match
+    // a zero maximum) on each load's packed maximum (recomputed: keeping
+    // them would cost registers and so loads in flight), then inside the
+    // first load that holds M
+    const __nv_bfloat162 M2 = __float2bfloat162_rn(M);  // exact: M is a bf16 value
     int idx = 0x7fffffff;
 #pragma unroll
-    for (int r = 0; r < NL; ++r) {
-      const int e0 = v0 + (r * 32 + lane) * EV;
-      const uint32_t* w = &raw[r].x;
+    for (int r = NL - 1; r >= 0; --r) {
+      const __nv_bfloat162* w = reinterpret_cast<const __nv_bfloat162*>(&raw[r].x);
+      const __nv_bfloat162 e =
+          __heq2(__hmax2(__hmax2(w[0], w[1]), __hmax2(w[2], w[3])), M2);
+      if (*reinterpret_cast<const uint32_t*>(&e) != 0u) {  // rare: the load holding M
+        int k = 8;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t eq = __vcmpeq2(w[q] & msk, pat);
-        if (idx == 0x7fffffff && eq != 0u) idx = e0 + 2 * q + ((eq & 0xFFFFu) ? 0 : 1);
+        for (int q = 3; q >= 0; --q) {
+          const __nv_bfloat162 eq = __heq2(w[q], M2);
+          const uint32_t eb = *reinterpret_cast<const uint32_t*>(&eq);
+          if (eb & 0xFFFF0000u) k = 2 * q + 1;
+          if (eb & 0x0000FFFFu) k = 2 * q;
+        }
+        idx = v0 + (r * 32 + lane) * EV + k;
       }
     }
 #pragma unroll
@@ -223,10 +224,29 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   }
 }
 
+// Persistent grid (a few CTAs per SM): each warp takes items warp, warp +
+// total warps, ... so that no partial last wave of CTAs is left.
+template <typename T, bool TYPICAL>
+__global__ void __launch_bounds__(kRowWarps * 32,
+                                  (std::is_same<T, __nv_bfloat16>::value && !TYPICAL) ? 3 : 1)
+    verify_rows_kernel(const T* __restrict__ logits, int V, int n_chunks, long long n_items,
+                       float inv_T, RowPart* __restrict__ part, int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  for (long long item = (long long)blockIdx.x * kRowWarps + (threadIdx.x >> 5); item < n_items;
+       item += (long long)gridDim.x * kRowWarps)
+    verify_item<T, TYPICAL>(logits, V, n_chunks, item, lane, inv_T, part, status);
+}
+
+// One CTA of kPathThreads per sequence.  The chunk records of node i are
+// merged by a group of tpn consecutive threads (tpn a power of two, tpn * N <=
+// kPathThreads), each taking every tpn-th chunk, then shuffles within the
+// group; the path logic runs on threads 0..N-1.
+constexpr int kPathThreads = 1024;
+
 template <typename T>
-__global__ void __launch_bounds__(MEDUSA_MAX_NODES)
+__global__ void __launch_bounds__(kPathThreads)
     verify_path_kernel(const T* __restrict__ logits, const RowPart* __restrict__ part,
-                       int n_chunks, const int32_t* __restrict__ cand_ids,
+                       int n_chunks, int tpn, const int32_t* __restrict__ cand_ids,
                        const int32_t* __restrict__ parent, const int32_t* __restrict__ depth,
                        int N, int max_depth, int V, int typical, float inv_T, float eps,
                        float delta, int32_t* __restrict__ accept_len,
@@ -256,36 +276,67 @@ __global__ void __launch_bounds__(MEDUSA_MAX_NODES)
     const int dp = s_depth[i];
     const bool ok = (i == 0) ? (pa == -1 && dp == 0)
                              : (pa >= 0 && pa < i && dp == s_depth[pa] + 1 && dp <= max_depth);
-    // merge the chunks of row (b, i)
-    const RowPart* rp = part + ((size_t)b * N + i) * n_chunks;
+    if (!ok) atomicOr(&s_bad, 1);
+  }
+  {
+    // merge the chunks of row (b, node): this thread's share, then the group
+    const int node = i / tpn, sub = i - node * tpn;
+    const bool active = node < N;
+    const RowPart* rp = part + ((size_t)b * N + (active ? node : 0)) * n_chunks;
     float bv = -INFINITY;
     int bi = 0x7fffffff;
-    float M = -INFINITY;
-#pragma unroll 4
-    for (int c = 0; c < n_chunks; ++c) {
-      const RowPart q = rp[c];
-      if (better(q.maxz, q.idx, bv, bi)) {
-        bv = q.maxz;
-        bi = q.idx;
-      }
-    }
-    s_g[i] = bi;
-    if (typical) {
-      M = bv * inv_T;
-      float S = 0.f, Tt = 0.f;
-      for (int c = 0; c < n_chunks; ++c) {
+    float Mt = -INFINITY, S = 0.f, Tt = 0.f;  // sums relative to exp(Mt)
+    if (active) {
+      for (int c = sub; c < n_chunks; c += tpn) {
         const RowPart q = rp[c];
-        const float w = expf(q.maxz * inv_T - M);
-        S += q.s * w;
-        Tt += q.t * w;
+        if (better(q.maxz, q.idx, bv, bi)) {
+          bv = q.maxz;
+          bi = q.idx;
+        }
+        if (typical) {
+          const float mq = q.maxz * inv_T;
+          if (mq > Mt) {
+            const float w = Mt == -INFINITY ? 0.f : expf(Mt - mq);
+            S = S * w + q.s;
+            Tt = Tt * w + q.t;
+            Mt = mq;
+          } else if (mq != -INFINITY) {
+            const float w = expf(mq - Mt);
+            S += q.s * w;
+            Tt += q.t * w;
+          }
+        }
       }
-      const float lse = M + logf(S);
-      const float H = lse - Tt / S;
-      const float thr = fminf(eps, delta * expf(-H));
-      s_lse[i] = lse;
-      s_logthr[i] = thr > 0.f ? logf(thr) : -INFINITY;
     }
-    if (!ok) atomicOr(&s_bad, 1);
+    for (int o = 1; o < tpn; o <<= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (better(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+      if (typical) {
+        const float oM = __shfl_xor_sync(0xffffffffu, Mt, o);
+        const float oS = __shfl_xor_sync(0xffffffffu, S, o);
+        const float oT = __shfl_xor_sync(0xffffffffu, Tt, o);
+        const float nM = fmaxf(Mt, oM);
+        const float wa = Mt == -INFINITY ? 0.f : expf(Mt - nM);
+        const float wb = oM == -INFINITY ? 0.f : expf(oM - nM);
+        S = S * wa + oS * wb;
+        Tt = Tt * wa + oT * wb;
+        Mt = nM;
+      }
+    }
+    if (active && sub == 0) {
+      s_g[node] = bi;
+      if (typical) {
+        const float lse = Mt + logf(S);
+        const float H = lse - Tt / S;
+        const float thr = fminf(eps, delta * expf(-H));
+        s_lse[node] = lse;
+        s_logthr[node] = thr > 0.f ? logf(thr) : -INFINITY;
+      }
+    }
   }
   __syncthreads();
   if (s_bad) {
@@ -337,6 +388,22 @@ __global__ void __launch_bounds__(MEDUSA_MAX_NODES)
   }
 }
 
+// CTAs for the persistent row kernel: as many as stay resident, fewer when
+// there are fewer work items
+template <typename K>
+static unsigned rows_grid(K kernel, long long n_items) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kRowWarps * 32, 0) !=
+          cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  const long long resident = (long long)per_sm * device_sm_count();
+  const long long need = (n_items + kRowWarps - 1) / kRowWarps;
+  return (unsigned)(need < resident ? need : resident);
+}
+
 size_t verify_accept_workspace_size(int B, int N, int V) {
   const size_t n_chunks = (size_t)(V + kVChunk - 1) / kVChunk;
   return align256((size_t)B * N * n_chunks * sizeof(RowPart));
@@ -353,34 +420,41 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
   const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
   const float inv_T = typical ? 1.0f / temperature : 1.0f;
   const long long n_items = (long long)B * N * n_chunks;
-  const unsigned grid = (unsigned)((n_items + kRowWarps - 1) / kRowWarps);
+  int tpn = 1;  // threads merging one node's chunks
+  while (tpn < 32 && tpn * 2 * N <= kPathThreads && tpn < n_chunks) tpn *= 2;
   if (dt == MEDUSA_BF16) {
     const __nv_bfloat16* lg = static_cast<const __nv_bfloat16*>(logits);
-    if (typical)
-      verify_rows_kernel<__nv_bfloat16, true><<<grid, kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items,
-                                                                                 inv_T, part, status);
-    else
-      verify_rows_kernel<__nv_bfloat16, false><<<grid, kRowWarps * 32, 0, stream>>>(
-          lg, V, n_chunks, n_items, inv_T, part, status);
+    if (typical) {
+      auto k = verify_rows_kernel<__nv_bfloat16, true>;
+      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T,
+                                                              part, status);
+    } else {
+      auto k = verify_rows_kernel<__nv_bfloat16, false>;
+      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T,
+                                                              part, status);
+    }
     medusa_status_t st = check_launch("verify_rows");
     if (st != MEDUSA_OK) return st;
-    verify_path_kernel<__nv_bfloat16><<<B, MEDUSA_MAX_NODES, 0, stream>>>(
-        lg, part, n_chunks, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
+    verify_path_kernel<__nv_bfloat16><<<B, kPathThreads, 0, stream>>>(
+        lg, part, n_chunks, tpn, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
         typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
         status);
     return check_launch("verify_path");
   }
   const float* lg = static_cast<const float*>(logits);
-  if (typical)
-    verify_rows_kernel<float, true><<<grid, kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T, part,
-                                                                      status);
-  else
-    verify_rows_kernel<float, false><<<grid, kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T,
-                                                                       part, status);
+  if (typical) {
+    auto k = verify_rows_kernel<float, true>;
+    k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T, part,
+                                                            status);
+  } else {
+    auto k = verify_rows_kernel<float, false>;
+    k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T, part,
+                                                            status);
+  }
   medusa_status_t st = check_launch("verify_rows");
   if (st != MEDUSA_OK) return st;
-  verify_path_kernel<float><<<B, MEDUSA_MAX_NODES, 0, stream>>>(
-      lg, part, n_chunks, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
+  verify_path_kernel<float><<<B, kPathThreads, 0, stream>>>(
+      lg, part, n_chunks, tpn, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
       typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
       status);
   return check_launch("verify_path");
