@@ -23,8 +23,12 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <cooperative_groups.h>
+
 #include "abi_internal.h"
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace medusa {
 
@@ -291,25 +295,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ----------------------------------------------------------------------------
 // top-k merge: best kmax of C candidates per row
+//
+// A row is shared by a cluster of kMergeCtas CTAs of kMergeWarps warps: warp w
+// of CTA r walks the candidate chunks (w * kMergeCtas + r) * 32, + 32 * all
+// warps, keeping a sorted best-32 list filtered by its kmax-th entry.  The
+// warps of a CTA merge pairwise through shared memory (three rounds), then CTA
+// 0 of the cluster reads the other CTAs' lists from distributed shared memory
+// and merges them.
 // ----------------------------------------------------------------------------
-constexpr int kMergeWarps = 32;
-constexpr int kMergeUnroll = 4;  // 32-candidate chunks each warp has in flight
+constexpr int kMergeWarps = 8;
+constexpr int kMergeCtas = 8;    // cluster size (portable)
+constexpr int kMergeUnroll = 2;  // 32-candidate chunks each warp has in flight
 
-__global__ void __launch_bounds__(kMergeWarps * 32)
+__global__ void __cluster_dims__(kMergeCtas, 1, 1) __launch_bounds__(kMergeWarps * 32)
     topk_merge_kernel(const float* __restrict__ vals, const int32_t* __restrict__ ids, long long C,
                       int kmax, int32_t* __restrict__ out_ids, float* __restrict__ out_vals) {
   __shared__ float sv[kMergeWarps][32];
   __shared__ int si[kMergeWarps][32];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = static_cast<int>(cluster.block_rank());
+  const long long row = blockIdx.x / kMergeCtas;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const size_t base = (size_t)blockIdx.x * C;
+  const size_t base = (size_t)row * C;
+  constexpr long long kStride = (long long)kMergeCtas * kMergeWarps * 32 * kMergeUnroll;
   // running best-32 of this warp, sorted, and its kmax-th entry as a filter
   float rv = -INFINITY;
   int ri = 0x7fffffff;
   float tv = -INFINITY;
   int ti = 0x7fffffff;
-  for (long long c = (long long)warp * 32 * kMergeUnroll; c < C;
-       c += (long long)kMergeWarps * 32 * kMergeUnroll) {
+  for (long long c = (long long)(warp * kMergeCtas + crank) * 32 * kMergeUnroll; c < C;
+       c += kStride) {
     float v[kMergeUnroll];
     int i[kMergeUnroll];
 #pragma unroll
@@ -332,16 +348,33 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
       }
     }
   }
+  // warps of the CTA: pairwise rounds
   sv[warp][lane] = rv;
   si[warp][lane] = ri;
-  __syncthreads();
-  if (warp == 0) {
-    for (int w = 1; w < kMergeWarps; ++w) warp_merge_top32(rv, ri, sv[w][lane], si[w][lane]);
-    if (lane < kmax) {
-      out_ids[(size_t)blockIdx.x * kmax + lane] = ri;
-      out_vals[(size_t)blockIdx.x * kmax + lane] = rv;
+#pragma unroll
+  for (int s = kMergeWarps / 2; s > 0; s >>= 1) {
+    __syncthreads();
+    if (warp < s) {
+      warp_merge_top32(rv, ri, sv[warp + s][lane], si[warp + s][lane]);
+      sv[warp][lane] = rv;
+      si[warp][lane] = ri;
     }
   }
+  // CTAs of the cluster: CTA 0 merges the others' lists (row 0 of their sv/si)
+  cluster.sync();
+  if (crank == 0 && warp == 0) {
+    for (int r = 1; r < kMergeCtas; ++r) {
+      const float* rsv = cluster.map_shared_rank(&sv[0][0], r);
+      const int* rsi = cluster.map_shared_rank(&si[0][0], r);
+      warp_merge_top32(rv, ri, rsv[lane], rsi[lane]);
+    }
+    if (lane < kmax) {
+      out_ids[(size_t)row * kmax + lane] = ri;
+      out_vals[(size_t)row * kmax + lane] = rv;
+    }
+  }
+  // no CTA leaves while CTA 0 may still read its shared memory
+  cluster.sync();
 }
 
 // ----------------------------------------------------------------------------
@@ -482,8 +515,8 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
         y, static_cast<const float*>(W2), B, d, V, K, z);
     st = check_launch("heads_f32_w2");
     if (st != MEDUSA_OK) return st;
-    topk_merge_kernel<<<B * K, kMergeWarps * 32, 0, stream>>>(z, nullptr, V, kmax, topk_ids,
-                                                              topk_vals);
+    topk_merge_kernel<<<B * K * kMergeCtas, kMergeWarps * 32, 0, stream>>>(z, nullptr, V, kmax,
+                                                                            topk_ids, topk_vals);
     return check_launch("topk_merge");
   }
 
@@ -525,7 +558,7 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
   st = launch_gemm_nb<kModeW2>(nb2, mA2, mB2, p2, stream);
   if (st != MEDUSA_OK) return st;
 
-  topk_merge_kernel<<<B * K, kMergeWarps * 32, 0, stream>>>(
+  topk_merge_kernel<<<B * K * kMergeCtas, kMergeWarps * 32, 0, stream>>>(
       part_vals, part_ids, (long long)p2.tiles_per_head * kmax, kmax, topk_ids, topk_vals);
   return check_launch("topk_merge");
 }
