@@ -355,6 +355,29 @@ def kv_compact(Kc: np.ndarray, Vc: np.ndarray, prefix_len: np.ndarray,
 # ---------------------------------------------------------------------------
 
 
+def lmhead_verify(hidden: np.ndarray, lm_head: np.ndarray, cand: np.ndarray,
+                  parent: np.ndarray, depth: np.ndarray, max_depth: int,
+                  accept_mode: str = "greedy", temperature: float = 1.0,
+                  eps: float = 0.09, delta: float = 0.3) -> Dict[str, np.ndarray]:
+    """Verification from the base model's last hidden states of the tree
+    nodes instead of from materialised logits.
+
+    The verify logits of node n of sequence b are lm_head(hidden[b, n])
+    ([GLOSS-TREE]: one forward pass scores every node; [GLOSS-HEADS]: the
+    base model's next-token distribution is lm_head of its last hidden
+    state).  hidden [B, N, d], lm_head [V, d].  Returns the verify outputs
+    plus the logits [B, N, V] (fp64)."""
+    hidden = np.asarray(hidden, np.float64)
+    B, N, d = hidden.shape
+    logits = lm_head_logits(hidden.reshape(B * N, d), lm_head).reshape(B, N, -1)
+    if accept_mode == "greedy":
+        res = verify_greedy(logits, cand, parent, depth, max_depth)
+    else:
+        res = verify_typical(logits, cand, parent, depth, max_depth, temperature, eps, delta)
+    res["logits"] = logits
+    return res
+
+
 def decode_verify_step(inp: Dict[str, np.ndarray], tree: Dict[str, np.ndarray],
                        kmax: int, accept_mode: str = "greedy", temperature: float = 1.0,
                        eps: float = 0.09, delta: float = 0.3,

@@ -419,3 +419,54 @@ def test_kv_compact_literal_and_out_of_place_equivalence():
             np.testing.assert_array_equal(res["Kc"][0, :, 6 + j], Kc[0, :, 6 + n])
             np.testing.assert_array_equal(res["Vc"][0, :, 6 + j], Vc[0, :, 6 + n])
         np.testing.assert_array_equal(res["Kc"][0, :, 6 + L + 1:], Kc[0, :, 6 + L + 1:])
+
+
+# ----------------------------------------------------------------------------
+# Verification from hidden states (lm_head fused in front of the verify)
+# ----------------------------------------------------------------------------
+
+
+def test_lmhead_verify_planted_basis_rows():
+    """lm_head rows are scaled unit vectors (V = 300 < d = 320, so a transposed
+    operand cannot even multiply) and every node's hidden state is the unit
+    vector of the token its model should choose: the glossary example of the
+    greedy literal test is reproduced, and the logits are the planted values."""
+    spec = W.cartesian_tree([2, 3])
+    V, d = 300, 320
+    lm = np.zeros((V, d))
+    lm[np.arange(V), np.arange(V)] = 1.0 + np.arange(V) / 1000.0
+    cand = np.array([[7, 100, 101, 200, 201, 202, 200, 201, 202]], dtype=np.int32)
+    want = {0: 101, 2: 201, 7: 42}
+    hidden = np.zeros((1, 9, d))
+    for n in range(9):
+        hidden[0, n, want.get(n, 250 + n)] = 1.0
+    res = O.lmhead_verify(hidden, lm, cand, spec.parent, spec.depth, 2)
+    assert res["accept_len"].tolist() == [2]
+    assert res["accepted_nodes"].tolist() == [[0, 2, 7]]
+    assert res["accepted_tokens"].tolist() == [[101, 201, 42]]
+    assert res["logits"].shape == (1, 9, V)
+    assert res["logits"][0, 2, 201] == 1.0 + 201 / 1000.0
+    assert np.count_nonzero(res["logits"]) == 9
+
+
+def test_lmhead_verify_logits_bruteforce_and_typical_mode():
+    rng = np.random.default_rng(11)
+    B, N, d, V = 2, 4, 5, 7
+    spec = W.cartesian_tree([3])
+    hidden = rng.standard_normal((B, N, d))
+    lm = rng.standard_normal((V, d))
+    cand = rng.integers(0, V, size=(B, N)).astype(np.int32)
+    res = O.lmhead_verify(hidden, lm, cand, spec.parent, spec.depth, 1, "typical", 0.8, 0.3, 0.5)
+    for b in range(B):
+        for n in range(N):
+            for v in range(V):
+                s = 0.0
+                for j in range(d):
+                    s += hidden[b, n, j] * lm[v, j]
+                assert abs(res["logits"][b, n, v] - s) < 1e-12
+    # the typical decision depends only on the logits: same result as the
+    # logits-level verify on the brute-force logits
+    z = np.einsum("bnj,vj->bnv", hidden, lm)
+    ref = O.verify_typical(z, cand, spec.parent, spec.depth, 1, 0.8, 0.3, 0.5)
+    assert res["accept_len"].tolist() == ref["accept_len"].tolist()
+    assert res["bonus"].tolist() == ref["bonus"].tolist()
