@@ -312,6 +312,45 @@ MEDUSA_API medusa_status_t medusa_verify_accept_noalloc(
     int32_t* accept_len, int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
     int32_t* dev_status, void* stream);
 
+/* ------------------------------------------------------------------------
+ * medusa_lmhead_verify
+ *
+ * "Medusa Heads" glossary, "Attention arborescente et acceptation": one
+ * forward pass scores every tree node, and the longest branch the base model
+ * agrees with is kept; "Comment les têtes prédisent les tokens suivants": the
+ * base model's next-token scores at a node are its lm_head applied to the
+ * node's last hidden state.
+ *
+ * The verification of medusa_verify_accept, with the verify logits never
+ * materialised: logits[b][i][v] = sum_j lm_head[v][j] * hidden[b][i][j]
+ * (bf16 inputs, fp32 accumulation on the tensor cores), reduced tile by tile
+ * to each node's argmax (greedy) or to its log-sum-exp and entropy
+ * (typical); then exactly the acceptance rules of medusa_verify_accept.  In
+ * typical mode the candidate's logit at its parent is recomputed as one dot
+ * product (fp32), so near the threshold its decision may differ from one
+ * taken on the GEMM's own value by the rounding of the two sums.
+ *
+ * Inputs (device): hidden [B, N, d] bf16 (node rows in tree order); lm_head
+ *   [V, d] bf16 (torch Linear layout, no bias); cand_ids [B, N] int32; tree.
+ * Outputs (device): accept_len [B], accepted_nodes [B, max_depth+1],
+ *   accepted_tokens [B, max_depth+1], bonus [B] (int32, as
+ *   medusa_verify_accept).  logits: optional [B, N, V] fp32 copy of the
+ *   logits for checking (NULL in normal use; it adds B*N*V*4 bytes of writes).
+ * dt must be MEDUSA_BF16 (MEDUSA_ERR_UNSUPPORTED otherwise).
+ * Workspace: medusa_lmhead_verify_workspace_size(...) bytes, 256-byte
+ *   aligned; the size depends on the current device's multiprocessor count.
+ * Limits: d a positive multiple of 64; N <= MEDUSA_MAX_NODES; B * N <= 65535;
+ *   hidden and lm_head 16-byte aligned; temperature > 0 (typical).
+ * Device checks: a NaN logit, a candidate id outside [0, V).
+ * ---------------------------------------------------------------------- */
+MEDUSA_API size_t medusa_lmhead_verify_workspace_size(int B, int N, int d, int V);
+MEDUSA_API medusa_status_t medusa_lmhead_verify(
+    const void* hidden, const void* lm_head, medusa_dtype_t dt, const int32_t* cand_ids,
+    const medusa_tree_t* tree, int B, int d, int V, medusa_accept_t mode, float temperature,
+    float eps, float delta, int32_t* accept_len, int32_t* accepted_nodes,
+    int32_t* accepted_tokens, int32_t* bonus, float* logits, void* ws, size_t ws_bytes,
+    int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,6 +36,7 @@ EXPORTS = (
     "medusa_tree_attention_workspace_size", "medusa_tree_attention",
     "medusa_verify_accept_workspace_size", "medusa_verify_accept",
     "medusa_kv_compact", "medusa_verify_accept_noalloc",
+    "medusa_lmhead_verify_workspace_size", "medusa_lmhead_verify",
 )
 
 
@@ -91,6 +92,11 @@ def lib() -> ctypes.CDLL:
                                                _F, _F, _F, _V, _V, _V, _V, _V, _V]
     L.medusa_kv_compact.restype = _I
     L.medusa_kv_compact.argtypes = [_V, _V, _I, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V, _V]
+    L.medusa_lmhead_verify_workspace_size.restype = _Z
+    L.medusa_lmhead_verify_workspace_size.argtypes = [_I, _I, _I, _I]
+    L.medusa_lmhead_verify.restype = _I
+    L.medusa_lmhead_verify.argtypes = [_V, _V, _I, _V, ctypes.POINTER(medusa_tree_t), _I, _I, _I,
+                                       _I, _F, _F, _F, _V, _V, _V, _V, _V, _V, _Z, _V, _V]
     _lib = L
     return L
 
@@ -263,3 +269,29 @@ def medusa_verify_accept_noalloc(logits, cand_ids, tree: Tree, accept_len, accep
                                               float(eps), float(delta), _p(accept_len),
                                               _p(accepted_nodes), _p(accepted_tokens), _p(bonus),
                                               _p(dev_status), _stream(stream)))
+
+
+def medusa_lmhead_verify_workspace_size(B: int, N: int, d: int, V: int) -> int:
+    return int(lib().medusa_lmhead_verify_workspace_size(B, N, d, V))
+
+
+def medusa_lmhead_verify(hidden, lm_head, cand_ids, tree: Tree, accept_len, accepted_nodes,
+                         accepted_tokens, bonus, mode: int = MEDUSA_ACCEPT_GREEDY,
+                         temperature: float = 1.0, eps: float = 0.09, delta: float = 0.3,
+                         logits=None, ws=None, dev_status=None, stream=None) -> None:
+    """hidden [B,N,d] bf16, lm_head [V,d] bf16 -> the verify outputs of
+    medusa_verify_accept on logits = hidden @ lm_head^T, never materialised
+    unless ``logits`` ([B,N,V] fp32) is given."""
+    _req(hidden, "hidden")
+    _req(lm_head, "lm_head")
+    B, N, d = hidden.shape
+    V = lm_head.shape[0]
+    if ws is None:
+        ws = workspace(medusa_lmhead_verify_workspace_size(B, N, d, V), hidden.device)
+    ct = tree.c()
+    _check(lib().medusa_lmhead_verify(_p(hidden), _p(lm_head), _dt(hidden), _p(cand_ids),
+                                      ctypes.byref(ct), B, d, V, mode, float(temperature),
+                                      float(eps), float(delta), _p(accept_len),
+                                      _p(accepted_nodes), _p(accepted_tokens), _p(bonus),
+                                      _p(logits), _p(ws), ws.numel(), _p(dev_status),
+                                      _stream(stream)))

@@ -186,6 +186,43 @@ medusa_status_t medusa_verify_accept(const void* logits, medusa_dtype_t dt,
                                static_cast<cudaStream_t>(stream));
 }
 
+size_t medusa_lmhead_verify_workspace_size(int B, int N, int d, int V) {
+  if (B < 1 || N < 1 || d < 1 || V < 1 || (long long)B * N > 65535) return 0;
+  return medusa::lmhead_verify_workspace_size(B, N, d, V);
+}
+
+medusa_status_t medusa_lmhead_verify(const void* hidden, const void* lm_head, medusa_dtype_t dt,
+                                     const int32_t* cand_ids, const medusa_tree_t* tree, int B,
+                                     int d, int V, medusa_accept_t mode, float temperature,
+                                     float eps, float delta, int32_t* accept_len,
+                                     int32_t* accepted_nodes, int32_t* accepted_tokens,
+                                     int32_t* bonus, float* logits, void* ws, size_t ws_bytes,
+                                     int32_t* dev_status, void* stream) {
+  medusa_status_t st = check_tree(tree);
+  if (st != MEDUSA_OK) return st;
+  if (!hidden || !lm_head || !cand_ids || !accept_len || !accepted_nodes || !accepted_tokens ||
+      !bonus)
+    return fail(MEDUSA_ERR_INVALID_ARG, "lmhead_verify: null pointer");
+  if (!valid_dtype(dt)) return fail(MEDUSA_ERR_INVALID_ARG, "lmhead_verify: bad dtype");
+  if (dt != MEDUSA_BF16) return fail(MEDUSA_ERR_UNSUPPORTED, "lmhead_verify: bf16 only");
+  if (mode != MEDUSA_ACCEPT_GREEDY && mode != MEDUSA_ACCEPT_TYPICAL)
+    return fail(MEDUSA_ERR_INVALID_ARG, "lmhead_verify: bad mode");
+  if (B < 1 || V < 1 || d < 64 || d % 64 != 0 || (long long)B * tree->n_nodes > 65535 ||
+      (long long)V * d > (1LL << 40))
+    return fail(MEDUSA_ERR_SHAPE, "lmhead_verify: need d a multiple of 64, B*N <= 65535");
+  if (mode == MEDUSA_ACCEPT_TYPICAL && (!(temperature > 0.f) || !(eps >= 0.f) || !(delta >= 0.f)))
+    return fail(MEDUSA_ERR_INVALID_ARG, "lmhead_verify: need temperature > 0, eps >= 0, delta >= 0");
+  if (!aligned16(hidden) || !aligned16(lm_head) ||
+      (logits != nullptr && reinterpret_cast<uintptr_t>(logits) % 4 != 0))
+    return fail(MEDUSA_ERR_ALIGNMENT, "lmhead_verify: hidden/lm_head not 16-byte aligned");
+  const size_t need = medusa::lmhead_verify_workspace_size(B, tree->n_nodes, d, V);
+  if (ws == nullptr || ws_bytes < need || !aligned256(ws))
+    return fail(MEDUSA_ERR_WORKSPACE, "lmhead_verify: workspace null, misaligned or too small");
+  return medusa::lmhead_verify(hidden, lm_head, cand_ids, *tree, B, d, V, mode, temperature, eps,
+                               delta, accept_len, accepted_nodes, accepted_tokens, bonus, logits,
+                               ws, dev_status, static_cast<cudaStream_t>(stream));
+}
+
 medusa_status_t medusa_kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
                                   const int32_t* accepted_nodes, const int32_t* accept_len, int B,
                                   int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,

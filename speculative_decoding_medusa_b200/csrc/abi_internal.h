@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -44,12 +45,42 @@ medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_n
                                int max_prefix, float scale, void* out, medusa_dtype_t out_dt,
                                void* ws, int32_t* status, cudaStream_t stream);
 
+// Per-(row, chunk) statistics of verify logits: the chunk's largest logit,
+// its lowest index, and for typical acceptance sum exp(z/T - maxz/T) and
+// sum exp(z/T - maxz/T) * z/T.
+struct RowPart {
+  float maxz;
+  int idx;
+  float s;
+  float t;
+};
+
+// Merges B*N rows of n_chunks RowParts each ([row][chunk], row = b*N + node)
+// and runs the path selection.  Typical acceptance reads the candidate's
+// logit as lm_head[tok] . hidden[b, parent] (bf16, d a multiple of 64).
+medusa_status_t verify_path_from_parts(const RowPart* part, int n_chunks,
+                                       const __nv_bfloat16* hidden,
+                                       const __nv_bfloat16* lm_head, int d,
+                                       const int32_t* cand_ids, const medusa_tree_t& tree, int B,
+                                       int V, medusa_accept_t mode, float temperature, float eps,
+                                       float delta, int32_t* accept_len,
+                                       int32_t* accepted_nodes, int32_t* accepted_tokens,
+                                       int32_t* bonus, int32_t* status, cudaStream_t stream);
+
 size_t verify_accept_workspace_size(int B, int N, int V);
 medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32_t* cand_ids,
                               const medusa_tree_t& tree, int B, int V, medusa_accept_t mode,
                               float temperature, float eps, float delta, int32_t* accept_len,
                               int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
                               void* ws, int32_t* status, cudaStream_t stream);
+
+size_t lmhead_verify_workspace_size(int B, int N, int d, int V);
+medusa_status_t lmhead_verify(const void* hidden, const void* lm_head, const int32_t* cand_ids,
+                              const medusa_tree_t& tree, int B, int d, int V,
+                              medusa_accept_t mode, float temperature, float eps, float delta,
+                              int32_t* accept_len, int32_t* accepted_nodes,
+                              int32_t* accepted_tokens, int32_t* bonus, float* logits, void* ws,
+                              int32_t* status, cudaStream_t stream);
 
 medusa_status_t kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
                            const int32_t* accepted_nodes, const int32_t* accept_len, int B,

@@ -28,13 +28,6 @@ namespace medusa {
 constexpr int kVChunk = 4096;   // tokens per warp work item
 constexpr int kRowWarps = 8;    // work items per CTA
 
-struct RowPart {
-  float maxz;
-  int idx;
-  float s;  // sum exp(z/T - maxz/T)
-  float t;  // sum exp(z/T - maxz/T) * z/T
-};
-
 template <typename T>
 struct Elt;
 template <>
@@ -245,8 +238,10 @@ constexpr int kPathThreads = 1024;
 
 template <typename T>
 __global__ void __launch_bounds__(kPathThreads)
-    verify_path_kernel(const T* __restrict__ logits, const RowPart* __restrict__ part,
-                       int n_chunks, int tpn, const int32_t* __restrict__ cand_ids,
+    verify_path_kernel(const T* __restrict__ logits, const __nv_bfloat16* __restrict__ hidden,
+                       const __nv_bfloat16* __restrict__ lm_head, int d,
+                       const RowPart* __restrict__ part, int n_chunks, int tpn,
+                       const int32_t* __restrict__ cand_ids,
                        const int32_t* __restrict__ parent, const int32_t* __restrict__ depth,
                        int N, int max_depth, int V, int typical, float inv_T, float eps,
                        float delta, int32_t* __restrict__ accept_len,
@@ -258,6 +253,7 @@ __global__ void __launch_bounds__(kPathThreads)
   __shared__ int s_parent[MEDUSA_MAX_NODES];
   __shared__ int s_depth[MEDUSA_MAX_NODES];
   __shared__ int s_pass[MEDUSA_MAX_NODES];
+  __shared__ float s_zc[MEDUSA_MAX_NODES];  // logit of node i's candidate at its parent
   __shared__ int s_best;
   __shared__ int s_bad;
   const int b = blockIdx.x;
@@ -346,6 +342,36 @@ __global__ void __launch_bounds__(kPathThreads)
     }
     return;
   }
+  if (typical && logits == nullptr) {
+    // no materialised logits: z = lm_head[tok] . hidden[b, parent], one warp
+    // per node, 16-byte loads (d is a multiple of 64)
+    const int warp = i >> 5, lane = i & 31;
+    for (int c = 1 + warp; c < N; c += kPathThreads / 32) {
+      const int tok = cand_ids[(size_t)b * N + c];
+      float acc = 0.f;
+      if (tok >= 0 && tok < V) {
+        const uint4* wr = reinterpret_cast<const uint4*>(lm_head + (size_t)tok * d);
+        const uint4* hr =
+            reinterpret_cast<const uint4*>(hidden + ((size_t)b * N + s_parent[c]) * d);
+        for (int e = lane; e < d / 8; e += 32) {
+          const uint4 x = wr[e], y = hr[e];
+          const uint32_t* xw = &x.x;
+          const uint32_t* yw = &y.x;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[q]));
+            const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&yw[q]));
+            acc = fmaf(xf.x, yf.x, acc);
+            acc = fmaf(xf.y, yf.y, acc);
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) s_zc[c] = acc;
+    }
+    __syncthreads();
+  }
   if (i < N) {
     int pass = 1;
     if (i > 0) {
@@ -357,7 +383,9 @@ __global__ void __launch_bounds__(kPathThreads)
       } else if (!typical) {
         pass = s_g[pa] == tok;
       } else {
-        const float lp = load1<T>(logits + ((size_t)b * N + pa) * V + tok) * inv_T - s_lse[pa];
+        const float z = logits != nullptr ? load1<T>(logits + ((size_t)b * N + pa) * V + tok)
+                                          : s_zc[i];
+        const float lp = z * inv_T - s_lse[pa];
         pass = lp > s_logthr[pa];
       }
     }
@@ -404,6 +432,30 @@ static unsigned rows_grid(K kernel, long long n_items) {
   return (unsigned)(need < resident ? need : resident);
 }
 
+int path_threads_per_node(int N, int n_chunks) {
+  int tpn = 1;  // threads merging one node's chunks
+  while (tpn < 32 && tpn * 2 * N <= kPathThreads && tpn < n_chunks) tpn *= 2;
+  return tpn;
+}
+
+medusa_status_t verify_path_from_parts(const RowPart* part, int n_chunks,
+                                       const __nv_bfloat16* hidden,
+                                       const __nv_bfloat16* lm_head, int d,
+                                       const int32_t* cand_ids, const medusa_tree_t& tree, int B,
+                                       int V, medusa_accept_t mode, float temperature, float eps,
+                                       float delta, int32_t* accept_len,
+                                       int32_t* accepted_nodes, int32_t* accepted_tokens,
+                                       int32_t* bonus, int32_t* status, cudaStream_t stream) {
+  const int N = tree.n_nodes;
+  const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
+  const float inv_T = typical ? 1.0f / temperature : 1.0f;
+  verify_path_kernel<__nv_bfloat16><<<B, kPathThreads, 0, stream>>>(
+      nullptr, hidden, lm_head, d, part, n_chunks, path_threads_per_node(N, n_chunks), cand_ids,
+      tree.parent, tree.depth, N, tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta,
+      accept_len, accepted_nodes, accepted_tokens, bonus, status);
+  return check_launch("verify_path");
+}
+
 size_t verify_accept_workspace_size(int B, int N, int V) {
   const size_t n_chunks = (size_t)(V + kVChunk - 1) / kVChunk;
   return align256((size_t)B * N * n_chunks * sizeof(RowPart));
@@ -420,8 +472,7 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
   const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
   const float inv_T = typical ? 1.0f / temperature : 1.0f;
   const long long n_items = (long long)B * N * n_chunks;
-  int tpn = 1;  // threads merging one node's chunks
-  while (tpn < 32 && tpn * 2 * N <= kPathThreads && tpn < n_chunks) tpn *= 2;
+  const int tpn = path_threads_per_node(N, n_chunks);
   if (dt == MEDUSA_BF16) {
     const __nv_bfloat16* lg = static_cast<const __nv_bfloat16*>(logits);
     if (typical) {
@@ -436,7 +487,7 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
     medusa_status_t st = check_launch("verify_rows");
     if (st != MEDUSA_OK) return st;
     verify_path_kernel<__nv_bfloat16><<<B, kPathThreads, 0, stream>>>(
-        lg, part, n_chunks, tpn, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
+        lg, nullptr, nullptr, 0, part, n_chunks, tpn, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
         typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
         status);
     return check_launch("verify_path");
@@ -454,7 +505,7 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
   medusa_status_t st = check_launch("verify_rows");
   if (st != MEDUSA_OK) return st;
   verify_path_kernel<float><<<B, kPathThreads, 0, stream>>>(
-      lg, part, n_chunks, tpn, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
+      lg, nullptr, nullptr, 0, part, n_chunks, tpn, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
       typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
       status);
   return check_launch("verify_path");

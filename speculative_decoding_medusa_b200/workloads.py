@@ -26,6 +26,7 @@ plainest reading is taken:
 from __future__ import annotations
 
 import dataclasses
+import math
 from typing import Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
@@ -346,3 +347,36 @@ def verify_logits(w: Workload, spec: TreeSpec, cand_ids: torch.Tensor, seed: int
         rowmax = logits[rb, ri].max(dim=-1).values
         logits[rb, ri, rc] = rowmax + 1.0
     return logits.to(torch_dtype(dt))
+
+
+_S_HID, _S_LMH = 31, 32
+
+
+def lmhead_inputs(w: Workload, spec: TreeSpec, cand_ids: torch.Tensor, seed: int = 0,
+                  device="cpu", attempt: int = 0, plant: float = 8.0,
+                  noise: float = 1.0) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Synthetic tree-node hidden states and lm_head, bf16.
+
+    lm_head [V, d] rows are N(0, 1/d) (unit length on average); hidden
+    [B, N, d] entries are N(0, noise^2), so unplanted scores are about
+    N(0, noise^2).  For each non-leaf node, with
+    probability ``p_match`` one child is picked uniformly and ``plant`` times
+    the lm_head row of its candidate token is added to the node's hidden
+    state, so that this token's score stands about ``plant`` above the rest.
+    ``attempt`` shifts the seed (used to redraw a whole set)."""
+    B, N = cand_ids.shape
+    s = seed + 7919 * attempt
+    lm = randn((w.V, w.d), s, _S_LMH, 1.0 / math.sqrt(w.d), "f32", device)
+    hid = randn((B, N, w.d), s, _S_HID, noise, "f32", device)
+    rng = np.random.default_rng(seed * 37 + 5 + attempt)
+    ch = children_lists(spec)
+    cand = cand_ids.to("cpu").numpy()
+    for b in range(B):
+        for i in range(N):
+            if not ch[i]:
+                continue
+            u = rng.uniform()
+            c = ch[i][int(rng.integers(len(ch[i])))]
+            if u < w.p_match:
+                hid[b, i] += plant * lm[int(cand[b, c])]
+    return hid.to(torch.bfloat16), lm.to(torch.bfloat16)
