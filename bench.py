@@ -232,7 +232,7 @@ def parse():
     ap.add_argument("--nodes", type=int, default=None, help="tree size override (long: 16/64/128)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--stage", choices=["all", "attention", "verify"], default="all",
+    ap.add_argument("--stage", choices=["all", "attention", "verify", "lmhead"], default="all",
                     help="time one stage alone (profiling aid; prints a stage line, not the metric)")
     return ap.parse_args()
 
@@ -272,6 +272,18 @@ def run_stage(args):
         P = att["prefix_len"].tolist()
         nbytes = (sum(P) * w.Hkv * w.dh * 2 + w.B * N * (2 * w.Hq + 4 * w.Hkv) * w.dh) * e
         flops = 4.0 * w.Hq * w.dh * N * sum(p + N for p in P)
+    elif args.stage == "lmhead":
+        # verification from the nodes' hidden states: lm_head GEMM + reduction
+        hidden, lm = W.lmhead_inputs(w, spec, cand.cpu(), seed=0, device=dev)
+        Wd = spec.max_depth + 1
+        outs = [torch.empty(w.B, **i32), torch.empty(w.B, Wd, **i32), torch.empty(w.B, Wd, **i32),
+                torch.empty(w.B, **i32)]
+        ws = M.workspace(M.medusa_lmhead_verify_workspace_size(w.B, N, w.d, w.V), dev)
+        mode = M.MEDUSA_ACCEPT_TYPICAL if w.accept == "typical" else M.MEDUSA_ACCEPT_GREEDY
+        fn = lambda: M.medusa_lmhead_verify(hidden, lm, cand, tree, *outs, mode, w.temperature,
+                                            w.eps, w.delta, ws=ws, dev_status=status)
+        nbytes = (w.V * w.d + w.B * N * w.d) * 2
+        flops = 2.0 * w.B * N * w.V * w.d
     else:
         torch.cuda.synchronize()
         logits = W.verify_logits(w, spec, cand, seed=0, device=dev)

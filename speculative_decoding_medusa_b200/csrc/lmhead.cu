@@ -42,7 +42,7 @@ constexpr int kLmTileM = 128;    // vocabulary rows per tile (UMMA M)
 constexpr int kLmTileK = 64;     // bf16 per 128-byte swizzled row
 constexpr int kLmHalf = 256;     // columns per MMA (UMMA N <= 256)
 constexpr int kLmBlock = 512;    // columns per block (two halves)
-constexpr int kLmStages = 2;
+constexpr int kLmStages = 4;    // a stage: one k-block of lm_head and of one hidden half
 constexpr int kLmThreads = 192;
 
 struct LmParams {
@@ -60,12 +60,12 @@ struct LmParams {
 struct LmSmem {
   static constexpr int kABytes = kLmTileM * kLmTileK * 2;  // 16 KB
   static constexpr int kBHalfBytes = kLmHalf * kLmTileK * 2;  // 32 KB
-  static constexpr int kBBytes = 2 * kBHalfBytes;
+  static constexpr int kBBytes = kBHalfBytes;
   static constexpr int kAOff = 0;
   static constexpr int kBOff = kAOff + kLmStages * kABytes;
-  static constexpr int kRunOff = kBOff + kLmStages * kBBytes;   // RowPart run[512]
-  static constexpr int kRedOff = kRunOff + kLmBlock * 16;       // RowPart red[4][256]
-  static constexpr int kBarOff = kRedOff + 4 * kLmHalf * 16;
+  static constexpr int kRedOff = kBOff + kLmStages * kBBytes;   // RowPart red[4][256]
+  static constexpr int kScrOff = kRedOff + 4 * kLmHalf * 16;    // float [4][32][33]
+  static constexpr int kBarOff = kScrOff + 4 * 32 * 33 * 4;
   // full[S], empty[S], tfull, tempty[2], drain, epi
   static constexpr int kNumBars = 2 * kLmStages + 5;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
@@ -213,20 +213,21 @@ __global__ void __launch_bounds__(kLmThreads, 1)
         const int cb = u / p.n_vt, vt = u - cb * p.n_vt;
         int ncols, nb0, nb1;
         block_shape(p, cb, ncols, nb0, nb1);
-        for (int kb = 0; kb < nkb; ++kb, ++g) {
+        // stages in order (kb, half): the second half's copy of the lm_head
+        // k-block comes from L2
+        const int nh = nb1 > 0 ? 2 : 1;
+        for (int st = 0; st < nkb * nh; ++st, ++g) {
+          const int kb = st / nh, h = st - kb * nh;
           const int s = g % kLmStages;
           if (!mbar_wait_bounded(&empty[s], ((g / kLmStages) & 1) ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], L::kABytes + (nb1 > 0 ? 2 : 1) * L::kBHalfBytes);
-          uint8_t* b_st = smem + L::kBOff + s * L::kBBytes;
+          mbar_arrive_expect_tx(&full[s], L::kABytes + L::kBBytes);
           tma_load_3d(smem + L::kAOff + s * L::kABytes, &tmA, &full[s], kb * kLmTileK,
                       vt * kLmTileM, 0, pol_a);
-          tma_load_3d(b_st, &tmB, &full[s], kb * kLmTileK, cb * kLmBlock, 0, pol_b);
-          if (nb1 > 0)
-            tma_load_3d(b_st + L::kBHalfBytes, &tmB, &full[s], kb * kLmTileK,
-                        cb * kLmBlock + kLmHalf, 0, pol_b);
+          tma_load_3d(smem + L::kBOff + s * L::kBBytes, &tmB, &full[s], kb * kLmTileK,
+                      cb * kLmBlock + h * kLmHalf, 0, pol_b);
         }
       }
       // let every copy this thread issued land before the CTA can exit
@@ -247,39 +248,28 @@ __global__ void __launch_bounds__(kLmThreads, 1)
         block_shape(p, cb, ncols, nb0, nb1);
         const uint32_t idesc0 = umma_idesc_bf16(kLmTileM, nb0);
         const uint32_t idesc1 = nb1 > 0 ? umma_idesc_bf16(kLmTileM, nb1) : 0u;
-        for (int kb = 0; kb < nkb; ++kb, ++g) {
+        const int nh = nb1 > 0 ? 2 : 1;
+        for (int st = 0; st < nkb * nh; ++st, ++g) {
+          const int kb = st / nh, h = st - kb * nh;
           const int s = g % kLmStages;
           if (!mbar_wait_bounded(&full[s], (g / kLmStages) & 1, abort_flag, p.status)) {
             ok = false;
             break;
           }
           // a TMEM half is written again only once the epilogue has read it
-          if (kb == 0 &&
-              !mbar_wait_bounded(&tempty[0], (it & 1) ^ 1u, abort_flag, p.status)) {
+          if (kb == 0 && !mbar_wait_bounded(&tempty[h], (h == 0 ? (it & 1) : (n1 & 1)) ^ 1u,
+                                            abort_flag, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + L::kAOff + s * L::kABytes);
           const uint32_t b_addr = smem_u32(smem + L::kBOff + s * L::kBBytes);
+          const uint32_t idesc = h == 0 ? idesc0 : idesc1;
 #pragma unroll
           for (int kk = 0; kk < kLmTileK / 16; ++kk)
-            umma_bf16(tmem_base, umma_desc_sw128(a_addr + kk * 32),
-                      umma_desc_sw128(b_addr + kk * 32), idesc0, (kb | kk) != 0 ? 1u : 0u);
-          if (nb1 > 0) {
-            if (kb == 0) {
-              if (!mbar_wait_bounded(&tempty[1], (n1 & 1) ^ 1u, abort_flag, p.status)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-            }
-#pragma unroll
-            for (int kk = 0; kk < kLmTileK / 16; ++kk)
-              umma_bf16(tmem_base + kLmHalf, umma_desc_sw128(a_addr + kk * 32),
-                        umma_desc_sw128(b_addr + L::kBHalfBytes + kk * 32), idesc1,
-                        (kb | kk) != 0 ? 1u : 0u);
-          }
+            umma_bf16(tmem_base + h * kLmHalf, umma_desc_sw128(a_addr + kk * 32),
+                      umma_desc_sw128(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
           umma_commit(&empty[s]);
         }
         if (!ok) break;
@@ -296,8 +286,9 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
     const int te = threadIdx.x - 64;  // 0..127
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    RowPart* run = reinterpret_cast<RowPart*>(smem + L::kRunOff);  // [512] this CTA's records
     RowPart* red = reinterpret_cast<RowPart*>(smem + L::kRedOff);  // [4][256] per-warp results
+    // this warp's 32 x 32 transpose scratch, rows padded to 33 words
+    float* tsc = reinterpret_cast<float*>(smem + L::kScrOff) + quad * 32 * 33;
     const bool typical = p.typical != 0;
     // the four epilogue warps synchronise on an mbarrier with a bounded wait
     uint32_t epi_phase = 0;
@@ -308,7 +299,12 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       epi_phase ^= 1u;
       return epi_ok;
     };
-    for (int c = te; c < kLmBlock; c += 128) run[c] = empty_record();
+    // the CTA's running records of block-local columns h * 256 + te + 128 k
+    RowPart run[2][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int k = 0; k < 2; ++k) run[h][k] = empty_record();
     bool bad = false;  // a NaN logit
     int it = 0;
     for (int u = u0; epi_ok && u < u1; ++u, ++it) {
@@ -317,52 +313,77 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       block_shape(p, cb, ncols, nb0, nb1);
       if (!mbar_wait_bounded(tfull, it & 1, abort_flag, p.status)) break;
       tc_fence_after();
-      const int vrow = vt * kLmTileM + quad * 32 + lane;  // this thread's vocabulary row
-      const bool row_ok = vrow < p.V;
-      for (int h = 0; epi_ok && h < 2; ++h) {
+      const int row0 = vt * kLmTileM + quad * 32;  // vocabulary row of this warp's lane 0
+      const bool row_ok = row0 + lane < p.V;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
         const int nbh = h ? nb1 : nb0;
-        if (nbh == 0) break;
+        if (!epi_ok || nbh == 0) break;
         const int ngroups = (nbh + 31) / 32;
 #pragma unroll 1
         for (int gq = 0; gq < ngroups; ++gq) {
           const int col0 = h * kLmHalf + gq * 32;  // block-local column of z[0]
           float z[32];
           tmem_ld32(tmem_base + lane_off + col0, z);
-          float v[32];
-          int id[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const bool ok = row_ok && (col0 + j < ncols);
-            bad |= ok && (z[j] != z[j]);
-            v[j] = ok ? z[j] : -INFINITY;
-            id[j] = ok ? vrow : 0x7fffffff;
-          }
           if (p.logits != nullptr && row_ok) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               if (col0 + j < ncols)
-                p.logits[(size_t)(cb * kLmBlock + col0 + j) * p.V + vrow] = z[j];
+                p.logits[(size_t)(cb * kLmBlock + col0 + j) * p.V + row0 + lane] = z[j];
           }
-          warp_colmax32(v, id, lane);
+          // transpose through shared memory: lane = row on the way in, lane =
+          // column on the way out (padding keeps both directions free of bank
+          // conflicts)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            bad |= row_ok && (col0 + j < ncols) && (z[j] != z[j]);
+            tsc[lane * 33 + j] = row_ok ? z[j] : -INFINITY;
+          }
+          __syncwarp();
+          float c[32];
+#pragma unroll
+          for (int r = 0; r < 32; ++r) c[r] = tsc[r * 33 + lane];
+          __syncwarp();
+          // column `lane`: largest value, lowest row among equals (four
+          // chains over rows r = q, q + 4, ..., then merged in row order)
+          float bv[4];
+          int br[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            bv[q] = c[q];
+            br[q] = q;
+          }
+#pragma unroll
+          for (int r = 4; r < 32; ++r) {
+            if (c[r] > bv[r & 3]) {
+              bv[r & 3] = c[r];
+              br[r & 3] = r;
+            }
+          }
+          float m = bv[0];
+          int mr = br[0];
+#pragma unroll
+          for (int q = 1; q < 4; ++q) {
+            if (bv[q] > m || (bv[q] == m && br[q] < mr)) {
+              m = bv[q];
+              mr = br[q];
+            }
+          }
           RowPart rec;
-          rec.maxz = v[0];
-          rec.idx = id[0];
+          rec.maxz = m;
+          rec.idx = m == -INFINITY ? 0x7fffffff : row0 + mr;
           rec.s = 0.f;
           rec.t = 0.f;
-          if (typical) {
-            // weights relative to the column's maximum over this warp's rows
-            float a[32], b[32];
+          if (typical && m != -INFINITY) {
+            float s = 0.f, t = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float mj = __shfl_sync(0xffffffffu, rec.maxz, j);
-              const bool ok = row_ok && (col0 + j < ncols) && mj != -INFINITY;
-              const float w = ok ? lm_ex2((z[j] - mj) * p.t_log2) : 0.f;
-              a[j] = w;
-              b[j] = ok ? w * (z[j] * p.inv_T) : 0.f;
+            for (int r = 0; r < 32; ++r) {
+              const float w = lm_ex2((c[r] - m) * p.t_log2);  // -inf rows give 0
+              s += w;
+              t += c[r] == -INFINITY ? 0.f : w * (c[r] * p.inv_T);
             }
-            warp_colsum32x2(a, b, lane);
-            rec.s = a[0];
-            rec.t = b[0];
+            rec.s = s;
+            rec.t = t;
           }
           red[quad * kLmHalf + gq * 32 + lane] = rec;
         }
@@ -370,11 +391,15 @@ __global__ void __launch_bounds__(kLmThreads, 1)
         tc_fence_before();
         mbar_arrive(&tempty[h]);
         if (!epi_sync()) break;
-        for (int c = te; c < ngroups * 32; c += 128) {
-          RowPart r = red[c];
 #pragma unroll
-          for (int q = 1; q < 4; ++q) merge_record(r, red[q * kLmHalf + c], typical, p.t_log2);
-          merge_record(run[h * kLmHalf + c], r, typical, p.t_log2);
+        for (int k = 0; k < 2; ++k) {
+          const int cc = te + 128 * k;
+          if (cc < ngroups * 32) {
+            RowPart r = red[cc];
+#pragma unroll
+            for (int q = 1; q < 4; ++q) merge_record(r, red[q * kLmHalf + cc], typical, p.t_log2);
+            merge_record(run[h][k], r, typical, p.t_log2);
+          }
         }
         if (!epi_sync()) break;
       }
@@ -383,14 +408,20 @@ __global__ void __launch_bounds__(kLmThreads, 1)
         const int c_first = (cb * p.n_vt) / p.per;
         const int c_last = (cb * p.n_vt + p.n_vt - 1) / p.per;
         const int slot = static_cast<int>(blockIdx.x) - c_first;
-        for (int c = te; c < ncols; c += 128) {
-          RowPart* dst = p.part + (size_t)(cb * kLmBlock + c) * p.n_slots;
-          dst[slot] = run[c];
-          run[c] = empty_record();
-          // the block's last CTA pads its columns' unused record slots
-          if (static_cast<int>(blockIdx.x) == c_last)
-            for (int s2 = slot + 1; s2 < p.n_slots; ++s2) dst[s2] = empty_record();
-        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int cc = h * kLmHalf + te + 128 * k;
+            if (cc < ncols) {
+              RowPart* dst = p.part + (size_t)(cb * kLmBlock + cc) * p.n_slots;
+              dst[slot] = run[h][k];
+              // the block's last CTA pads its columns' unused record slots
+              if (static_cast<int>(blockIdx.x) == c_last)
+                for (int s2 = slot + 1; s2 < p.n_slots; ++s2) dst[s2] = empty_record();
+            }
+            run[h][k] = empty_record();
+          }
       }
     }
     if (bad) report(p.status, MEDUSA_ERR_DEVICE_CHECK);
