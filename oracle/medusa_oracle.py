@@ -355,6 +355,24 @@ def kv_compact(Kc: np.ndarray, Vc: np.ndarray, prefix_len: np.ndarray,
 # ---------------------------------------------------------------------------
 
 
+def next_step_inputs(node_hidden: np.ndarray, accept_len: np.ndarray,
+                     accepted_nodes: np.ndarray, bonus: np.ndarray
+                     ) -> Tuple[np.ndarray, np.ndarray]:
+    """Inputs of the next decode step after a verification.
+
+    [GLOSS-TREE]: the accepted candidates enter the sequence; the heads of
+    the next round read the base model's last hidden state, i.e. that of the
+    last accepted node (the kept node), and the next round's first token is
+    the base model's own choice there (the bonus token; [DEPLOY-PT]: the
+    conventionally generated token).  node_hidden [B, N, d] -> (h_next
+    [B, d], root_next [B])."""
+    node_hidden = np.asarray(node_hidden)
+    B = node_hidden.shape[0]
+    kept = np.array([accepted_nodes[b, int(accept_len[b])] for b in range(B)], dtype=np.int64)
+    h_next = np.stack([node_hidden[b, kept[b]] for b in range(B)])
+    return h_next, np.asarray(bonus, dtype=np.int32).copy()
+
+
 def lmhead_verify(hidden: np.ndarray, lm_head: np.ndarray, cand: np.ndarray,
                   parent: np.ndarray, depth: np.ndarray, max_depth: int,
                   accept_mode: str = "greedy", temperature: float = 1.0,

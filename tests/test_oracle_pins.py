@@ -470,3 +470,26 @@ def test_lmhead_verify_logits_bruteforce_and_typical_mode():
     ref = O.verify_typical(z, cand, spec.parent, spec.depth, 1, 0.8, 0.3, 0.5)
     assert res["accept_len"].tolist() == ref["accept_len"].tolist()
     assert res["bonus"].tolist() == ref["bonus"].tolist()
+
+
+def test_next_step_inputs_take_the_kept_node_and_bonus():
+    """Glossary tree, kept branch 0 -> 2 -> 7 for sequence 0 and the root
+    only for sequence 1: the next heads read node 7's (resp. node 0's) hidden
+    state and the next root is each sequence's bonus token."""
+    spec = W.cartesian_tree([2, 3])
+    cand = np.array([[7, 100, 101, 200, 201, 202, 200, 201, 202]] * 2, dtype=np.int32)
+    V, d = 300, 320
+    lm = np.zeros((V, d))
+    lm[np.arange(V), np.arange(V)] = 1.0
+    hidden = np.zeros((2, 9, d))
+    for n, t in {0: 101, 2: 201, 7: 42}.items():
+        hidden[0, n, t] = 1.0
+    hidden[1, 0, 9] = 1.0
+    for n in range(9):
+        hidden[:, n, 300 + n % 20] += 0.5  # node-specific tag outside the vocabulary
+    res = O.lmhead_verify(hidden, lm, cand, spec.parent, spec.depth, 2)
+    h_next, root_next = O.next_step_inputs(hidden, res["accept_len"], res["accepted_nodes"],
+                                           res["bonus"])
+    np.testing.assert_array_equal(h_next[0], hidden[0, 7])
+    np.testing.assert_array_equal(h_next[1], hidden[1, 0])
+    assert root_next.tolist() == [42, 9]
