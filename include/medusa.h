@@ -351,6 +351,34 @@ MEDUSA_API medusa_status_t medusa_lmhead_verify(
     int32_t* accepted_tokens, int32_t* bonus, float* logits, void* ws, size_t ws_bytes,
     int32_t* dev_status, void* stream);
 
+/* ------------------------------------------------------------------------
+ * medusa_next_step
+ *
+ * "Medusa Heads" glossary, "Attention arborescente et acceptation": the
+ * accepted candidates join the sequence, and the heads of the next round
+ * read the base model's last hidden state - that of the kept node; "Medusa
+ * no contexto de LLMs": the base model's own token at the kept node (the
+ * bonus token) is the next generated token, the next tree's root.
+ *
+ *   kept = accepted_nodes[b][accept_len[b]];
+ *   h_next[b][:] = node_hidden[b][kept][:];   root_next[b] = bonus[b].
+ *
+ * Inputs (device): node_hidden [B, N, d] of dtype dt (the base model's last
+ *   hidden states of the tree nodes); accept_len [B], accepted_nodes
+ *   [B, max_depth+1], bonus [B] (int32, as written by the verification).
+ * Outputs (device): h_next [B, d] of dtype dt; root_next [B] int32.
+ * Limits: d * element size a multiple of 16; N <= MEDUSA_MAX_NODES;
+ *   node_hidden and h_next 16-byte aligned.
+ * Device checks: accept_len outside [0, max_depth] or a kept node outside
+ *   [0, N) (that sequence's outputs are left unwritten).
+ * ---------------------------------------------------------------------- */
+MEDUSA_API medusa_status_t medusa_next_step(const void* node_hidden, medusa_dtype_t dt,
+                                            const int32_t* accept_len,
+                                            const int32_t* accepted_nodes, const int32_t* bonus,
+                                            int B, int N, int d, int max_depth, void* h_next,
+                                            int32_t* root_next, int32_t* dev_status,
+                                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif

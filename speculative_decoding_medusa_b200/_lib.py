@@ -36,7 +36,7 @@ EXPORTS = (
     "medusa_tree_attention_workspace_size", "medusa_tree_attention",
     "medusa_verify_accept_workspace_size", "medusa_verify_accept",
     "medusa_kv_compact", "medusa_verify_accept_noalloc",
-    "medusa_lmhead_verify_workspace_size", "medusa_lmhead_verify",
+    "medusa_lmhead_verify_workspace_size", "medusa_lmhead_verify", "medusa_next_step",
 )
 
 
@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
     L.medusa_kv_compact.argtypes = [_V, _V, _I, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V, _V]
     L.medusa_lmhead_verify_workspace_size.restype = _Z
     L.medusa_lmhead_verify_workspace_size.argtypes = [_I, _I, _I, _I]
+    L.medusa_next_step.restype = _I
+    L.medusa_next_step.argtypes = [_V, _I, _V, _V, _V, _I, _I, _I, _I, _V, _V, _V, _V]
     L.medusa_lmhead_verify.restype = _I
     L.medusa_lmhead_verify.argtypes = [_V, _V, _I, _V, ctypes.POINTER(medusa_tree_t), _I, _I, _I,
                                        _I, _F, _F, _F, _V, _V, _V, _V, _V, _V, _Z, _V, _V]
@@ -295,3 +297,15 @@ def medusa_lmhead_verify(hidden, lm_head, cand_ids, tree: Tree, accept_len, acce
                                       _p(accepted_nodes), _p(accepted_tokens), _p(bonus),
                                       _p(logits), _p(ws), ws.numel(), _p(dev_status),
                                       _stream(stream)))
+
+
+def medusa_next_step(node_hidden, accept_len, accepted_nodes, bonus, h_next, root_next,
+                     dev_status=None, stream=None) -> None:
+    """h_next[b] = node_hidden[b, kept node], root_next[b] = bonus[b]."""
+    _req(node_hidden, "node_hidden")
+    _req(h_next, "h_next")
+    B, N, d = node_hidden.shape
+    max_depth = accepted_nodes.shape[1] - 1
+    _check(lib().medusa_next_step(_p(node_hidden), _dt(node_hidden), _p(accept_len),
+                                  _p(accepted_nodes), _p(bonus), B, N, d, max_depth, _p(h_next),
+                                  _p(root_next), _p(dev_status), _stream(stream)))

@@ -223,6 +223,25 @@ medusa_status_t medusa_lmhead_verify(const void* hidden, const void* lm_head, me
                                ws, dev_status, static_cast<cudaStream_t>(stream));
 }
 
+medusa_status_t medusa_next_step(const void* node_hidden, medusa_dtype_t dt,
+                                 const int32_t* accept_len, const int32_t* accepted_nodes,
+                                 const int32_t* bonus, int B, int N, int d, int max_depth,
+                                 void* h_next, int32_t* root_next, int32_t* dev_status,
+                                 void* stream) {
+  if (!node_hidden || !accept_len || !accepted_nodes || !bonus || !h_next || !root_next)
+    return fail(MEDUSA_ERR_INVALID_ARG, "next_step: null pointer");
+  if (!valid_dtype(dt)) return fail(MEDUSA_ERR_INVALID_ARG, "next_step: bad dtype");
+  if (B < 1 || B > 65535 || N < 1 || N > MEDUSA_MAX_NODES || d < 1 || max_depth < 0 ||
+      max_depth >= MEDUSA_MAX_HEADS)
+    return fail(MEDUSA_ERR_SHAPE, "next_step: B, N, d or max_depth out of range");
+  const int eb = dt == MEDUSA_BF16 ? 2 : 4;
+  if ((d * eb) % 16 != 0) return fail(MEDUSA_ERR_SHAPE, "next_step: d * element size % 16 != 0");
+  if (!aligned16(node_hidden) || !aligned16(h_next))
+    return fail(MEDUSA_ERR_ALIGNMENT, "next_step: hidden buffers must be 16-byte aligned");
+  return medusa::next_step(node_hidden, eb, accept_len, accepted_nodes, bonus, B, N, d, max_depth,
+                           h_next, root_next, dev_status, static_cast<cudaStream_t>(stream));
+}
+
 medusa_status_t medusa_kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
                                   const int32_t* accepted_nodes, const int32_t* accept_len, int B,
                                   int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,

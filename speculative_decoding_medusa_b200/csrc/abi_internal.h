@@ -82,6 +82,11 @@ medusa_status_t lmhead_verify(const void* hidden, const void* lm_head, const int
                               int32_t* accepted_tokens, int32_t* bonus, float* logits, void* ws,
                               int32_t* status, cudaStream_t stream);
 
+medusa_status_t next_step(const void* node_hidden, int elem_bytes, const int32_t* accept_len,
+                          const int32_t* accepted_nodes, const int32_t* bonus, int B, int N,
+                          int d, int max_depth, void* h_next, int32_t* root_next,
+                          int32_t* status, cudaStream_t stream);
+
 medusa_status_t kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
                            const int32_t* accepted_nodes, const int32_t* accept_len, int B,
                            int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,

@@ -61,3 +61,72 @@ class DecodeVerifyStep:
                                self.status, stream)
         M.medusa_kv_compact(Kc, Vc, prefix_len, self.accepted_nodes, self.accept_len,
                             self.compact_src, self.status, stream)
+
+
+class DecodeLoop:
+    """Decode steps chained on the device (greedy or typical acceptance with
+    the verification taken from the tree nodes' hidden states):
+
+        heads + top-k (h) -> tree build (root) -> base model (external; gives
+        the nodes' hidden states and tree Q/K/V) -> tree attention ->
+        lm_head verify -> KV compaction -> next step (h := kept node's hidden
+        state, root := bonus token)
+
+    ``step`` enqueues one step and records its accept_len in ``history``;
+    nothing synchronises with the host, so a run of steps can be captured in
+    one CUDA graph."""
+
+    def __init__(self, *, B: int, d: int, V: int, K: int, kmax: int, tree: M.Tree, Hq: int,
+                 Hkv: int, dh: int, cap: int, max_prefix: int, steps: int,
+                 accept: str = "greedy", temperature: float = 1.0, eps: float = 0.09,
+                 delta: float = 0.3, device="cuda"):
+        self.B, self.d, self.V, self.K, self.kmax = B, d, V, K, kmax
+        self.tree, self.Hq, self.Hkv, self.dh = tree, Hq, Hkv, dh
+        self.max_prefix = max_prefix
+        self.mode = M.MEDUSA_ACCEPT_TYPICAL if accept == "typical" else M.MEDUSA_ACCEPT_GREEDY
+        self.temperature, self.eps, self.delta = temperature, eps, delta
+        N, W = tree.n_nodes, tree.max_depth + 1
+        i32 = dict(dtype=torch.int32, device=device)
+        self.topk_ids = torch.empty(B, K, kmax, **i32)
+        self.topk_vals = torch.empty(B, K, kmax, dtype=torch.float32, device=device)
+        self.cand_ids = torch.empty(B, N, **i32)
+        self.pos_ids = torch.empty(B, N, **i32)
+        self.anc_mask = torch.empty(N, (N + 31) // 32, **i32)
+        self.retrieve = torch.empty(tree.n_leaves, W, **i32)
+        self.attn_out = torch.empty(B, N, Hq, dh, dtype=torch.bfloat16, device=device)
+        self.accept_len = torch.empty(B, **i32)
+        self.accepted_nodes = torch.empty(B, W, **i32)
+        self.accepted_tokens = torch.empty(B, W, **i32)
+        self.bonus = torch.empty(B, **i32)
+        self.compact_src = torch.empty(B, W, **i32)
+        self.history = torch.zeros(steps, B, **i32)
+        self.tokens = torch.zeros(steps, B, W, **i32)
+        self.status = torch.zeros(1, **i32)
+        bf = M.MEDUSA_BF16
+        self.ws_heads = M.workspace(M.medusa_heads_topk_workspace_size(B, d, V, K, kmax, bf), device)
+        self.ws_attn = M.workspace(M.medusa_tree_attention_workspace_size(
+            B, N, Hq, Hkv, dh, max_prefix, bf), device)
+        self.ws_lm = M.workspace(M.medusa_lmhead_verify_workspace_size(B, N, d, V), device)
+
+    def step(self, r: int, h, root, W1, b1, W2, lm_head, base_model, q, k_new, v_new, Kc, Vc,
+             prefix_len, stream=None) -> None:
+        """Enqueue step ``r``.  h [B, d] bf16 and root [B] int32 are replaced
+        by the next step's; Kc/Vc/prefix_len advance by the kept branch."""
+        M.medusa_heads_topk(h, W1, b1, W2, self.kmax, self.topk_ids, self.topk_vals, None,
+                            self.ws_heads, self.status, stream)
+        M.medusa_tree_build(self.tree, root, self.topk_ids, prefix_len, self.cand_ids,
+                            self.pos_ids, self.anc_mask, self.retrieve, self.status, stream)
+        node_hidden = base_model.forward(self.cand_ids, r)
+        M.medusa_tree_attention(q, k_new, v_new, Kc, Vc, prefix_len, self.anc_mask,
+                                self.max_prefix, self.attn_out, None, self.ws_attn, self.status,
+                                stream)
+        M.medusa_lmhead_verify(node_hidden, lm_head, self.cand_ids, self.tree, self.accept_len,
+                               self.accepted_nodes, self.accepted_tokens, self.bonus, self.mode,
+                               self.temperature, self.eps, self.delta, None, self.ws_lm,
+                               self.status, stream)
+        M.medusa_kv_compact(Kc, Vc, prefix_len, self.accepted_nodes, self.accept_len,
+                            self.compact_src, self.status, stream)
+        M.medusa_next_step(node_hidden, self.accept_len, self.accepted_nodes, self.bonus, h, root,
+                           self.status, stream)
+        self.history[r].copy_(self.accept_len)
+        self.tokens[r].copy_(self.accepted_tokens)

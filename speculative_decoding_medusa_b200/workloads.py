@@ -380,3 +380,43 @@ def lmhead_inputs(w: Workload, spec: TreeSpec, cand_ids: torch.Tensor, seed: int
             if u < w.p_match:
                 hid[b, i] += plant * lm[int(cand[b, c])]
     return hid.to(torch.bfloat16), lm.to(torch.bfloat16)
+
+
+class SyntheticBaseModel:
+    """Stand-in for the base model's forward over the tree, whose transformer
+    layers are outside this library: it only produces the tree nodes' last
+    hidden states, on the device, from the step's candidate tokens.
+
+    Hidden states are a fixed N(0, noise^2) draw; at step r, each non-leaf
+    node is, with probability ``p_match``, given ``plant`` times the lm_head
+    row of one (pre-drawn) child's candidate token, so that the verification
+    accepts that child.  All picks are drawn up front, so forward() is a few
+    device tensor ops that a CUDA graph can capture."""
+
+    def __init__(self, w: Workload, spec: TreeSpec, lm_head: torch.Tensor, steps: int,
+                 seed: int = 0, device="cuda", plant: float = 8.0, noise: float = 1.0):
+        B, N = w.B, spec.n_nodes
+        self.B, self.N, self.d, self.plant = B, N, w.d, plant
+        self.lm = lm_head
+        self.noise = randn((B, N, w.d), seed, _S_HID, noise, "f32", device)
+        rng = np.random.default_rng(seed * 41 + 3)
+        ch = children_lists(spec)
+        pick = np.zeros((steps, B, N), dtype=np.int64)
+        on = np.zeros((steps, B, N, 1), dtype=np.float32)
+        for r in range(steps):
+            for b in range(B):
+                for n in range(N):
+                    if ch[n]:
+                        pick[r, b, n] = ch[n][int(rng.integers(len(ch[n])))]
+                        on[r, b, n, 0] = plant if rng.uniform() < w.p_match else 0.0
+        self.pick = torch.from_numpy(pick).to(device)
+        self.on = torch.from_numpy(on).to(device)
+        self.tmp = torch.empty(B, N, w.d, dtype=torch.float32, device=device)
+        self.out = torch.empty(B, N, w.d, dtype=torch.bfloat16, device=device)
+
+    def forward(self, cand_ids: torch.Tensor, r: int) -> torch.Tensor:
+        tok = torch.gather(cand_ids.long(), 1, self.pick[r])
+        rows = self.lm.index_select(0, tok.reshape(-1)).view(self.B, self.N, self.d)
+        torch.addcmul(self.noise, rows.float(), self.on[r], out=self.tmp)
+        self.out.copy_(self.tmp)
+        return self.out
