@@ -232,9 +232,90 @@ def parse():
     ap.add_argument("--nodes", type=int, default=None, help="tree size override (long: 16/64/128)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--stage", choices=["all", "attention", "verify", "lmhead"], default="all",
+    ap.add_argument("--loop-steps", type=int, default=16,
+                    help="decode steps per CUDA graph (--stage loop)")
+    ap.add_argument("--stage", choices=["all", "attention", "verify", "lmhead", "loop"],
+                    default="all",
                     help="time one stage alone (profiling aid; prints a stage line, not the metric)")
     return ap.parse_args()
+
+
+def run_loop(args):
+    """Decode steps chained on the device and replayed from one CUDA graph:
+    heads -> tree -> (synthetic base model: node hidden states) -> tree
+    attention -> lm_head verify -> KV compaction -> next step.  Reports
+    tokens per second (kept candidates + the bonus token, all sequences)
+    with the mean accept_len the synthetic base model produced."""
+    import math
+    import speculative_decoding_medusa_b200 as M
+    from speculative_decoding_medusa_b200 import workloads as W
+    from speculative_decoding_medusa_b200.step import DecodeLoop
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = W.WORKLOADS[args.workload]
+    R = args.loop_steps
+    spec = W.tree_for(w)
+    N = spec.n_nodes
+    tree = M.Tree.from_spec(spec, dev)
+    heads = W.heads_inputs(w, seed=0, device=dev)
+    max_prefix = w.ctx_hi + R * (spec.max_depth + 1)
+    cap = max_prefix + N
+    att = W.attention_inputs(W.scaled(w, ctx_hi=cap - N), seed=0, device=dev, n_nodes=N)
+    p0 = W.prefix_lengths(w, seed=0, device=dev)
+    lm = W.randn((w.V, w.d), 0, 77, 1.0 / math.sqrt(w.d), "bf16", dev)
+    bm = W.SyntheticBaseModel(w, spec, lm, R, seed=0, device=dev)
+    loop = DecodeLoop(B=w.B, d=w.d, V=w.V, K=w.K, kmax=w.kmax, tree=tree, Hq=w.Hq, Hkv=w.Hkv,
+                      dh=w.dh, cap=cap, max_prefix=max_prefix, steps=R, accept=w.accept,
+                      temperature=w.temperature, eps=w.eps, delta=w.delta, device=dev)
+    h0 = heads["h"].clone()
+    r0 = W.random_root_tokens(w, 0, device=dev)
+    h, root, pl = h0.clone(), r0.clone(), p0.clone()
+
+    def reset():
+        h.copy_(h0)
+        root.copy_(r0)
+        pl.copy_(p0)
+
+    def steps():
+        for r in range(R):
+            loop.step(r, h, root, heads["W1"], heads["b1"], heads["W2"], lm, bm, att["q"],
+                      att["k_new"], att["v_new"], att["Kc"], att["Vc"], pl)
+
+    reset()
+    steps()  # eager warm-up (first-call setup outside the capture)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            steps()
+    torch.cuda.current_stream().wait_stream(side)
+    times, toks = [], []
+    for i in range(max(args.warmup, 3) + args.steps):
+        reset()
+        loop.status.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        assert int(loop.status.item()) == 0, int(loop.status.item())
+        if i >= max(args.warmup, 3):
+            times.append(e0.elapsed_time(e1) / 1e3)
+            toks.append(int(loop.history.sum()) + R * w.B)
+    del graph
+    sec = sum(times)
+    line = {"stage": "loop", "workload": args.workload, "n_nodes": N, "steps_per_graph": R,
+            "graphs": len(times), "us_per_step": sec / (len(times) * R) * 1e6,
+            "tokens_per_s": sum(toks) / sec,
+            "mean_accept_len": (sum(toks) - len(times) * R * w.B) / (len(times) * R * w.B),
+            "tokens_per_step_per_seq": sum(toks) / (len(times) * R * w.B),
+            "base_model": "synthetic node hidden states (p_match %.2f planted matches)" % w.p_match}
+    print(json.dumps(line))
+    return 0
 
 
 def run_stage(args):
@@ -351,6 +432,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.stage == "loop":
+        return run_loop(args)
     if args.stage != "all":
         return run_stage(args)
 
