@@ -45,6 +45,7 @@ int64/int32) and returns new arrays; nothing is modified in place.
 """
 from __future__ import annotations
 
+import itertools
 import math
 from typing import Dict, List, Sequence, Tuple
 
@@ -155,6 +156,44 @@ def tree_build(parent: np.ndarray, depth: np.ndarray, rank: np.ndarray,
             paths.append(path + [-1] * (dmax + 1 - len(path)))
     retrieve = np.array(paths, dtype=np.int32).reshape(len(paths), dmax + 1)
     return {"cand": cand, "pos": pos, "mask": mask, "retrieve": retrieve}
+
+
+def tree_from_accuracies(acc: np.ndarray, n_nodes: int, max_depth: int) -> Dict[str, np.ndarray]:
+    """The sparse tree of the most accurate combinations.
+
+    [GLOSS-TREE]: a sparse tree built from the most accurate combinations of
+    the heads' top choices beats a dense one.  Reading: acc[t-1][r] is the
+    probability that head t's rank-r token is the base model's choice (one
+    rank at most is right, heads independent), so a node with rank path
+    (r1..rt) is accepted with probability prod acc[i-1][r_i], and a tree's
+    expected accept length is the sum of that over its non-root nodes.  The
+    tree keeps the n_nodes - 1 rank paths of depth <= max_depth with the
+    largest products (equal products: lexicographically smaller path first,
+    so a prefix precedes its extensions), plus the root.  Node order: by
+    depth, then lexicographic rank path (parents precede children).
+
+    Written as the definition: every path of depth <= max_depth is scored and
+    sorted.  acc [K, kmax] with values in [0, 1].  Returns parent, depth, rank
+    [N] int32 and the expected accept length."""
+    acc = np.asarray(acc, np.float64)
+    K, kmax = acc.shape
+    D = min(K, max_depth)
+    scored = []
+    for t in range(1, D + 1):
+        for path in itertools.product(range(kmax), repeat=t):
+            prob = 1.0
+            for i, r in enumerate(path):
+                prob *= acc[i, r]
+            scored.append((-prob, path))
+    scored.sort()
+    keep = [path for _, path in scored[:n_nodes - 1]]
+    nodes = [()] + sorted(keep, key=lambda p: (len(p), p))
+    index = {p: i for i, p in enumerate(nodes)}
+    parent = np.array([-1] + [index[p[:-1]] for p in nodes[1:]], dtype=np.int32)
+    depth = np.array([len(p) for p in nodes], dtype=np.int32)
+    rank = np.array([0] + [p[-1] for p in nodes[1:]], dtype=np.int32)
+    expected = float(sum(-s for s, _ in scored[:n_nodes - 1]))
+    return {"parent": parent, "depth": depth, "rank": rank, "expected_accept_len": expected}
 
 
 def mask_bit(mask: np.ndarray, i: int, j: int) -> bool:

@@ -493,3 +493,56 @@ def test_next_step_inputs_take_the_kept_node_and_bonus():
     np.testing.assert_array_equal(h_next[0], hidden[0, 7])
     np.testing.assert_array_equal(h_next[1], hidden[1, 0])
     assert root_next.tolist() == [42, 9]
+
+
+# ----------------------------------------------------------------------------
+# Sparse tree from head accuracies
+# ----------------------------------------------------------------------------
+
+
+def _ancestor_closed_subsets(paths, size):
+    """All subsets of ``paths`` of the given size that contain every prefix
+    of each member (brute force, tiny inputs only)."""
+    pset = set(paths)
+    for combo in itertools.combinations(paths, size):
+        s = set(combo)
+        if all((p[:-1] in s or len(p) == 1) for p in s) and s <= pset:
+            yield s
+
+
+def test_tree_from_accuracies_maximises_expected_accept_length():
+    """Brute force over every ancestor-closed set of rank paths: the tree
+    reaches the largest expected accept length (sum of path products)."""
+    rng = np.random.default_rng(12)
+    for trial in range(12):
+        K, kmax = int(rng.integers(1, 4)), int(rng.integers(1, 4))
+        acc = rng.uniform(0, 1, size=(K, kmax))
+        if trial % 4 == 0:
+            acc[:, 0] = 1.0  # products equal along a path: ties
+        paths = [p for t in range(1, K + 1) for p in itertools.product(range(kmax), repeat=t)]
+        n_nodes = int(rng.integers(1, min(len(paths), 7) + 1)) + 1
+
+        def value(s):
+            return sum(np.prod([acc[i, r] for i, r in enumerate(p)]) for p in s)
+
+        best = max(value(s) for s in _ancestor_closed_subsets(paths, n_nodes - 1))
+        t = O.tree_from_accuracies(acc, n_nodes, K)
+        assert abs(t["expected_accept_len"] - best) < 1e-12
+        assert t["parent"].shape == (n_nodes,)
+        # a valid tree in BFS order
+        for i in range(1, n_nodes):
+            assert 0 <= t["parent"][i] < i
+            assert t["depth"][i] == t["depth"][t["parent"][i]] + 1
+
+
+def test_tree_from_accuracies_glossary_shape():
+    """Head 1 right with 0.6 / 0.3 for ranks 0 / 1, head 2 with 0.5 / 0.3 /
+    0.2 for ranks 0..2 and nothing else: the 9-node tree is the glossary's
+    top-2 x top-3 Cartesian tree."""
+    acc = np.array([[0.6, 0.3, 0.0], [0.5, 0.3, 0.2]])
+    t = O.tree_from_accuracies(acc, 9, 2)
+    ref = W.cartesian_tree([2, 3])
+    np.testing.assert_array_equal(t["parent"], ref.parent)
+    np.testing.assert_array_equal(t["depth"], ref.depth)
+    np.testing.assert_array_equal(t["rank"], ref.rank)
+    assert abs(t["expected_accept_len"] - (0.9 + 0.9 * 1.0)) < 1e-12
