@@ -379,6 +379,33 @@ MEDUSA_API medusa_status_t medusa_next_step(const void* node_hidden, medusa_dtyp
                                             int32_t* root_next, int32_t* dev_status,
                                             void* stream);
 
+/* ------------------------------------------------------------------------
+ * medusa_tree_from_accuracies   (host only: no device memory, no launch)
+ *
+ * "Medusa Heads" glossary, "Attention arborescente et acceptation": a sparse
+ * tree built from the most accurate combinations of the heads' top choices
+ * beats a dense one.
+ *
+ * acc [n_heads * kmax] (host, row-major): acc[t-1][r] = probability that head
+ * t's rank-r token is the base model's choice, in [0, 1].  A node with rank
+ * path (r1..rt) is accepted with probability prod acc[i-1][r_i] (one rank at
+ * most is right, heads independent); the tree holds the root and the
+ * n_nodes - 1 paths of depth <= min(n_heads, max_depth) with the largest
+ * products (equal products: lexicographically smaller path first), which
+ * maximises the expected accept length (the sum of the products, returned in
+ * *expected_accept_len when that pointer is not NULL).  Nodes are numbered by
+ * depth, then lexicographic path: parent[0] = -1, parent[i] < i.
+ * Outputs (host): parent, depth, rank [n_nodes] int32 - the arrays of a
+ *   medusa_tree_t once copied to the device.
+ * Errors: MEDUSA_ERR_SHAPE when fewer than n_nodes - 1 paths exist or a size
+ *   is out of range; MEDUSA_ERR_INVALID_ARG for an accuracy outside [0, 1].
+ * ---------------------------------------------------------------------- */
+MEDUSA_API medusa_status_t medusa_tree_from_accuracies(const float* acc, int n_heads, int kmax,
+                                                       int n_nodes, int max_depth,
+                                                       int32_t* parent, int32_t* depth,
+                                                       int32_t* rank,
+                                                       double* expected_accept_len);
+
 #ifdef __cplusplus
 }
 #endif

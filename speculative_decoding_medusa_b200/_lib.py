@@ -37,6 +37,7 @@ EXPORTS = (
     "medusa_verify_accept_workspace_size", "medusa_verify_accept",
     "medusa_kv_compact", "medusa_verify_accept_noalloc",
     "medusa_lmhead_verify_workspace_size", "medusa_lmhead_verify", "medusa_next_step",
+    "medusa_tree_from_accuracies",
 )
 
 
@@ -94,6 +95,8 @@ def lib() -> ctypes.CDLL:
     L.medusa_kv_compact.argtypes = [_V, _V, _I, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V, _V]
     L.medusa_lmhead_verify_workspace_size.restype = _Z
     L.medusa_lmhead_verify_workspace_size.argtypes = [_I, _I, _I, _I]
+    L.medusa_tree_from_accuracies.restype = _I
+    L.medusa_tree_from_accuracies.argtypes = [_V, _I, _I, _I, _I, _V, _V, _V, _V]
     L.medusa_next_step.restype = _I
     L.medusa_next_step.argtypes = [_V, _I, _V, _V, _V, _I, _I, _I, _I, _V, _V, _V, _V]
     L.medusa_lmhead_verify.restype = _I
@@ -309,3 +312,18 @@ def medusa_next_step(node_hidden, accept_len, accepted_nodes, bonus, h_next, roo
     _check(lib().medusa_next_step(_p(node_hidden), _dt(node_hidden), _p(accept_len),
                                   _p(accepted_nodes), _p(bonus), B, N, d, max_depth, _p(h_next),
                                   _p(root_next), _p(dev_status), _stream(stream)))
+
+
+def medusa_tree_from_accuracies(acc, n_nodes: int, max_depth: int):
+    """acc [K, kmax] (array-like, probabilities) -> (parent, depth, rank)
+    int32 numpy arrays of the n_nodes-node tree of the most accurate
+    combinations, and its expected accept length.  Host only."""
+    import numpy as np
+    a = np.ascontiguousarray(np.asarray(acc, dtype=np.float32))
+    K, kmax = a.shape
+    out = [np.zeros(n_nodes, dtype=np.int32) for _ in range(3)]
+    e = ctypes.c_double(0.0)
+    _check(lib().medusa_tree_from_accuracies(a.ctypes.data, K, kmax, n_nodes, max_depth,
+                                             out[0].ctypes.data, out[1].ctypes.data,
+                                             out[2].ctypes.data, ctypes.byref(e)))
+    return out[0], out[1], out[2], e.value

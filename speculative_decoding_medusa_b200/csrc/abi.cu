@@ -242,6 +242,22 @@ medusa_status_t medusa_next_step(const void* node_hidden, medusa_dtype_t dt,
                            h_next, root_next, dev_status, static_cast<cudaStream_t>(stream));
 }
 
+medusa_status_t medusa_tree_from_accuracies(const float* acc, int n_heads, int kmax,
+                                            int n_nodes, int max_depth, int32_t* parent,
+                                            int32_t* depth, int32_t* rank,
+                                            double* expected_accept_len) {
+  if (!acc || !parent || !depth || !rank)
+    return fail(MEDUSA_ERR_INVALID_ARG, "tree_from_accuracies: null pointer");
+  if (n_heads < 1 || n_heads > MEDUSA_MAX_HEADS || kmax < 1 || kmax > MEDUSA_MAX_KMAX ||
+      n_nodes < 1 || n_nodes > MEDUSA_MAX_NODES || max_depth < 1)
+    return fail(MEDUSA_ERR_SHAPE, "tree_from_accuracies: sizes out of range");
+  for (int i = 0; i < n_heads * kmax; ++i)
+    if (!(acc[i] >= 0.f && acc[i] <= 1.f))
+      return fail(MEDUSA_ERR_INVALID_ARG, "tree_from_accuracies: accuracies must be in [0, 1]");
+  return medusa::tree_from_accuracies(acc, n_heads, kmax, n_nodes, max_depth, parent, depth, rank,
+                                      expected_accept_len);
+}
+
 medusa_status_t medusa_kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
                                   const int32_t* accepted_nodes, const int32_t* accept_len, int B,
                                   int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,

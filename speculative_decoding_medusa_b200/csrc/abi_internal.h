@@ -87,6 +87,10 @@ medusa_status_t next_step(const void* node_hidden, int elem_bytes, const int32_t
                           int d, int max_depth, void* h_next, int32_t* root_next,
                           int32_t* status, cudaStream_t stream);
 
+medusa_status_t tree_from_accuracies(const float* acc, int n_heads, int kmax, int n_nodes,
+                                     int max_depth, int32_t* parent, int32_t* depth,
+                                     int32_t* rank, double* expected_accept_len);
+
 medusa_status_t kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
                            const int32_t* accepted_nodes, const int32_t* accept_len, int B,
                            int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,
