@@ -394,6 +394,55 @@ def kv_compact(Kc: np.ndarray, Vc: np.ndarray, prefix_len: np.ndarray,
 # ---------------------------------------------------------------------------
 
 
+def philox4x32_10(counter: Sequence[int], key: Sequence[int]) -> List[int]:
+    """The Philox4x32-10 counter-based generator as published by Salmon,
+    Moraes, Dror and Shaw ("Parallel Random Numbers: As Easy as 1, 2, 3",
+    SC 2011): ten rounds of two 32x32 -> 64-bit multiplications with the
+    multipliers 0xD2511F53 and 0xCD9E8D57, the high halves xored with the
+    other counter words and the key, the key bumped by 0x9E3779B9 and
+    0xBB67AE85 after each round.  counter: 4 words, key: 2 words."""
+    c = [int(x) & 0xFFFFFFFF for x in counter]
+    k = [int(x) & 0xFFFFFFFF for x in key]
+    for rnd in range(10):
+        p0 = 0xD2511F53 * c[0]
+        p1 = 0xCD9E8D57 * c[2]
+        hi0, lo0 = p0 >> 32, p0 & 0xFFFFFFFF
+        hi1, lo1 = p1 >> 32, p1 & 0xFFFFFFFF
+        c = [hi1 ^ c[1] ^ k[0], lo1, hi0 ^ c[3] ^ k[1], lo0]
+        if rnd < 9:
+            k = [(k[0] + 0x9E3779B9) & 0xFFFFFFFF, (k[1] + 0xBB67AE85) & 0xFFFFFFFF]
+    return c
+
+
+def bonus_uniform(seed: int, offset: int, b: int) -> float:
+    """The uniform number of sequence b: the top 24 bits of the first Philox
+    word for key (seed low, seed high) and counter (offset low, offset high,
+    b, 0), as a multiple of 2^-24 in [0, 1)."""
+    x = philox4x32_10([offset & 0xFFFFFFFF, (offset >> 32) & 0xFFFFFFFF, b, 0],
+                      [seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF])[0]
+    return (x >> 8) * 2.0 ** -24
+
+
+def sample_bonus(logits: np.ndarray, accept_len: np.ndarray, accepted_nodes: np.ndarray,
+                 temperature: float, seed: int, offset: int) -> np.ndarray:
+    """A sampled bonus token: at the kept node, the first token whose
+    cumulative probability under softmax(logits / T) exceeds the sequence's
+    uniform number (inverse CDF).  [DEPLOY-PT]: the token the base model
+    generates itself at the kept node - here drawn from its distribution
+    rather than taken as its first choice.  logits [B, N, V]."""
+    logits = np.asarray(logits, np.float64)
+    B = logits.shape[0]
+    out = np.zeros(B, dtype=np.int32)
+    for b in range(B):
+        kept = int(accepted_nodes[b, int(accept_len[b])])
+        zt = logits[b, kept] / temperature
+        p = np.exp(zt - zt.max())
+        cdf = np.cumsum(p) / p.sum()
+        u = bonus_uniform(seed, offset, b)
+        out[b] = min(int(np.searchsorted(cdf, u, side="right")), logits.shape[2] - 1)
+    return out
+
+
 def next_step_inputs(node_hidden: np.ndarray, accept_len: np.ndarray,
                      accepted_nodes: np.ndarray, bonus: np.ndarray
                      ) -> Tuple[np.ndarray, np.ndarray]:

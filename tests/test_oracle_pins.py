@@ -546,3 +546,37 @@ def test_tree_from_accuracies_glossary_shape():
     np.testing.assert_array_equal(t["depth"], ref.depth)
     np.testing.assert_array_equal(t["rank"], ref.rank)
     assert abs(t["expected_accept_len"] - (0.9 + 0.9 * 1.0)) < 1e-12
+
+
+# ----------------------------------------------------------------------------
+# Sampled bonus token (Philox4x32-10, inverse CDF)
+# ----------------------------------------------------------------------------
+
+
+def test_philox_known_answers():
+    """Known-answer vectors of Philox4x32-10 from the reference distribution
+    of Salmon et al., SC 2011 (zero, all-ones and pi-digit counter/key)."""
+    assert O.philox4x32_10([0, 0, 0, 0], [0, 0]) == [0x6627E8D5, 0xE169C58D, 0xBC57AC4C, 0x9B00DBD8]
+    assert O.philox4x32_10([0xFFFFFFFF] * 4, [0xFFFFFFFF] * 2) == \
+        [0x408F276D, 0x41C83B0E, 0xA20BC7C6, 0x6D5451FD]
+    assert O.philox4x32_10([0x243F6A88, 0x85A308D3, 0x13198A2E, 0x03707344],
+                           [0xA4093822, 0x299F31D0]) == \
+        [0xD16CFE09, 0x94FDCCEB, 0x5001E420, 0x24126EA1]
+
+
+def test_sample_bonus_closed_forms():
+    """Uniform row: the token is floor(u * V).  A row with one logit far
+    above the rest: always that token.  The kept node's row is the one read."""
+    B, N, V = 5, 3, 1000
+    logits = np.zeros((B, N, V))
+    nodes = np.array([[0, 2, -1]] * B, dtype=np.int32)
+    acc = np.ones(B, dtype=np.int32)  # kept node 2
+    logits[:, 0, 7] = 1e3            # the root row must not be read
+    got = O.sample_bonus(logits, acc, nodes, 0.9, 1234, 5)
+    for b in range(B):
+        assert got[b] == int(O.bonus_uniform(1234, 5, b) * V)
+    logits[:, 2, 321] = 200.0
+    assert (O.sample_bonus(logits, acc, nodes, 1.0, 99, 0) == 321).all()
+    # different offsets give different draws
+    us = {O.bonus_uniform(7, off, 0) for off in range(8)}
+    assert len(us) == 8
