@@ -380,6 +380,40 @@ MEDUSA_API medusa_status_t medusa_next_step(const void* node_hidden, medusa_dtyp
                                             void* stream);
 
 /* ------------------------------------------------------------------------
+ * medusa_sample_bonus
+ *
+ * "Medusa no contexto de LLMs", "o que significa medusa na prática de
+ * deploy": the token the base model generates itself at the kept node enters
+ * the sequence after the kept candidates.  medusa_verify_accept writes its
+ * first choice; this call replaces it with a draw from the base model's
+ * distribution there, p = softmax(logits[b][kept] / temperature):
+ *
+ *   x = first word of Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel
+ *       Random Numbers: As Easy as 1, 2, 3", SC 2011) with key
+ *       (seed low 32 bits, seed high 32 bits) and counter (offset low,
+ *       offset high, b, 0);  u = (x >> 8) * 2^-24 in [0, 1);
+ *   token = the first v whose cumulative probability exceeds u.
+ *
+ * Call it after medusa_verify_accept on the same logits; it overwrites
+ * bonus[b] and accepted_tokens[b][accept_len[b]].  Advance offset between
+ * steps for fresh draws.  The cumulative sums are fp32 (chunked scan), so a u
+ * within about 1e-6 of a boundary may select the neighbouring token of an
+ * fp64 inverse CDF.
+ * Inputs (device): logits [B, N, V] of dtype dt; accept_len [B] and
+ *   accepted_nodes [B, max_depth+1] int32 from the verification.
+ * Outputs (device): bonus [B], accepted_tokens [B, max_depth+1] (one entry).
+ * Limits: temperature > 0.  Device checks: a kept node outside [0, N), a
+ *   row with no probability mass (NaN logits).
+ * ---------------------------------------------------------------------- */
+MEDUSA_API medusa_status_t medusa_sample_bonus(const void* logits, medusa_dtype_t dt,
+                                               const int32_t* accept_len,
+                                               const int32_t* accepted_nodes, int B, int N,
+                                               int V, int max_depth, float temperature,
+                                               uint64_t seed, uint64_t offset, int32_t* bonus,
+                                               int32_t* accepted_tokens, int32_t* dev_status,
+                                               void* stream);
+
+/* ------------------------------------------------------------------------
  * medusa_tree_from_accuracies   (host only: no device memory, no launch)
  *
  * "Medusa Heads" glossary, "Attention arborescente et acceptation": a sparse

@@ -37,7 +37,7 @@ EXPORTS = (
     "medusa_verify_accept_workspace_size", "medusa_verify_accept",
     "medusa_kv_compact", "medusa_verify_accept_noalloc",
     "medusa_lmhead_verify_workspace_size", "medusa_lmhead_verify", "medusa_next_step",
-    "medusa_tree_from_accuracies",
+    "medusa_tree_from_accuracies", "medusa_sample_bonus",
 )
 
 
@@ -95,6 +95,9 @@ def lib() -> ctypes.CDLL:
     L.medusa_kv_compact.argtypes = [_V, _V, _I, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V, _V]
     L.medusa_lmhead_verify_workspace_size.restype = _Z
     L.medusa_lmhead_verify_workspace_size.argtypes = [_I, _I, _I, _I]
+    L.medusa_sample_bonus.restype = _I
+    L.medusa_sample_bonus.argtypes = [_V, _I, _V, _V, _I, _I, _I, _I, _F, ctypes.c_uint64,
+                                      ctypes.c_uint64, _V, _V, _V, _V]
     L.medusa_tree_from_accuracies.restype = _I
     L.medusa_tree_from_accuracies.argtypes = [_V, _I, _I, _I, _I, _V, _V, _V, _V]
     L.medusa_next_step.restype = _I
@@ -327,3 +330,17 @@ def medusa_tree_from_accuracies(acc, n_nodes: int, max_depth: int):
                                              out[0].ctypes.data, out[1].ctypes.data,
                                              out[2].ctypes.data, ctypes.byref(e)))
     return out[0], out[1], out[2], e.value
+
+
+def medusa_sample_bonus(logits, accept_len, accepted_nodes, bonus, accepted_tokens,
+                        temperature: float, seed: int, offset: int = 0, dev_status=None,
+                        stream=None) -> None:
+    """Redraw the bonus token of each sequence from softmax(logits/T) at the
+    kept node (Philox4x32-10, inverse CDF); updates bonus and accepted_tokens."""
+    _req(logits, "logits")
+    B, N, V = logits.shape
+    max_depth = accepted_nodes.shape[1] - 1
+    _check(lib().medusa_sample_bonus(_p(logits), _dt(logits), _p(accept_len), _p(accepted_nodes),
+                                     B, N, V, max_depth, float(temperature), int(seed),
+                                     int(offset), _p(bonus), _p(accepted_tokens), _p(dev_status),
+                                     _stream(stream)))

@@ -258,6 +258,24 @@ medusa_status_t medusa_tree_from_accuracies(const float* acc, int n_heads, int k
                                       expected_accept_len);
 }
 
+medusa_status_t medusa_sample_bonus(const void* logits, medusa_dtype_t dt,
+                                    const int32_t* accept_len, const int32_t* accepted_nodes,
+                                    int B, int N, int V, int max_depth, float temperature,
+                                    uint64_t seed, uint64_t offset, int32_t* bonus,
+                                    int32_t* accepted_tokens, int32_t* dev_status, void* stream) {
+  if (!logits || !accept_len || !accepted_nodes || !bonus || !accepted_tokens)
+    return fail(MEDUSA_ERR_INVALID_ARG, "sample_bonus: null pointer");
+  if (!valid_dtype(dt)) return fail(MEDUSA_ERR_INVALID_ARG, "sample_bonus: bad dtype");
+  if (B < 1 || B > 65535 || N < 1 || N > MEDUSA_MAX_NODES || V < 1 || max_depth < 0 ||
+      max_depth >= MEDUSA_MAX_HEADS)
+    return fail(MEDUSA_ERR_SHAPE, "sample_bonus: B, N, V or max_depth out of range");
+  if (!(temperature > 0.f))
+    return fail(MEDUSA_ERR_INVALID_ARG, "sample_bonus: temperature must be > 0");
+  return medusa::sample_bonus(logits, dt, accept_len, accepted_nodes, B, N, V, max_depth,
+                              temperature, seed, offset, bonus, accepted_tokens, dev_status,
+                              static_cast<cudaStream_t>(stream));
+}
+
 medusa_status_t medusa_kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
                                   const int32_t* accepted_nodes, const int32_t* accept_len, int B,
                                   int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,

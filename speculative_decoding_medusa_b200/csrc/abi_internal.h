@@ -91,6 +91,11 @@ medusa_status_t tree_from_accuracies(const float* acc, int n_heads, int kmax, in
                                      int max_depth, int32_t* parent, int32_t* depth,
                                      int32_t* rank, double* expected_accept_len);
 
+medusa_status_t sample_bonus(const void* logits, medusa_dtype_t dt, const int32_t* accept_len,
+                             const int32_t* accepted_nodes, int B, int N, int V, int max_depth,
+                             float temperature, uint64_t seed, uint64_t offset, int32_t* bonus,
+                             int32_t* accepted_tokens, int32_t* status, cudaStream_t stream);
+
 medusa_status_t kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
                            const int32_t* accepted_nodes, const int32_t* accept_len, int B,
                            int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,
