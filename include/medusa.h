@@ -380,6 +380,70 @@ MEDUSA_API medusa_status_t medusa_next_step(const void* node_hidden, medusa_dtyp
                                             void* stream);
 
 /* ------------------------------------------------------------------------
+ * Vocabulary sharding (several GPUs, each holding a slice of the vocabulary)
+ *
+ * No counterpart on the pages; these calls split medusa_heads_topk and
+ * medusa_verify_accept at their only reduction over the vocabulary, so that
+ * a caller can keep W2 rows and verify logits for tokens [v_offset,
+ * v_offset + V_shard) on each GPU and exchange a few KB between them (for
+ * example one all-gather and one max all-reduce).  The arithmetic of every
+ * shard and of the merge runs here; the exchange is the caller's.
+ *
+ * A row record summarises one row of logits over a set of tokens: its
+ * largest logit, the lowest token id holding it, and for typical acceptance
+ * s = sum exp(z/T - maxz/T) and t = sum exp(z/T - maxz/T) * z/T.
+ * ---------------------------------------------------------------------- */
+typedef struct medusa_row_record {
+  float maxz;
+  int32_t idx;
+  float s;
+  float t;
+} medusa_row_record_t;
+
+/* medusa_topk_merge: the best kmax of n_lists lists of list_len candidates
+ * per row (values descending, equal values by ascending id).  Candidate j of
+ * list g of row r is vals/ids[r * row_stride + g * list_stride + j] (device);
+ * its id gains id_offsets[g] (device int32 [n_lists], or NULL).  With the
+ * per-shard outputs of medusa_heads_topk all-gathered as [G][B*K][kmax]:
+ * rows = B*K, n_lists = G, list_len = kmax, row_stride = kmax, list_stride =
+ * B*K*kmax, id_offsets = each shard's first token.  Outputs (device):
+ * topk_ids, topk_vals [rows, kmax].  Limits: kmax <= MEDUSA_MAX_KMAX and
+ * <= n_lists * list_len; rows <= 65535. */
+MEDUSA_API medusa_status_t medusa_topk_merge(const float* vals, const int32_t* ids, int rows,
+                                             int n_lists, int list_len, long long row_stride,
+                                             long long list_stride, const int32_t* id_offsets,
+                                             int kmax, int32_t* topk_ids, float* topk_vals,
+                                             void* stream);
+
+/* medusa_verify_records: this shard's row records and candidate logits.
+ * Inputs (device): logits [B, N, V_shard] of dtype dt (tokens v_offset ..
+ * v_offset + V_shard - 1), cand_ids [B, N] (global token ids), tree.
+ * Outputs (device): records [B*N] (token ids global); cand_logit [B*N]
+ * float: node c's candidate token's logit at its parent when that token is in
+ * this shard, else -inf (root: -inf).  Workspace:
+ * medusa_verify_records_workspace_size(B, N, V_shard) bytes, 256-aligned. */
+MEDUSA_API size_t medusa_verify_records_workspace_size(int B, int N, int V_shard);
+MEDUSA_API medusa_status_t medusa_verify_records(const void* logits, medusa_dtype_t dt,
+                                                 const int32_t* cand_ids,
+                                                 const medusa_tree_t* tree, int B, int V_shard,
+                                                 int v_offset, medusa_accept_t mode,
+                                                 float temperature,
+                                                 medusa_row_record_t* records, float* cand_logit,
+                                                 void* ws, size_t ws_bytes, int32_t* dev_status,
+                                                 void* stream);
+
+/* medusa_verify_from_records: the verification of medusa_verify_accept from
+ * the G shards' records, shard-major [G][B*N] (device), and the candidate
+ * logits [B*N] maximised over the shards (device; typical mode only, may be
+ * NULL for greedy).  V is the full vocabulary size.  Outputs as
+ * medusa_verify_accept. */
+MEDUSA_API medusa_status_t medusa_verify_from_records(
+    const medusa_row_record_t* records, int G, const float* cand_logit, const int32_t* cand_ids,
+    const medusa_tree_t* tree, int B, int V, medusa_accept_t mode, float temperature, float eps,
+    float delta, int32_t* accept_len, int32_t* accepted_nodes, int32_t* accepted_tokens,
+    int32_t* bonus, int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
  * medusa_sample_bonus
  *
  * "Medusa no contexto de LLMs", "o que significa medusa na prática de

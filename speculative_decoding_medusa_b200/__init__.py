@@ -8,7 +8,8 @@ from ._lib import (  # noqa: F401
     EXPORTS, LIB_PATH, MEDUSA_ACCEPT_GREEDY, MEDUSA_ACCEPT_TYPICAL, MEDUSA_BF16, MEDUSA_F32,
     MedusaError, Tree, lib, medusa_heads_topk, medusa_heads_topk_workspace_size,
     medusa_kv_compact, medusa_lmhead_verify, medusa_lmhead_verify_workspace_size,
-    medusa_next_step, medusa_sample_bonus, medusa_tree_from_accuracies,
+    medusa_next_step, medusa_sample_bonus, medusa_topk_merge, medusa_tree_from_accuracies,
+    medusa_verify_from_records, medusa_verify_records, medusa_verify_records_workspace_size,
     medusa_tree_attention, medusa_tree_attention_workspace_size,
     medusa_tree_build, medusa_verify_accept, medusa_verify_accept_noalloc,
     medusa_verify_accept_workspace_size, new_status,

@@ -37,7 +37,8 @@ EXPORTS = (
     "medusa_verify_accept_workspace_size", "medusa_verify_accept",
     "medusa_kv_compact", "medusa_verify_accept_noalloc",
     "medusa_lmhead_verify_workspace_size", "medusa_lmhead_verify", "medusa_next_step",
-    "medusa_tree_from_accuracies", "medusa_sample_bonus",
+    "medusa_tree_from_accuracies", "medusa_sample_bonus", "medusa_topk_merge",
+    "medusa_verify_records_workspace_size", "medusa_verify_records", "medusa_verify_from_records",
 )
 
 
@@ -95,6 +96,17 @@ def lib() -> ctypes.CDLL:
     L.medusa_kv_compact.argtypes = [_V, _V, _I, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V, _V]
     L.medusa_lmhead_verify_workspace_size.restype = _Z
     L.medusa_lmhead_verify_workspace_size.argtypes = [_I, _I, _I, _I]
+    _LL = ctypes.c_longlong
+    L.medusa_topk_merge.restype = _I
+    L.medusa_topk_merge.argtypes = [_V, _V, _I, _I, _I, _LL, _LL, _V, _I, _V, _V, _V]
+    L.medusa_verify_records_workspace_size.restype = _Z
+    L.medusa_verify_records_workspace_size.argtypes = [_I, _I, _I]
+    L.medusa_verify_records.restype = _I
+    L.medusa_verify_records.argtypes = [_V, _I, _V, ctypes.POINTER(medusa_tree_t), _I, _I, _I, _I,
+                                        _F, _V, _V, _V, _Z, _V, _V]
+    L.medusa_verify_from_records.restype = _I
+    L.medusa_verify_from_records.argtypes = [_V, _I, _V, _V, ctypes.POINTER(medusa_tree_t), _I, _I,
+                                             _I, _F, _F, _F, _V, _V, _V, _V, _V, _V]
     L.medusa_sample_bonus.restype = _I
     L.medusa_sample_bonus.argtypes = [_V, _I, _V, _V, _I, _I, _I, _I, _F, ctypes.c_uint64,
                                       ctypes.c_uint64, _V, _V, _V, _V]
@@ -344,3 +356,52 @@ def medusa_sample_bonus(logits, accept_len, accepted_nodes, bonus, accepted_toke
                                      B, N, V, max_depth, float(temperature), int(seed),
                                      int(offset), _p(bonus), _p(accepted_tokens), _p(dev_status),
                                      _stream(stream)))
+
+
+def medusa_topk_merge(vals, ids, rows: int, n_lists: int, list_len: int, row_stride: int,
+                      list_stride: int, id_offsets, kmax: int, topk_ids, topk_vals,
+                      stream=None) -> None:
+    """Best kmax of n_lists candidate lists per row (see include/medusa.h)."""
+    _req(vals, "vals")
+    _req(ids, "ids")
+    _check(lib().medusa_topk_merge(_p(vals), _p(ids), rows, n_lists, list_len, int(row_stride),
+                                   int(list_stride), _p(id_offsets), kmax, _p(topk_ids),
+                                   _p(topk_vals), _stream(stream)))
+
+
+def medusa_verify_records_workspace_size(B: int, N: int, V_shard: int) -> int:
+    return int(lib().medusa_verify_records_workspace_size(B, N, V_shard))
+
+
+def medusa_verify_records(logits, cand_ids, tree: Tree, v_offset: int, records, cand_logit,
+                          mode: int = MEDUSA_ACCEPT_GREEDY, temperature: float = 1.0, ws=None,
+                          dev_status=None, stream=None) -> None:
+    """This vocabulary shard's row records ([B*N, 4] float32 view of
+    medusa_row_record_t) and candidate logits ([B*N] float32)."""
+    _req(logits, "logits")
+    B, N, Vs = logits.shape
+    if ws is None:
+        ws = workspace(medusa_verify_records_workspace_size(B, N, Vs), logits.device)
+    ct = tree.c()
+    _check(lib().medusa_verify_records(_p(logits), _dt(logits), _p(cand_ids), ctypes.byref(ct), B,
+                                       Vs, v_offset, mode, float(temperature), _p(records),
+                                       _p(cand_logit), _p(ws), ws.numel(), _p(dev_status),
+                                       _stream(stream)))
+
+
+def medusa_verify_from_records(records, cand_logit, cand_ids, tree: Tree, V: int, accept_len,
+                               accepted_nodes, accepted_tokens, bonus,
+                               mode: int = MEDUSA_ACCEPT_GREEDY, temperature: float = 1.0,
+                               eps: float = 0.09, delta: float = 0.3, dev_status=None,
+                               stream=None) -> None:
+    """Verification from G shards' records [G, B*N, 4] and the candidate
+    logits maximised over the shards [B*N] (typical only)."""
+    _req(records, "records")
+    G = records.shape[0]
+    B = cand_ids.shape[0]
+    ct = tree.c()
+    _check(lib().medusa_verify_from_records(_p(records), G, _p(cand_logit), _p(cand_ids),
+                                            ctypes.byref(ct), B, V, mode, float(temperature),
+                                            float(eps), float(delta), _p(accept_len),
+                                            _p(accepted_nodes), _p(accepted_tokens), _p(bonus),
+                                            _p(dev_status), _stream(stream)))

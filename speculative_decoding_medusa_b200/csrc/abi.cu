@@ -276,6 +276,77 @@ medusa_status_t medusa_sample_bonus(const void* logits, medusa_dtype_t dt,
                               static_cast<cudaStream_t>(stream));
 }
 
+medusa_status_t medusa_topk_merge(const float* vals, const int32_t* ids, int rows, int n_lists,
+                                  int list_len, long long row_stride, long long list_stride,
+                                  const int32_t* id_offsets, int kmax, int32_t* topk_ids,
+                                  float* topk_vals, void* stream) {
+  if (!vals || !ids || !topk_ids || !topk_vals)
+    return fail(MEDUSA_ERR_INVALID_ARG, "topk_merge: null pointer");
+  if (rows < 1 || rows > 65535 || n_lists < 1 || list_len < 1 || kmax < 1 ||
+      kmax > MEDUSA_MAX_KMAX || (long long)n_lists * list_len < kmax || row_stride < 0 ||
+      list_stride < 0)
+    return fail(MEDUSA_ERR_SHAPE, "topk_merge: sizes out of range");
+  return medusa::topk_merge_lists(vals, ids, rows, n_lists, list_len, row_stride, list_stride,
+                                  id_offsets, kmax, topk_ids, topk_vals,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+size_t medusa_verify_records_workspace_size(int B, int N, int V_shard) {
+  if (B < 1 || N < 1 || V_shard < 1) return 0;
+  return medusa::verify_records_workspace_size(B, N, V_shard);
+}
+
+medusa_status_t medusa_verify_records(const void* logits, medusa_dtype_t dt,
+                                      const int32_t* cand_ids, const medusa_tree_t* tree, int B,
+                                      int V_shard, int v_offset, medusa_accept_t mode,
+                                      float temperature, medusa_row_record_t* records,
+                                      float* cand_logit, void* ws, size_t ws_bytes,
+                                      int32_t* dev_status, void* stream) {
+  medusa_status_t st = check_tree(tree);
+  if (st != MEDUSA_OK) return st;
+  if (!logits || !cand_ids || !records || !cand_logit)
+    return fail(MEDUSA_ERR_INVALID_ARG, "verify_records: null pointer");
+  if (!valid_dtype(dt)) return fail(MEDUSA_ERR_INVALID_ARG, "verify_records: bad dtype");
+  if (mode != MEDUSA_ACCEPT_GREEDY && mode != MEDUSA_ACCEPT_TYPICAL)
+    return fail(MEDUSA_ERR_INVALID_ARG, "verify_records: bad mode");
+  if (B < 1 || V_shard < 1 || v_offset < 0 || (long long)B * tree->n_nodes > 65535)
+    return fail(MEDUSA_ERR_SHAPE, "verify_records: B, V_shard or v_offset out of range");
+  if (mode == MEDUSA_ACCEPT_TYPICAL && !(temperature > 0.f))
+    return fail(MEDUSA_ERR_INVALID_ARG, "verify_records: temperature must be > 0");
+  if (!aligned16(logits)) return fail(MEDUSA_ERR_ALIGNMENT, "verify_records: logits not 16-byte aligned");
+  const size_t need = medusa::verify_records_workspace_size(B, tree->n_nodes, V_shard);
+  if (ws == nullptr || ws_bytes < need || !aligned256(ws))
+    return fail(MEDUSA_ERR_WORKSPACE, "verify_records: workspace null, misaligned or too small");
+  return medusa::verify_records(logits, dt, cand_ids, *tree, B, V_shard, v_offset, mode,
+                                temperature, reinterpret_cast<medusa::RowPart*>(records),
+                                cand_logit, ws, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+medusa_status_t medusa_verify_from_records(const medusa_row_record_t* records, int G,
+                                           const float* cand_logit, const int32_t* cand_ids,
+                                           const medusa_tree_t* tree, int B, int V,
+                                           medusa_accept_t mode, float temperature, float eps,
+                                           float delta, int32_t* accept_len,
+                                           int32_t* accepted_nodes, int32_t* accepted_tokens,
+                                           int32_t* bonus, int32_t* dev_status, void* stream) {
+  medusa_status_t st = check_tree(tree);
+  if (st != MEDUSA_OK) return st;
+  if (!records || !cand_ids || !accept_len || !accepted_nodes || !accepted_tokens || !bonus ||
+      (mode == MEDUSA_ACCEPT_TYPICAL && !cand_logit))
+    return fail(MEDUSA_ERR_INVALID_ARG, "verify_from_records: null pointer");
+  if (mode != MEDUSA_ACCEPT_GREEDY && mode != MEDUSA_ACCEPT_TYPICAL)
+    return fail(MEDUSA_ERR_INVALID_ARG, "verify_from_records: bad mode");
+  if (B < 1 || V < 1 || G < 1 || G > 4096 || (long long)B * tree->n_nodes > 65535)
+    return fail(MEDUSA_ERR_SHAPE, "verify_from_records: B, V or G out of range");
+  if (mode == MEDUSA_ACCEPT_TYPICAL && (!(temperature > 0.f) || !(eps >= 0.f) || !(delta >= 0.f)))
+    return fail(MEDUSA_ERR_INVALID_ARG,
+                "verify_from_records: need temperature > 0, eps >= 0, delta >= 0");
+  return medusa::verify_from_records(reinterpret_cast<const medusa::RowPart*>(records), G,
+                                     cand_logit, cand_ids, *tree, B, V, mode, temperature, eps,
+                                     delta, accept_len, accepted_nodes, accepted_tokens, bonus,
+                                     dev_status, static_cast<cudaStream_t>(stream));
+}
+
 medusa_status_t medusa_kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
                                   const int32_t* accepted_nodes, const int32_t* accept_len, int B,
                                   int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,

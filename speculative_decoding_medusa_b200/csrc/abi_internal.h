@@ -54,6 +54,7 @@ struct RowPart {
   float s;
   float t;
 };
+static_assert(sizeof(RowPart) == sizeof(medusa_row_record_t), "record layout");
 
 // Merges B*N rows of n_chunks RowParts each ([row][chunk], row = b*N + node)
 // and runs the path selection.  Typical acceptance reads the candidate's
@@ -95,6 +96,26 @@ medusa_status_t sample_bonus(const void* logits, medusa_dtype_t dt, const int32_
                              const int32_t* accepted_nodes, int B, int N, int V, int max_depth,
                              float temperature, uint64_t seed, uint64_t offset, int32_t* bonus,
                              int32_t* accepted_tokens, int32_t* status, cudaStream_t stream);
+
+// best kmax of n_lists lists of list_len (value, id) candidates per row;
+// entry (r, g, j) at r * row_stride + g * list_stride + j; ids of list g
+// gain id_offsets[g] (NULL: none)
+medusa_status_t topk_merge_lists(const float* vals, const int32_t* ids, int rows, int n_lists,
+                                 int list_len, long long row_stride, long long list_stride,
+                                 const int32_t* id_offsets, int kmax, int32_t* out_ids,
+                                 float* out_vals, cudaStream_t stream);
+
+size_t verify_records_workspace_size(int B, int N, int V_shard);
+medusa_status_t verify_records(const void* logits, medusa_dtype_t dt, const int32_t* cand_ids,
+                               const medusa_tree_t& tree, int B, int V_shard, int v_offset,
+                               medusa_accept_t mode, float temperature, RowPart* records,
+                               float* cand_logit, void* ws, int32_t* status, cudaStream_t stream);
+medusa_status_t verify_from_records(const RowPart* records, int G, const float* cand_logit,
+                                    const int32_t* cand_ids, const medusa_tree_t& tree, int B,
+                                    int V, medusa_accept_t mode, float temperature, float eps,
+                                    float delta, int32_t* accept_len, int32_t* accepted_nodes,
+                                    int32_t* accepted_tokens, int32_t* bonus, int32_t* status,
+                                    cudaStream_t stream);
 
 medusa_status_t kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
                            const int32_t* accepted_nodes, const int32_t* accept_len, int B,

@@ -303,13 +303,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // 0 of the cluster reads the other CTAs' lists from distributed shared memory
 // and merges them.
 // ----------------------------------------------------------------------------
+// Candidates of row r: C = n_lists * list_len entries; entry e is list
+// g = e / list_len, position j = e % list_len, stored at r * row_stride +
+// g * list_stride + j, and its id gains id_offsets[g] when id_offsets is set.
+// (The heads' own tile lists are one list of C contiguous entries per row.)
+struct MergeLayout {
+  long long row_stride, list_stride;
+  int list_len;
+  const int32_t* id_offsets;
+};
+
 constexpr int kMergeWarps = 8;
 constexpr int kMergeCtas = 8;    // cluster size (portable)
 constexpr int kMergeUnroll = 2;  // 32-candidate chunks each warp has in flight
 
 __global__ void __cluster_dims__(kMergeCtas, 1, 1) __launch_bounds__(kMergeWarps * 32)
     topk_merge_kernel(const float* __restrict__ vals, const int32_t* __restrict__ ids, long long C,
-                      int kmax, int32_t* __restrict__ out_ids, float* __restrict__ out_vals) {
+                      int kmax, int32_t* __restrict__ out_ids, float* __restrict__ out_vals,
+                      MergeLayout lay) {
   __shared__ float sv[kMergeWarps][32];
   __shared__ int si[kMergeWarps][32];
   cg::cluster_group cluster = cg::this_cluster();
@@ -317,7 +328,7 @@ __global__ void __cluster_dims__(kMergeCtas, 1, 1) __launch_bounds__(kMergeWarps
   const long long row = blockIdx.x / kMergeCtas;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const size_t base = (size_t)row * C;
+  const size_t base = (size_t)row * lay.row_stride;
   constexpr long long kStride = (long long)kMergeCtas * kMergeWarps * 32 * kMergeUnroll;
   // running best-32 of this warp, sorted, and its kmax-th entry as a filter
   float rv = -INFINITY;
@@ -334,8 +345,11 @@ __global__ void __cluster_dims__(kMergeCtas, 1, 1) __launch_bounds__(kMergeWarps
       v[u] = -INFINITY;
       i[u] = 0x7fffffff;
       if (e < C) {
-        v[u] = vals[base + e];
-        i[u] = ids != nullptr ? ids[base + e] : static_cast<int>(e);
+        const int g = static_cast<int>(e / lay.list_len);
+        const size_t at = base + (size_t)g * lay.list_stride + (e - (long long)g * lay.list_len);
+        v[u] = vals[at];
+        i[u] = ids != nullptr ? ids[at] : static_cast<int>(e);
+        if (lay.id_offsets != nullptr) i[u] += lay.id_offsets[g];
       }
     }
 #pragma unroll
@@ -427,6 +441,16 @@ __global__ void __launch_bounds__(256)
 // ----------------------------------------------------------------------------
 // host side
 // ----------------------------------------------------------------------------
+medusa_status_t topk_merge_lists(const float* vals, const int32_t* ids, int rows, int n_lists,
+                                 int list_len, long long row_stride, long long list_stride,
+                                 const int32_t* id_offsets, int kmax, int32_t* out_ids,
+                                 float* out_vals, cudaStream_t stream) {
+  const MergeLayout lay{row_stride, list_stride, list_len, id_offsets};
+  topk_merge_kernel<<<rows * kMergeCtas, kMergeWarps * 32, 0, stream>>>(
+      vals, ids, (long long)n_lists * list_len, kmax, out_ids, out_vals, lay);
+  return check_launch("topk_merge");
+}
+
 namespace {
 
 // bf16 tensor [dim2][dim1][dim0] (dim0 contiguous), box {64, box1, 1}
@@ -515,8 +539,10 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
         y, static_cast<const float*>(W2), B, d, V, K, z);
     st = check_launch("heads_f32_w2");
     if (st != MEDUSA_OK) return st;
+    const MergeLayout lay{(long long)V, (long long)V, V, nullptr};
     topk_merge_kernel<<<B * K * kMergeCtas, kMergeWarps * 32, 0, stream>>>(z, nullptr, V, kmax,
-                                                                            topk_ids, topk_vals);
+                                                                            topk_ids, topk_vals,
+                                                                            lay);
     return check_launch("topk_merge");
   }
 
@@ -558,8 +584,10 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
   st = launch_gemm_nb<kModeW2>(nb2, mA2, mB2, p2, stream);
   if (st != MEDUSA_OK) return st;
 
+  const long long C = (long long)p2.tiles_per_head * kmax;
+  const MergeLayout lay{C, C, (int)C, nullptr};
   topk_merge_kernel<<<B * K * kMergeCtas, kMergeWarps * 32, 0, stream>>>(
-      part_vals, part_ids, (long long)p2.tiles_per_head * kmax, kmax, topk_ids, topk_vals);
+      part_vals, part_ids, C, kmax, topk_ids, topk_vals, lay);
   return check_launch("topk_merge");
 }
 

@@ -240,7 +240,8 @@ template <typename T>
 __global__ void __launch_bounds__(kPathThreads)
     verify_path_kernel(const T* __restrict__ logits, const __nv_bfloat16* __restrict__ hidden,
                        const __nv_bfloat16* __restrict__ lm_head, int d,
-                       const RowPart* __restrict__ part, int n_chunks, int tpn,
+                       const RowPart* __restrict__ part, int n_chunks, long long row_stride,
+                       long long chunk_stride, int tpn, const float* __restrict__ cand_logit,
                        const int32_t* __restrict__ cand_ids,
                        const int32_t* __restrict__ parent, const int32_t* __restrict__ depth,
                        int N, int max_depth, int V, int typical, float inv_T, float eps,
@@ -278,13 +279,13 @@ __global__ void __launch_bounds__(kPathThreads)
     // merge the chunks of row (b, node): this thread's share, then the group
     const int node = i / tpn, sub = i - node * tpn;
     const bool active = node < N;
-    const RowPart* rp = part + ((size_t)b * N + (active ? node : 0)) * n_chunks;
+    const RowPart* rp = part + ((size_t)b * N + (active ? node : 0)) * row_stride;
     float bv = -INFINITY;
     int bi = 0x7fffffff;
     float Mt = -INFINITY, S = 0.f, Tt = 0.f;  // sums relative to exp(Mt)
     if (active) {
       for (int c = sub; c < n_chunks; c += tpn) {
-        const RowPart q = rp[c];
+        const RowPart q = rp[c * chunk_stride];
         if (better(q.maxz, q.idx, bv, bi)) {
           bv = q.maxz;
           bi = q.idx;
@@ -342,7 +343,7 @@ __global__ void __launch_bounds__(kPathThreads)
     }
     return;
   }
-  if (typical && logits == nullptr) {
+  if (typical && logits == nullptr && cand_logit == nullptr) {
     // no materialised logits: z = lm_head[tok] . hidden[b, parent], one warp
     // per node, 16-byte loads (d is a multiple of 64)
     const int warp = i >> 5, lane = i & 31;
@@ -383,8 +384,9 @@ __global__ void __launch_bounds__(kPathThreads)
       } else if (!typical) {
         pass = s_g[pa] == tok;
       } else {
-        const float z = logits != nullptr ? load1<T>(logits + ((size_t)b * N + pa) * V + tok)
-                                          : s_zc[i];
+        const float z = logits != nullptr       ? load1<T>(logits + ((size_t)b * N + pa) * V + tok)
+                        : cand_logit != nullptr ? cand_logit[(size_t)b * N + i]
+                                                : s_zc[i];
         const float lp = z * inv_T - s_lse[pa];
         pass = lp > s_logthr[pa];
       }
@@ -450,9 +452,131 @@ medusa_status_t verify_path_from_parts(const RowPart* part, int n_chunks,
   const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
   const float inv_T = typical ? 1.0f / temperature : 1.0f;
   verify_path_kernel<__nv_bfloat16><<<B, kPathThreads, 0, stream>>>(
-      nullptr, hidden, lm_head, d, part, n_chunks, path_threads_per_node(N, n_chunks), cand_ids,
+      nullptr, hidden, lm_head, d, part, n_chunks, n_chunks, 1, path_threads_per_node(N, n_chunks),
+      nullptr, cand_ids,
       tree.parent, tree.depth, N, tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta,
       accept_len, accepted_nodes, accepted_tokens, bonus, status);
+  return check_launch("verify_path");
+}
+
+// One record per row from a vocabulary shard's chunk records (merged in
+// chunk order, like the path kernel's merge), token ids moved to global by
+// v_offset; and each node's candidate logit at its parent when the candidate
+// token lies in this shard (-inf otherwise, and for the root).
+template <typename T>
+__global__ void __launch_bounds__(256)
+    shard_records_kernel(const T* __restrict__ logits, const RowPart* __restrict__ part,
+                         int n_chunks, const int32_t* __restrict__ cand_ids,
+                         const int32_t* __restrict__ parent, int B, int N, int V_shard,
+                         int v_offset, int typical, float inv_T, RowPart* __restrict__ records,
+                         float* __restrict__ cand_logit, int32_t* status) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= B * N) return;
+  const RowPart* rp = part + (size_t)r * n_chunks;
+  RowPart o;
+  o.maxz = -INFINITY;
+  o.idx = 0x7fffffff;
+  o.s = 0.f;
+  o.t = 0.f;
+  float Mt = -INFINITY;
+  for (int c = 0; c < n_chunks; ++c) {
+    const RowPart q = rp[c];
+    if (better(q.maxz, q.idx, o.maxz, o.idx)) {
+      o.maxz = q.maxz;
+      o.idx = q.idx;
+    }
+    if (typical) {
+      const float mq = q.maxz * inv_T;
+      if (mq > Mt) {
+        const float w = Mt == -INFINITY ? 0.f : expf(Mt - mq);
+        o.s = o.s * w + q.s;
+        o.t = o.t * w + q.t;
+        Mt = mq;
+      } else if (mq != -INFINITY) {
+        const float w = expf(mq - Mt);
+        o.s += q.s * w;
+        o.t += q.t * w;
+      }
+    }
+  }
+  if (o.idx != 0x7fffffff) o.idx += v_offset;
+  records[r] = o;
+  const int b = r / N, i = r - b * N;
+  float z = -INFINITY;
+  if (i > 0) {
+    const int pa = parent[i];
+    const int tok = cand_ids[r];
+    if (pa < 0 || pa >= N) {
+      report(status, MEDUSA_ERR_DEVICE_CHECK);
+    } else if (tok >= v_offset && tok < v_offset + V_shard) {
+      z = load1<T>(logits + ((size_t)b * N + pa) * V_shard + (tok - v_offset));
+    }
+  }
+  cand_logit[r] = z;
+}
+
+size_t verify_records_workspace_size(int B, int N, int V_shard) {
+  return verify_accept_workspace_size(B, N, V_shard);
+}
+
+medusa_status_t verify_records(const void* logits, medusa_dtype_t dt, const int32_t* cand_ids,
+                               const medusa_tree_t& tree, int B, int V_shard, int v_offset,
+                               medusa_accept_t mode, float temperature, RowPart* records,
+                               float* cand_logit, void* ws, int32_t* status, cudaStream_t stream) {
+  const int N = tree.n_nodes;
+  const int n_chunks = (V_shard + kVChunk - 1) / kVChunk;
+  RowPart* part = static_cast<RowPart*>(ws);
+  const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
+  const float inv_T = typical ? 1.0f / temperature : 1.0f;
+  const long long n_items = (long long)B * N * n_chunks;
+  const int grid = (B * N + 255) / 256;
+  if (dt == MEDUSA_BF16) {
+    const __nv_bfloat16* lg = static_cast<const __nv_bfloat16*>(logits);
+    if (typical) {
+      auto k = verify_rows_kernel<__nv_bfloat16, true>;
+      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V_shard, n_chunks, n_items,
+                                                              inv_T, part, status);
+    } else {
+      auto k = verify_rows_kernel<__nv_bfloat16, false>;
+      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V_shard, n_chunks, n_items,
+                                                              inv_T, part, status);
+    }
+    shard_records_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        lg, part, n_chunks, cand_ids, tree.parent, B, N, V_shard, v_offset, typical ? 1 : 0,
+        inv_T, records, cand_logit, status);
+  } else {
+    const float* lg = static_cast<const float*>(logits);
+    if (typical) {
+      auto k = verify_rows_kernel<float, true>;
+      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V_shard, n_chunks, n_items,
+                                                              inv_T, part, status);
+    } else {
+      auto k = verify_rows_kernel<float, false>;
+      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V_shard, n_chunks, n_items,
+                                                              inv_T, part, status);
+    }
+    shard_records_kernel<float><<<grid, 256, 0, stream>>>(
+        lg, part, n_chunks, cand_ids, tree.parent, B, N, V_shard, v_offset, typical ? 1 : 0,
+        inv_T, records, cand_logit, status);
+  }
+  return check_launch("verify_records");
+}
+
+medusa_status_t verify_from_records(const RowPart* records, int G, const float* cand_logit,
+                                    const int32_t* cand_ids, const medusa_tree_t& tree, int B,
+                                    int V, medusa_accept_t mode, float temperature, float eps,
+                                    float delta, int32_t* accept_len, int32_t* accepted_nodes,
+                                    int32_t* accepted_tokens, int32_t* bonus, int32_t* status,
+                                    cudaStream_t stream) {
+  const int N = tree.n_nodes;
+  const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
+  const float inv_T = typical ? 1.0f / temperature : 1.0f;
+  // records are shard-major: [G][B * N]
+  verify_path_kernel<float><<<B, kPathThreads, 0, stream>>>(
+      nullptr, nullptr, nullptr, 0, records, G, 1, (long long)B * N,
+      path_threads_per_node(N, G), cand_logit, cand_ids, tree.parent, tree.depth, N,
+      tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes,
+      accepted_tokens, bonus, status);
   return check_launch("verify_path");
 }
 
@@ -487,7 +611,7 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
     medusa_status_t st = check_launch("verify_rows");
     if (st != MEDUSA_OK) return st;
     verify_path_kernel<__nv_bfloat16><<<B, kPathThreads, 0, stream>>>(
-        lg, nullptr, nullptr, 0, part, n_chunks, tpn, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
+        lg, nullptr, nullptr, 0, part, n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
         typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
         status);
     return check_launch("verify_path");
@@ -505,7 +629,7 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
   medusa_status_t st = check_launch("verify_rows");
   if (st != MEDUSA_OK) return st;
   verify_path_kernel<float><<<B, kPathThreads, 0, stream>>>(
-      lg, nullptr, nullptr, 0, part, n_chunks, tpn, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
+      lg, nullptr, nullptr, 0, part, n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
       typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
       status);
   return check_launch("verify_path");
