@@ -13,6 +13,13 @@
  *                          (greedy match or typical acceptance);
  *   medusa_kv_compact      the kept branch's K/V moved into contiguous slots.
  *
+ * Around them: medusa_lmhead_verify (the verification from the nodes' hidden
+ * states, lm_head fused), medusa_next_step (inputs of the next step),
+ * medusa_sample_bonus (a drawn bonus token), medusa_tree_from_accuracies
+ * (the sparse tree of the most accurate combinations, host only), the
+ * vocabulary-sharding calls (medusa_topk_merge, medusa_verify_records,
+ * medusa_verify_from_records) and medusa_verify_accept_noalloc.
+ *
  * Sources (page title, then section):
  *   "Medusa Heads" glossary - "Comment les têtes prédisent les tokens
  *     suivants" (the head) and "Attention arborescente et acceptation" (tree,
