@@ -5,21 +5,25 @@
 // candidate tokens are appended to the input at once; a mask lets each one see
 // only its ancestors, so one forward pass scores every branch.
 //
-// bf16 path (tcgen05): split-KV.  A CTA takes 256 query rows of one (sequence,
-// kv head) - the N nodes x G grouped query heads, as two M = 128 tiles - and
-// one split of the keys: a chunk of the cached prefix, or the N tree keys (read
-// from k_new/v_new and masked by the ancestor bitmask).  Roles:
-//   warp 0      TMA producer: 64-key K and V tiles into a 3-stage ring;
-//   warp 1      MMA issuer: S = Q K^T into TMEM (double-buffered per M tile),
-//               then O += P V with P = P_hi + P_lo (two bf16 terms) from
-//               shared memory and V as an M/N-major operand;
+// bf16 path (tcgen05): persistent, stream-K over balanced tiles.  A segment
+// is 256 query rows of one (sequence, kv head) - the N nodes x G grouped query
+// heads, as two M = 128 tiles - and its key tiles: ceil(P/128) prefix tiles,
+// then the tree tiles (k_new/v_new, masked by the ancestor bitmask).  Every
+// CTA takes an equal contiguous range of the concatenated tiles.  Roles:
+//   warp 0      TMA producer: 128-key K and V tiles into a 2-stage ring, with
+//               one word of tile facts per stage;
+//   warp 1      MMA issuer: S = Q K^T into TMEM (one S/P buffer per M tile),
+//               then O += P V with P as packed fp16 in TMEM (over the S
+//               columns) and V as an M/N-major shared-memory operand;
 //   warps 2..9  two softmax warpgroups, one query row per thread: the row's
 //               scores come out of TMEM, max and sum stay in the thread,
 //               O is rescaled in TMEM only when the row maximum grows by more
-//               than 2^8 (the stale maximum cancels in the final O / l).
-// Each CTA writes its normalised partial output and log2-sum-exp; a combine
-// kernel merges the splits.  The tree split of query group 0 also writes the
-// tree K/V into cache slots P + i.
+//               than 2^8 (the stale maximum cancels in the final O / l);
+//   warps 10,11 V converters: each landed V tile is rewritten in place from
+//               bf16 to fp16; for the tree tiles of query group 0 they first
+//               store the tree K/V into cache slots P + i.
+// Each piece of a range writes its normalised partial output and log2-sum-exp;
+// a combine kernel merges the pieces.
 //
 // fp32 path: one warp per query row on CUDA cores (small shapes).
 #include <cuda_bf16.h>
