@@ -2,6 +2,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "abi_internal.h"
@@ -13,6 +14,14 @@ static thread_local char g_last_error[512] = "";
 medusa_status_t fail(medusa_status_t code, const char* msg) {
   snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
   return code;
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MEDUSA_PDL");
+    return v == nullptr || strcmp(v, "0") != 0;
+  }();
+  return on;
 }
 
 medusa_status_t check_launch(const char* what) {

@@ -297,6 +297,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         const __grid_constant__ CUtensorMap tmKs1,
                         const __grid_constant__ CUtensorMap tmVs1,
                         const __grid_constant__ CUtensorMap tmQ, AttnParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   using L = AttnSmem<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -836,6 +838,8 @@ constexpr int kCombineRows = 32;
 template <int DH>
 __global__ void __launch_bounds__(256)
     attn_combine_kernel(AttnParams p, void* __restrict__ out, int out_f32) {
+  grid_dep_wait();
+  grid_dep_launch();
   constexpr int C4 = DH / 4;  // column groups of 4 floats
   __shared__ int cumT[kAttnMaxB + 1];
   __shared__ int sched_ok;
@@ -927,6 +931,8 @@ __global__ void tree_kv_write_f32_kernel(const float* __restrict__ k_new,
                                          const int32_t* __restrict__ prefix_len, int B, int N,
                                          int Hkv, int dh, int cap, int max_prefix,
                                          int32_t* status) {
+  grid_dep_wait();
+  grid_dep_launch();
   const size_t total = (size_t)B * N * Hkv * dh;
   for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
        e += (size_t)gridDim.x * blockDim.x) {
@@ -953,6 +959,8 @@ __global__ void __launch_bounds__(256)
                          const uint32_t* __restrict__ anc_mask, int B, int N, int Hq, int Hkv,
                          int dh, int cap, int max_prefix, int words, float scale, void* out,
                          int out_f32) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= B * N * Hq) return;
@@ -1077,13 +1085,13 @@ static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaSt
                            L::kAlloc) != cudaSuccess)
     return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(tree_attention) failed");
   p.grid = device_sm_count();  // persistent: one CTA per SM
-  tree_attn_tc_kernel<DH><<<p.grid, kAttnThreads, L::kAlloc, stream>>>(mK, mV, mKn, mVn, mKs0,
+  launch(tree_attn_tc_kernel<DH>, p.grid, kAttnThreads, L::kAlloc, stream, mK, mV, mKn, mVn, mKs0,
                                                                         mVs0, mKs1, mVs1, mQ, p);
   medusa_status_t st = check_launch("tree_attention");
   if (st != MEDUSA_OK) return st;
   const int rows = p.B * p.Hkv * p.R;
-  attn_combine_kernel<DH>
-      <<<(rows + kCombineRows - 1) / kCombineRows, 256, 0, stream>>>(p, out, out_f32);
+  launch(attn_combine_kernel<DH>, (rows + kCombineRows - 1) / kCombineRows, 256, 0, stream, p,
+         out, out_f32);
   return check_launch("tree_attention_combine");
 }
 
@@ -1097,14 +1105,14 @@ medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_n
   if (dt == MEDUSA_F32) {
     const size_t total = (size_t)B * N * Hkv * dh;
     const int blocks = (int)((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
-    tree_kv_write_f32_kernel<<<blocks, 256, 0, stream>>>(
+    launch(tree_kv_write_f32_kernel, blocks, 256, 0, stream,
         static_cast<const float*>(k_new), static_cast<const float*>(v_new),
         static_cast<float*>(Kc), static_cast<float*>(Vc), prefix_len, B, N, Hkv, dh, cap,
         max_prefix, status);
     medusa_status_t st = check_launch("tree_kv_write_f32");
     if (st != MEDUSA_OK) return st;
     const int rows = B * N * Hq;
-    tree_attn_f32_kernel<<<(rows + 7) / 8, 256, 0, stream>>>(
+    launch(tree_attn_f32_kernel, (rows + 7) / 8, 256, 0, stream,
         static_cast<const float*>(q), static_cast<const float*>(k_new),
         static_cast<const float*>(v_new), static_cast<const float*>(Kc),
         static_cast<const float*>(Vc), prefix_len, anc_mask, B, N, Hq, Hkv, dh, cap, max_prefix,

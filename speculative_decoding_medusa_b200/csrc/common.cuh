@@ -22,6 +22,43 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t x) {
   return __uint_as_float(static_cast<uint32_t>(x) << 16);
 }
 
+// ----------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library is launched with
+// programmatic stream serialisation, so it can be made resident while its
+// predecessor in the stream drains.  Its first statement is grid_dep_wait():
+// nothing (no global access, no tensor-memory allocation) happens before the
+// predecessor grid has completed and its memory is visible, so the overlap
+// hides only the launch and the rasterisation of the grid.  grid_dep_launch()
+// lets this grid's own dependents be launched early.  Both are no-ops for a
+// kernel launched without the attribute.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch `kern` on `stream` with programmatic stream serialisation (unless
+// disabled by the environment variable MEDUSA_PDL=0, read once).  Returns the
+// launch's error code; the caller still checks it with check_launch().
+bool pdl_enabled();
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                   cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Upper bound of any spin in this library, in SM clock cycles (about one to
 // two seconds on B200).  A wait that runs out reports MEDUSA_ERR_TIMEOUT and
 // returns false instead of hanging the GPU.

@@ -87,6 +87,8 @@ template <int NB, int S, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     heads_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   using L = GemmSmem<NB, S>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -321,6 +323,8 @@ __global__ void __cluster_dims__(kMergeCtas, 1, 1) __launch_bounds__(kMergeWarps
     topk_merge_kernel(const float* __restrict__ vals, const int32_t* __restrict__ ids, long long C,
                       int kmax, int32_t* __restrict__ out_ids, float* __restrict__ out_vals,
                       MergeLayout lay) {
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ float sv[kMergeWarps][32];
   __shared__ int si[kMergeWarps][32];
   cg::cluster_group cluster = cg::this_cluster();
@@ -404,6 +408,8 @@ __device__ __forceinline__ float warp_sum(float x) {
 __global__ void __launch_bounds__(256)
     heads_f32_w1_kernel(const float* __restrict__ h, const float* __restrict__ W1,
                         const float* __restrict__ b1, int B, int d, int K, float* __restrict__ y) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int k = blockIdx.y;
   const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -424,6 +430,8 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     heads_f32_w2_kernel(const float* __restrict__ y, const float* __restrict__ W2, int B, int d,
                         int V, int K, float* __restrict__ z) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int k = blockIdx.y;
   const int v = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -446,7 +454,7 @@ medusa_status_t topk_merge_lists(const float* vals, const int32_t* ids, int rows
                                  const int32_t* id_offsets, int kmax, int32_t* out_ids,
                                  float* out_vals, cudaStream_t stream) {
   const MergeLayout lay{row_stride, list_stride, list_len, id_offsets};
-  topk_merge_kernel<<<rows * kMergeCtas, kMergeWarps * 32, 0, stream>>>(
+  launch(topk_merge_kernel, rows * kMergeCtas, kMergeWarps * 32, 0, stream,
       vals, ids, (long long)n_lists * list_len, kmax, out_ids, out_vals, lay);
   return check_launch("topk_merge");
 }
@@ -473,7 +481,7 @@ medusa_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const Ge
       cudaSuccess)
     return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(heads_gemm) failed");
   const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
-  kern<<<grid, kGemmThreads, L::kAlloc, stream>>>(a, b, p);
+  launch(kern, grid, kGemmThreads, L::kAlloc, stream, a, b, p);
   return check_launch("heads_gemm");
 }
 
@@ -530,17 +538,17 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
   if (dt == MEDUSA_F32) {
     float* y = reinterpret_cast<float*>(wsb);
     float* z = logits != nullptr ? logits : reinterpret_cast<float*>(wsb + w.y_bytes);
-    heads_f32_w1_kernel<<<dim3((d + 7) / 8, K), 256, 0, stream>>>(
+    launch(heads_f32_w1_kernel, dim3((d + 7) / 8, K), 256, 0, stream,
         static_cast<const float*>(h), static_cast<const float*>(W1),
         static_cast<const float*>(b1), B, d, K, y);
     medusa_status_t st = check_launch("heads_f32_w1");
     if (st != MEDUSA_OK) return st;
-    heads_f32_w2_kernel<<<dim3((V + 7) / 8, K), 256, 0, stream>>>(
+    launch(heads_f32_w2_kernel, dim3((V + 7) / 8, K), 256, 0, stream,
         y, static_cast<const float*>(W2), B, d, V, K, z);
     st = check_launch("heads_f32_w2");
     if (st != MEDUSA_OK) return st;
     const MergeLayout lay{(long long)V, (long long)V, V, nullptr};
-    topk_merge_kernel<<<B * K * kMergeCtas, kMergeWarps * 32, 0, stream>>>(z, nullptr, V, kmax,
+    launch(topk_merge_kernel, B * K * kMergeCtas, kMergeWarps * 32, 0, stream, z, nullptr, V, kmax,
                                                                             topk_ids, topk_vals,
                                                                             lay);
     return check_launch("topk_merge");
@@ -586,7 +594,7 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
 
   const long long C = (long long)p2.tiles_per_head * kmax;
   const MergeLayout lay{C, C, (int)C, nullptr};
-  topk_merge_kernel<<<B * K * kMergeCtas, kMergeWarps * 32, 0, stream>>>(
+  launch(topk_merge_kernel, B * K * kMergeCtas, kMergeWarps * 32, 0, stream,
       part_vals, part_ids, C, kmax, topk_ids, topk_vals, lay);
   return check_launch("topk_merge");
 }

@@ -24,6 +24,8 @@ __global__ void __launch_bounds__(kCompactThreads)
                       const int32_t* __restrict__ accepted_nodes,
                       const int32_t* __restrict__ accept_len, int Hkv, int cap, int max_depth,
                       int heads_at_once, int32_t* __restrict__ compact_src, int32_t* status) {
+  grid_dep_wait();
+  grid_dep_launch();
   // [2][max_depth+1][row_bytes], or [2][Hkv][max_depth+1][row_bytes] when
   // every head is staged at once
   extern __shared__ __align__(16) uint8_t stage[];
@@ -31,21 +33,23 @@ __global__ void __launch_bounds__(kCompactThreads)
   __shared__ int s_ok;
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
+  const int W = max_depth + 1;
+  // prefix length, accept length and the path's nodes in one round trip
   const int P = prefix_len[b];
   const int L = accept_len[b];
-  const int W = max_depth + 1;
-  if (tid == 0) {
-    int ok = (L >= 0 && L <= max_depth && P >= 0) ? 1 : 0;
-    for (int j = 0; ok && j <= L; ++j) {
-      const int node = accepted_nodes[(size_t)b * W + j];
-      const long long slot = (long long)P + node;
-      if (node < j || slot >= cap) ok = 0;  // a depth-j node has index >= j
-      s_src[j] = (int)slot;
-    }
-    s_ok = ok;
-    if (!ok) report(status, MEDUSA_ERR_DEVICE_CHECK);
+  const int node = tid < W ? accepted_nodes[(size_t)b * W + tid] : 0;
+  if (tid == 0) s_ok = (L >= 0 && L <= max_depth && P >= 0) ? 1 : 0;
+  __syncthreads();
+  if (tid <= L && tid < W) {
+    const long long slot = (long long)P + node;
+    if (node < tid || slot >= cap) s_ok = 0;  // a depth-j node has index >= j
+    s_src[tid] = (int)slot;
   }
   __syncthreads();
+  if (!s_ok) {
+    if (tid == 0) report(status, MEDUSA_ERR_DEVICE_CHECK);
+    return;
+  }
   if (!s_ok) return;
 
   const int vec_per_row = row_bytes / 16;
@@ -107,7 +111,7 @@ medusa_status_t kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefi
   if (per_head > 48 * 1024)
     return fail(MEDUSA_ERR_UNSUPPORTED, "kv_compact: (max_depth+1) * row too large");
   const bool all_heads = per_head * Hkv <= 48 * 1024;
-  kv_compact_kernel<<<B, kCompactThreads, all_heads ? per_head * Hkv : per_head, stream>>>(
+  launch(kv_compact_kernel, B, kCompactThreads, all_heads ? per_head * Hkv : per_head, stream,
       static_cast<uint8_t*>(Kc), static_cast<uint8_t*>(Vc), row_bytes, prefix_len, accepted_nodes,
       accept_len, Hkv, cap, max_depth, all_heads ? Hkv : 1, compact_src, status);
   return check_launch("kv_compact");

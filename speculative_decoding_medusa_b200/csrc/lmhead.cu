@@ -160,6 +160,8 @@ __device__ __forceinline__ void warp_colsum32x2(float (&a)[32], float (&b)[32], 
 __global__ void __launch_bounds__(kLmThreads, 1)
     lmhead_reduce_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB, LmParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   using L = LmSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -508,7 +510,7 @@ medusa_status_t lmhead_verify(const void* hidden, const void* lm_head, const int
   p.logits = logits;
   p.part = static_cast<RowPart*>(ws);
   p.status = status;
-  lmhead_reduce_kernel<<<q.grid, kLmThreads, LmSmem::kAlloc, stream>>>(mA, mB, p);
+  launch(lmhead_reduce_kernel, q.grid, kLmThreads, LmSmem::kAlloc, stream, mA, mB, p);
   medusa_status_t st = check_launch("lmhead_reduce");
   if (st != MEDUSA_OK) return st;
   return verify_path_from_parts(p.part, q.n_slots, static_cast<const __nv_bfloat16*>(hidden),

@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(128)
                      const int32_t* __restrict__ accepted_nodes, int width,
                      const int32_t* __restrict__ bonus, uint4* __restrict__ h_next,
                      int32_t* __restrict__ root_next, int32_t* status) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int b = blockIdx.x;
   const int L = accept_len[b];
   const int kept = (L >= 0 && L < width) ? accepted_nodes[(size_t)b * width + L] : -1;
@@ -40,7 +42,7 @@ medusa_status_t next_step(const void* node_hidden, int elem_bytes, const int32_t
                           int d, int max_depth, void* h_next, int32_t* root_next,
                           int32_t* status, cudaStream_t stream) {
   const int row_vecs = d * elem_bytes / 16;
-  next_step_kernel<<<B, 128, 0, stream>>>(static_cast<const uint4*>(node_hidden), N, row_vecs,
+  launch(next_step_kernel, B, 128, 0, stream, static_cast<const uint4*>(node_hidden), N, row_vecs,
                                           accept_len, accepted_nodes, max_depth + 1, bonus,
                                           static_cast<uint4*>(h_next), root_next, status);
   return check_launch("next_step");

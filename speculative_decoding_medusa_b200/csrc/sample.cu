@@ -61,6 +61,8 @@ __global__ void __launch_bounds__(kSampleThreads)
                         float inv_T, uint32_t seed_lo, uint32_t seed_hi, uint32_t off_lo,
                         uint32_t off_hi, int32_t* __restrict__ bonus,
                         int32_t* __restrict__ accepted_tokens, int32_t* status) {
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ float s_red[32];
   __shared__ int s_ired[32];
   __shared__ float s_max, s_total;
@@ -156,11 +158,11 @@ medusa_status_t sample_bonus(const void* logits, medusa_dtype_t dt, const int32_
   const uint32_t s0 = (uint32_t)seed, s1 = (uint32_t)(seed >> 32);
   const uint32_t o0 = (uint32_t)offset, o1 = (uint32_t)(offset >> 32);
   if (dt == MEDUSA_BF16)
-    sample_bonus_kernel<__nv_bfloat16><<<B, kSampleThreads, 0, stream>>>(
+    launch(sample_bonus_kernel<__nv_bfloat16>, B, kSampleThreads, 0, stream,
         static_cast<const __nv_bfloat16*>(logits), accept_len, accepted_nodes, N, V,
         max_depth + 1, inv_T, s0, s1, o0, o1, bonus, accepted_tokens, status);
   else
-    sample_bonus_kernel<float><<<B, kSampleThreads, 0, stream>>>(
+    launch(sample_bonus_kernel<float>, B, kSampleThreads, 0, stream,
         static_cast<const float*>(logits), accept_len, accepted_nodes, N, V, max_depth + 1, inv_T,
         s0, s1, o0, o1, bonus, accepted_tokens, status);
   return check_launch("sample_bonus");

@@ -25,19 +25,29 @@ __global__ void __launch_bounds__(MEDUSA_MAX_NODES)
                       int32_t* __restrict__ cand_ids, int32_t* __restrict__ pos_ids,
                       uint32_t* __restrict__ anc_mask, int32_t* __restrict__ retrieve,
                       int32_t* status) {
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ int s_parent[MEDUSA_MAX_NODES];
   __shared__ int s_depth[MEDUSA_MAX_NODES];
   __shared__ int s_has_child[MEDUSA_MAX_NODES];
+  __shared__ int s_rank[MEDUSA_MAX_NODES];
   __shared__ int s_warp_leaves[MEDUSA_MAX_NODES / 32];
   __shared__ int s_bad;
+  extern __shared__ int s_topk[];  // this sequence's K x kmax candidate ids
   const int i = threadIdx.x;
   const int b = blockIdx.x;
+  // every input is read in one round trip: the tree, this sequence's
+  // candidate table, its prefix length and root token
   if (i == 0) s_bad = 0;
   if (i < N) {
     s_parent[i] = parent[i];
     s_depth[i] = depth[i];
+    s_rank[i] = rank[i];
     s_has_child[i] = 0;
   }
+  for (int e = i; e < K * kmax; e += blockDim.x) s_topk[e] = topk_ids[(size_t)b * K * kmax + e];
+  const int P = prefix_len[b];
+  const int root = root_tok[b];
   __syncthreads();
 
   // structural checks: BFS order, depth chain, rank range
@@ -48,7 +58,7 @@ __global__ void __launch_bounds__(MEDUSA_MAX_NODES)
     if (i == 0) {
       ok = (pa == -1) && (dp == 0);
     } else {
-      const int rk = rank[i];
+      const int rk = s_rank[i];
       ok = pa >= 0 && pa < i && dp == s_depth[pa] + 1 && dp <= max_depth && dp <= K && rk >= 0 &&
            rk < kmax;
     }
@@ -66,13 +76,7 @@ __global__ void __launch_bounds__(MEDUSA_MAX_NODES)
   }
 
   if (i < N) {
-    const int P = prefix_len[b];
-    int tok;
-    if (i == 0) {
-      tok = root_tok[b];
-    } else {
-      tok = topk_ids[((size_t)b * K + (s_depth[i] - 1)) * kmax + rank[i]];
-    }
+    const int tok = i == 0 ? root : s_topk[(s_depth[i] - 1) * kmax + s_rank[i]];
     cand_ids[(size_t)b * N + i] = tok;
     pos_ids[(size_t)b * N + i] = P + s_depth[i];
   }
@@ -120,7 +124,7 @@ medusa_status_t tree_build(const medusa_tree_t& t, const int32_t* root_tok, cons
                            int K, int kmax, const int32_t* prefix_len, int B, int32_t* cand_ids,
                            int32_t* pos_ids, uint32_t* anc_mask, int32_t* retrieve,
                            int32_t* status, cudaStream_t stream) {
-  tree_build_kernel<<<B, MEDUSA_MAX_NODES, 0, stream>>>(
+  launch(tree_build_kernel, B, MEDUSA_MAX_NODES, (size_t)K * kmax * sizeof(int), stream,
       t.parent, t.depth, t.rank, t.n_nodes, t.max_depth, t.n_leaves, root_tok, topk_ids, K, kmax,
       prefix_len, cand_ids, pos_ids, anc_mask, retrieve, status);
   return check_launch("tree_build");

@@ -224,6 +224,8 @@ __global__ void __launch_bounds__(kRowWarps * 32,
                                   (std::is_same<T, __nv_bfloat16>::value && !TYPICAL) ? 3 : 1)
     verify_rows_kernel(const T* __restrict__ logits, int V, int n_chunks, long long n_items,
                        float inv_T, RowPart* __restrict__ part, int32_t* status) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   for (long long item = (long long)blockIdx.x * kRowWarps + (threadIdx.x >> 5); item < n_items;
        item += (long long)gridDim.x * kRowWarps)
@@ -248,6 +250,8 @@ __global__ void __launch_bounds__(kPathThreads)
                        float delta, int32_t* __restrict__ accept_len,
                        int32_t* __restrict__ accepted_nodes, int32_t* __restrict__ accepted_tokens,
                        int32_t* __restrict__ bonus, int32_t* status) {
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ int s_g[MEDUSA_MAX_NODES];
   __shared__ float s_lse[MEDUSA_MAX_NODES];
   __shared__ float s_logthr[MEDUSA_MAX_NODES];
@@ -255,6 +259,7 @@ __global__ void __launch_bounds__(kPathThreads)
   __shared__ int s_depth[MEDUSA_MAX_NODES];
   __shared__ int s_pass[MEDUSA_MAX_NODES];
   __shared__ float s_zc[MEDUSA_MAX_NODES];  // logit of node i's candidate at its parent
+  __shared__ int s_cand[MEDUSA_MAX_NODES];
   __shared__ int s_best;
   __shared__ int s_bad;
   const int b = blockIdx.x;
@@ -263,17 +268,11 @@ __global__ void __launch_bounds__(kPathThreads)
     s_best = 0xFFFF;  // the root: depth 0, node 0
     s_bad = 0;
   }
+  // the tree, the candidates and the chunk records are read in one round trip
   if (i < N) {
     s_parent[i] = parent[i];
     s_depth[i] = depth[i];
-  }
-  __syncthreads();
-  if (i < N) {
-    const int pa = s_parent[i];
-    const int dp = s_depth[i];
-    const bool ok = (i == 0) ? (pa == -1 && dp == 0)
-                             : (pa >= 0 && pa < i && dp == s_depth[pa] + 1 && dp <= max_depth);
-    if (!ok) atomicOr(&s_bad, 1);
+    s_cand[i] = cand_ids[(size_t)b * N + i];
   }
   {
     // merge the chunks of row (b, node): this thread's share, then the group
@@ -336,6 +335,14 @@ __global__ void __launch_bounds__(kPathThreads)
     }
   }
   __syncthreads();
+  if (i < N) {
+    const int pa = s_parent[i];
+    const int dp = s_depth[i];
+    const bool ok = (i == 0) ? (pa == -1 && dp == 0)
+                             : (pa >= 0 && pa < i && dp == s_depth[pa] + 1 && dp <= max_depth);
+    if (!ok) atomicOr(&s_bad, 1);
+  }
+  __syncthreads();
   if (s_bad) {
     if (i == 0) {
       report(status, MEDUSA_ERR_DEVICE_CHECK);
@@ -348,7 +355,7 @@ __global__ void __launch_bounds__(kPathThreads)
     // per node, 16-byte loads (d is a multiple of 64)
     const int warp = i >> 5, lane = i & 31;
     for (int c = 1 + warp; c < N; c += kPathThreads / 32) {
-      const int tok = cand_ids[(size_t)b * N + c];
+      const int tok = s_cand[c];
       float acc = 0.f;
       if (tok >= 0 && tok < V) {
         const uint4* wr = reinterpret_cast<const uint4*>(lm_head + (size_t)tok * d);
@@ -376,7 +383,7 @@ __global__ void __launch_bounds__(kPathThreads)
   if (i < N) {
     int pass = 1;
     if (i > 0) {
-      const int tok = cand_ids[(size_t)b * N + i];
+      const int tok = s_cand[i];
       const int pa = s_parent[i];
       if (tok < 0 || tok >= V) {
         report(status, MEDUSA_ERR_DEVICE_CHECK);
@@ -410,7 +417,7 @@ __global__ void __launch_bounds__(kPathThreads)
     }
     for (int j = best; j >= 0; j = s_parent[j]) {
       accepted_nodes[o + s_depth[j]] = j;
-      if (j > 0) accepted_tokens[o + s_depth[j] - 1] = cand_ids[(size_t)b * N + j];
+      if (j > 0) accepted_tokens[o + s_depth[j] - 1] = s_cand[j];
     }
     accepted_tokens[o + L] = s_g[best];
     accept_len[b] = L;
@@ -451,7 +458,7 @@ medusa_status_t verify_path_from_parts(const RowPart* part, int n_chunks,
   const int N = tree.n_nodes;
   const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
   const float inv_T = typical ? 1.0f / temperature : 1.0f;
-  verify_path_kernel<__nv_bfloat16><<<B, kPathThreads, 0, stream>>>(
+  launch(verify_path_kernel<__nv_bfloat16>, B, kPathThreads, 0, stream,
       nullptr, hidden, lm_head, d, part, n_chunks, n_chunks, 1, path_threads_per_node(N, n_chunks),
       nullptr, cand_ids,
       tree.parent, tree.depth, N, tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta,
@@ -470,6 +477,8 @@ __global__ void __launch_bounds__(256)
                          const int32_t* __restrict__ parent, int B, int N, int V_shard,
                          int v_offset, int typical, float inv_T, RowPart* __restrict__ records,
                          float* __restrict__ cand_logit, int32_t* status) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= B * N) return;
   const RowPart* rp = part + (size_t)r * n_chunks;
@@ -534,28 +543,28 @@ medusa_status_t verify_records(const void* logits, medusa_dtype_t dt, const int3
     const __nv_bfloat16* lg = static_cast<const __nv_bfloat16*>(logits);
     if (typical) {
       auto k = verify_rows_kernel<__nv_bfloat16, true>;
-      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V_shard, n_chunks, n_items,
+      launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V_shard, n_chunks, n_items,
                                                               inv_T, part, status);
     } else {
       auto k = verify_rows_kernel<__nv_bfloat16, false>;
-      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V_shard, n_chunks, n_items,
+      launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V_shard, n_chunks, n_items,
                                                               inv_T, part, status);
     }
-    shard_records_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+    launch(shard_records_kernel<__nv_bfloat16>, grid, 256, 0, stream,
         lg, part, n_chunks, cand_ids, tree.parent, B, N, V_shard, v_offset, typical ? 1 : 0,
         inv_T, records, cand_logit, status);
   } else {
     const float* lg = static_cast<const float*>(logits);
     if (typical) {
       auto k = verify_rows_kernel<float, true>;
-      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V_shard, n_chunks, n_items,
+      launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V_shard, n_chunks, n_items,
                                                               inv_T, part, status);
     } else {
       auto k = verify_rows_kernel<float, false>;
-      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V_shard, n_chunks, n_items,
+      launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V_shard, n_chunks, n_items,
                                                               inv_T, part, status);
     }
-    shard_records_kernel<float><<<grid, 256, 0, stream>>>(
+    launch(shard_records_kernel<float>, grid, 256, 0, stream,
         lg, part, n_chunks, cand_ids, tree.parent, B, N, V_shard, v_offset, typical ? 1 : 0,
         inv_T, records, cand_logit, status);
   }
@@ -572,7 +581,7 @@ medusa_status_t verify_from_records(const RowPart* records, int G, const float* 
   const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
   const float inv_T = typical ? 1.0f / temperature : 1.0f;
   // records are shard-major: [G][B * N]
-  verify_path_kernel<float><<<B, kPathThreads, 0, stream>>>(
+  launch(verify_path_kernel<float>, B, kPathThreads, 0, stream,
       nullptr, nullptr, nullptr, 0, records, G, 1, (long long)B * N,
       path_threads_per_node(N, G), cand_logit, cand_ids, tree.parent, tree.depth, N,
       tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes,
@@ -601,16 +610,16 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
     const __nv_bfloat16* lg = static_cast<const __nv_bfloat16*>(logits);
     if (typical) {
       auto k = verify_rows_kernel<__nv_bfloat16, true>;
-      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T,
+      launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V, n_chunks, n_items, inv_T,
                                                               part, status);
     } else {
       auto k = verify_rows_kernel<__nv_bfloat16, false>;
-      k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T,
+      launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V, n_chunks, n_items, inv_T,
                                                               part, status);
     }
     medusa_status_t st = check_launch("verify_rows");
     if (st != MEDUSA_OK) return st;
-    verify_path_kernel<__nv_bfloat16><<<B, kPathThreads, 0, stream>>>(
+    launch(verify_path_kernel<__nv_bfloat16>, B, kPathThreads, 0, stream,
         lg, nullptr, nullptr, 0, part, n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
         typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
         status);
@@ -619,16 +628,16 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
   const float* lg = static_cast<const float*>(logits);
   if (typical) {
     auto k = verify_rows_kernel<float, true>;
-    k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T, part,
+    launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V, n_chunks, n_items, inv_T, part,
                                                             status);
   } else {
     auto k = verify_rows_kernel<float, false>;
-    k<<<rows_grid(k, n_items), kRowWarps * 32, 0, stream>>>(lg, V, n_chunks, n_items, inv_T, part,
+    launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V, n_chunks, n_items, inv_T, part,
                                                             status);
   }
   medusa_status_t st = check_launch("verify_rows");
   if (st != MEDUSA_OK) return st;
-  verify_path_kernel<float><<<B, kPathThreads, 0, stream>>>(
+  launch(verify_path_kernel<float>, B, kPathThreads, 0, stream,
       lg, nullptr, nullptr, 0, part, n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
       typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
       status);
