@@ -94,7 +94,14 @@ def test_tiny_fp32():
     (2, 6, 2, 128, (50, 300), "sparse16", 5),      # G 3: Q rows gathered by threads
     (1, 16, 1, 64, (200, 200), "sparse64", 6),     # G 16: four query groups of 256 rows
 ])
-def test_bf16_small(B, Hq, Hkv, dh, ctx, tree, seed):
+@pytest.mark.parametrize("pair", [True, False], ids=["pair", "single"])
+def test_bf16_small(B, Hq, Hkv, dh, ctx, tree, seed, pair, monkeypatch):
+    # MEDUSA_ATTN_PAIR=1 opts into the CTA-pair (cta_group::2) kernel, which
+    # serves dh 128 when G divides 128; other shapes fall back to the
+    # single-CTA kernel, which the "single" cases cover
+    if pair and (dh != 128 or 128 % (Hq // Hkv) != 0):
+        pytest.skip("the pair kernel serves dh 128 with G dividing 128 only")
+    monkeypatch.setenv("MEDUSA_ATTN_PAIR", "1" if pair else "0")
     if tree == "sparse64":
         spec = W.sparse_tree(64, 4, 10, seed, max_depth=4)
     elif tree == "sparse16":
