@@ -118,11 +118,28 @@ def test_bf16_small(B, Hq, Hkv, dh, ctx, tree, seed, pair, monkeypatch):
 
 
 @pytest.mark.slow
-def test_llama3_8b_full_size_sampled_rows():
-    w = W.WORKLOADS["llama3_8b"]
+@pytest.mark.parametrize("name", ["llama3_8b", "llama3_70b", "long"])
+def test_full_size_sampled_rows(name):
+    # llama3_70b: 256-node dense tree (two tree tiles, 8 mask words), G = 8,
+    # eight query groups of 256 rows; long: 32 sequences of 32768 cached keys
+    w = W.WORKLOADS[name]
     spec = W.tree_for(w)
     inp = W.attention_inputs(w, seed=0)
     rng = np.random.default_rng(0)
     rows = [(int(rng.integers(w.B)), int(rng.integers(w.N))) for _ in range(24)]
+    rows += [(0, 0), (w.B - 1, w.N - 1)]
+    _compare(inp, spec, w.ctx_hi, rows=rows)
+
+
+@pytest.mark.slow
+def test_pair_kernel_full_size_sampled_rows(monkeypatch):
+    # the opt-in CTA-pair kernel on the Llama-3-70B shape: 256 nodes, G = 8,
+    # eight query groups, two tree tiles
+    monkeypatch.setenv("MEDUSA_ATTN_PAIR", "1")
+    w = W.WORKLOADS["llama3_70b"]
+    spec = W.tree_for(w)
+    inp = W.attention_inputs(w, seed=1)
+    rng = np.random.default_rng(1)
+    rows = [(int(rng.integers(w.B)), int(rng.integers(w.N))) for _ in range(16)]
     rows += [(0, 0), (w.B - 1, w.N - 1)]
     _compare(inp, spec, w.ctx_hi, rows=rows)

@@ -81,8 +81,10 @@ def test_bf16_topk_without_logits_output():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["vicuna7b", "llama3_8b"])
+@pytest.mark.parametrize("name", ["vicuna7b", "llama3_8b", "llama3_70b", "long"])
 def test_full_size(name):
+    # llama3_70b: d = 8192 (128 k-blocks per tile); long: B = 32, so the
+    # second GEMM runs 64 columns (hi and lo of every sequence) per MMA
     w = W.WORKLOADS[name]
     inp = W.heads_inputs(w, seed=0)
     ids, vals, z = _run(inp, w.kmax)
