@@ -1724,7 +1724,48 @@ __global__ void __launch_bounds__(256)
     m = mn;
   };
   const size_t hb = ((size_t)b * Hkv + kvh) * cap;
-  for (int t = 0; t < P; ++t) visit(Kc + (hb + t) * dh, Vc + (hb + t) * dh);
+  // the cached prefix eight keys at a time: their loads are in flight
+  // together, then one online-softmax update takes all eight
+  constexpr int KB = 8;
+  int t = 0;
+  for (; t + KB <= P; t += KB) {
+    float sc[KB];
+#pragma unroll
+    for (int u = 0; u < KB; ++u) {
+      const float* kp = Kc + (hb + t + u) * dh;
+      float sd = 0.f;
+#pragma unroll
+      for (int e = 0; e < MAXPER; ++e)
+        if (e < per) sd += qv[e] * kp[lane * per + e];
+      sc[u] = sd;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int u = 0; u < KB; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
+    }
+    float mn = m;
+#pragma unroll
+    for (int u = 0; u < KB; ++u) {
+      sc[u] *= scale;
+      mn = fmaxf(mn, sc[u]);
+    }
+    const float corr = expf(m - mn);
+    l *= corr;
+#pragma unroll
+    for (int e = 0; e < MAXPER; ++e) acc[e] *= corr;
+#pragma unroll
+    for (int u = 0; u < KB; ++u) {
+      const float pw = expf(sc[u] - mn);
+      const float* vp = Vc + (hb + t + u) * dh;
+      l += pw;
+#pragma unroll
+      for (int e = 0; e < MAXPER; ++e)
+        if (e < per) acc[e] += pw * vp[lane * per + e];
+    }
+    m = mn;
+  }
+  for (; t < P; ++t) visit(Kc + (hb + t) * dh, Vc + (hb + t) * dh);
   for (int j = 0; j < N; ++j) {
     if ((anc_mask[(size_t)i * words + (j >> 5)] >> (j & 31)) & 1u) {
       const size_t off = (((size_t)b * N + j) * Hkv + kvh) * dh;

@@ -63,6 +63,32 @@ struct Elt<float> {
   }
 };
 
+// paired fp32 arithmetic (two lanes in one 64-bit register, sm_100) and the
+// SFU's 2^x (relative error about 2^-22; -inf -> 0)
+__device__ __forceinline__ uint64_t f32x2_pack_v(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack_v(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f32x2_fma_v(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_add_v(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float ex2_approx_v(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -106,9 +132,9 @@ __device__ __forceinline__ void verify_item(const T* __restrict__ logits, int V,
       raw[r] = E::load_scalar(base + e0, e0 < V ? min(EV, V - e0) : 0);
     }
   }
-  if constexpr (std::is_same<T, __nv_bfloat16>::value && !TYPICAL) {
-    // greedy on bf16: packed maximum (NaN propagates, so one check at the
-    // end catches a NaN anywhere), then the first index holding that value
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    // bf16: packed maximum (NaN propagates, so one check at the end catches a
+    // NaN anywhere), then the first index holding that value
     __nv_bfloat162 m2 = __halves2bfloat162(__ushort_as_bfloat16(0xFF80u), __ushort_as_bfloat16(0xFF80u));
 #pragma unroll
     for (int r = 0; r < NL; ++r) {
@@ -148,12 +174,52 @@ __device__ __forceinline__ void verify_item(const T* __restrict__ logits, int V,
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) idx = min(idx, __shfl_xor_sync(0xffffffffu, idx, o));
+    float ss = 0.f, tt = 0.f;
+    if constexpr (TYPICAL) {
+      // typical: s = sum exp(z/T - M/T) and t = sum exp(z/T - M/T) * z/T, as
+      // 2^(z * log2(e)/T - M * log2(e)/T) on paired fp32 instructions and the
+      // SFU; padding (-inf) contributes 0 to both
+      const float cl = inv_T * 1.4426950408889634f;
+      const uint64_t c2 = f32x2_pack_v(cl, cl);
+      const uint64_t nb2 = f32x2_pack_v(-M * cl, -M * cl);
+      const uint64_t it2 = f32x2_pack_v(inv_T, inv_T);
+      uint64_t s2[2] = {0ull, 0ull}, t2[2] = {0ull, 0ull};
+#pragma unroll
+      for (int r = 0; r < NL; ++r) {
+        const uint32_t* w = &raw[r].x;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float z0 = __uint_as_float(w[q] << 16), z1 = __uint_as_float(w[q] & 0xffff0000u);
+          const uint64_t z2 = f32x2_pack_v(z0, z1);
+          float x0, x1;
+          f32x2_unpack_v(f32x2_fma_v(z2, c2, nb2), x0, x1);
+          const float e0 = ex2_approx_v(x0), e1 = ex2_approx_v(x1);
+          float zt0, zt1;
+          f32x2_unpack_v(f32x2_fma_v(z2, it2, 0ull), zt0, zt1);
+          zt0 = z0 == -INFINITY ? 0.f : zt0;
+          zt1 = z1 == -INFINITY ? 0.f : zt1;
+          const uint64_t e2 = f32x2_pack_v(e0, e1);
+          s2[q & 1] = f32x2_add_v(s2[q & 1], e2);
+          t2[q & 1] = f32x2_fma_v(e2, f32x2_pack_v(zt0, zt1), t2[q & 1]);
+        }
+      }
+      float a0, a1, b0, b1;
+      f32x2_unpack_v(f32x2_add_v(s2[0], s2[1]), a0, a1);
+      f32x2_unpack_v(f32x2_add_v(t2[0], t2[1]), b0, b1);
+      ss = a0 + a1;
+      tt = b0 + b1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        tt += __shfl_xor_sync(0xffffffffu, tt, o);
+      }
+    }
     if (lane == 0) {
       RowPart rp;
       rp.maxz = M;
       rp.idx = idx;
-      rp.s = 0.f;
-      rp.t = 0.f;
+      rp.s = ss;
+      rp.t = tt;
       part[row * n_chunks + c] = rp;
     }
     return;
@@ -221,7 +287,7 @@ __device__ __forceinline__ void verify_item(const T* __restrict__ logits, int V,
 // total warps, ... so that no partial last wave of CTAs is left.
 template <typename T, bool TYPICAL>
 __global__ void __launch_bounds__(kRowWarps * 32,
-                                  (std::is_same<T, __nv_bfloat16>::value && !TYPICAL) ? 3 : 1)
+                                  std::is_same<T, __nv_bfloat16>::value ? (TYPICAL ? 2 : 3) : 1)
     verify_rows_kernel(const T* __restrict__ logits, int V, int n_chunks, long long n_items,
                        float inv_T, RowPart* __restrict__ part, int32_t* status) {
   grid_dep_wait();

@@ -73,10 +73,15 @@ def _compact_case(seed, B=3, Hkv=2, dh=128, dtype=torch.bfloat16, max_depth=4, N
     return Kc, Vc, prefix, nodes, L, max_depth
 
 
-@pytest.mark.parametrize("seed,dtype,dh", [(0, torch.bfloat16, 128), (1, torch.bfloat16, 64),
-                                           (2, torch.float32, 64), (3, torch.bfloat16, 128)])
-def test_kv_compact_bit_exact(seed, dtype, dh):
-    Kc, Vc, prefix, nodes, L, max_depth = _compact_case(seed, dtype=dtype, dh=dh)
+@pytest.mark.parametrize("seed,dtype,dh,Hkv,max_depth", [
+    (0, torch.bfloat16, 128, 2, 4), (1, torch.bfloat16, 64, 2, 4), (2, torch.float32, 64, 2, 4),
+    (3, torch.bfloat16, 128, 2, 4),
+    (4, torch.bfloat16, 128, 32, 5),   # 32 kv heads staged in one round
+    (5, torch.float32, 256, 16, 5),    # 12 KB per head: two rounds of 8 heads
+])
+def test_kv_compact_bit_exact(seed, dtype, dh, Hkv, max_depth):
+    Kc, Vc, prefix, nodes, L, max_depth = _compact_case(seed, dtype=dtype, dh=dh, Hkv=Hkv,
+                                                        max_depth=max_depth)
     if seed == 3:  # overlapping chains: every destination is another step's source
         nodes[:] = -1
         for b in range(nodes.shape[0]):
