@@ -491,7 +491,7 @@ medusa_status_t launch_gemm_nb(int nb, const CUtensorMap& a, const CUtensorMap& 
   switch (nb) {
     case 16: return launch_gemm<16, 8, MODE>(a, b, p, s);
     case 32: return launch_gemm<32, 8, MODE>(a, b, p, s);
-    case 64: return launch_gemm<64, 6, MODE>(a, b, p, s);
+    case 64: return launch_gemm<64, 8, MODE>(a, b, p, s);  // 128 KB of weights in flight
     case 128: return launch_gemm<128, 4, MODE>(a, b, p, s);
     case 256: return launch_gemm<256, 3, MODE>(a, b, p, s);
   }
