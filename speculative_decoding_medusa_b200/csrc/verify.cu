@@ -287,7 +287,7 @@ __device__ __forceinline__ void verify_item(const T* __restrict__ logits, int V,
 // total warps, ... so that no partial last wave of CTAs is left.
 template <typename T, bool TYPICAL>
 __global__ void __launch_bounds__(kRowWarps * 32,
-                                  std::is_same<T, __nv_bfloat16>::value ? (TYPICAL ? 2 : 3) : 1)
+                                  std::is_same<T, __nv_bfloat16>::value ? 3 : 1)
     verify_rows_kernel(const T* __restrict__ logits, int V, int n_chunks, long long n_items,
                        float inv_T, RowPart* __restrict__ part, int32_t* status) {
   grid_dep_wait();
