@@ -58,6 +58,44 @@ struct GemmParams {
   float* part_vals;           // [B*K, tiles_per_head, kmax] (W2)
   int32_t* part_ids;
   int32_t* status;
+  // stream-K (W1 mode): every CTA takes kpc consecutive k-blocks of the
+  // (tile, k-block) sequence; 0 = whole tiles round-robin
+  int kpc;
+  float* sk_part;  // [grid][kTileM][NB] fp32 partial of a CTA's leading tile tail
+  int* sk_flag;    // [grid] 1 once that partial is written (zeroed before the launch)
+  int sk_grid;     // CTAs of a stream-K launch
+};
+
+// One CTA's work as (tile, first k-block, end k-block) segments, in order.
+// Round-robin: whole tiles blockIdx.x, + gridDim.x, ...  Stream-K: the
+// k-blocks [blockIdx.x * kpc, + kpc) of the tile-major sequence, cut at tile
+// ends; only the first segment can start inside a tile.
+struct SegIter {
+  int nkb, n_tiles, kpc, tile, g, g_hi;
+  __device__ __forceinline__ void init(const GemmParams& p, int nkb_) {
+    nkb = nkb_;
+    n_tiles = p.n_tiles;
+    kpc = p.kpc;
+    tile = blockIdx.x;
+    g = blockIdx.x * kpc;
+    g_hi = min(g + kpc, n_tiles * nkb);
+  }
+  __device__ __forceinline__ bool next(int& t, int& kb0, int& kb1) {
+    if (kpc > 0) {
+      if (g >= g_hi) return false;
+      t = g / nkb;
+      kb0 = g - t * nkb;
+      kb1 = min(nkb, kb0 + (g_hi - g));
+      g += kb1 - kb0;
+      return true;
+    }
+    if (tile >= n_tiles) return false;
+    t = tile;
+    kb0 = 0;
+    kb1 = nkb;
+    tile += gridDim.x;
+    return true;
+  }
 };
 
 template <int NB, int S>
@@ -81,6 +119,35 @@ struct GemmSmem {
 template <int NB>
 __host__ __device__ constexpr uint32_t tmem_cols() {
   return (2 * NB) < 32 ? 32u : static_cast<uint32_t>(2 * NB);
+}
+
+// release / acquire of a flag another CTA waits on
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Wait until *flag == 1; gives up (false) when *abort is raised or the spin
+// budget runs out, reporting MEDUSA_ERR_TIMEOUT in that case.
+__device__ __forceinline__ bool wait_flag_bounded(const int* flag, volatile int* abort,
+                                                  int32_t* status) {
+  if (ld_acquire_gpu(flag) == 1) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) == 1) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort) return false;
+      if (clock64() - t0 > kSpinBudgetCycles) {
+        *abort = 1;
+        report(status, MEDUSA_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
 }
 
 template <int NB, int S, int MODE>
@@ -138,10 +205,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint64_t pol_b = l2_policy_evict_last();
       int g = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x) {
+      SegIter seg;
+      seg.init(p, nkb);
+      int tile, kb0, kb1;
+      while (ok && seg.next(tile, kb0, kb1)) {
         const int head = tile / p.tiles_per_head;
         const int m0 = (tile - head * p.tiles_per_head) * kTileM;
-        for (int kb = 0; kb < nkb; ++kb, ++g) {
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
           const int s = g % S;
           const uint32_t ph = (g / S) & 1;
           if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.status)) {
@@ -168,13 +238,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       constexpr uint32_t idesc = umma_idesc_bf16(kTileM, NB);
       int g = 0, it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x, ++it) {
+      SegIter seg;
+      seg.init(p, nkb);
+      int tile, kb0, kb1;
+      for (; ok && seg.next(tile, kb0, kb1); ++it) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         if (!mbar_wait_bounded(&tempty[acc], aph ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * NB;
-        for (int kb = 0; kb < nkb; ++kb, ++g) {
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
           const int s = g % S;
           const uint32_t ph = (g / S) & 1;
           if (!mbar_wait_bounded(&full[s], ph, abort_flag, p.status)) {
@@ -187,7 +260,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kTileK / 16; ++kk) {
             umma_bf16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32),
-                      idesc, (kb | kk) != 0 ? 1u : 0u);
+                      idesc, (kb > kb0 || kk != 0) ? 1u : 0u);
           }
           umma_commit(&empty[s]);
         }
@@ -213,7 +286,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       return epi_ok;
     };
     int it = 0;
-    for (int tile = blockIdx.x; epi_ok && tile < p.n_tiles; tile += gridDim.x, ++it) {
+    SegIter seg;
+    seg.init(p, nkb);
+    int tile, kb0, kb1;
+    for (; epi_ok && seg.next(tile, kb0, kb1); ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       if (!mbar_wait_bounded(&tfull[acc], aph, abort_flag, p.status)) break;
@@ -223,10 +299,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int r = tile_in_head * kTileM + row;  // row within the head
       const bool valid = r < p.rows_per_head;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * NB;
+      if (MODE == kModeW1 && kb0 > 0) {
+        // stream-K: the tail of a tile that an earlier CTA finishes.  This
+        // CTA's fp32 partial goes to its slot, then its flag is raised.
+        float* dst = p.sk_part + ((size_t)blockIdx.x * kTileM + row) * NB;
+#pragma unroll 1
+        for (int c0 = 0; c0 < NB; c0 += 16) {
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+#pragma unroll
+          for (int t = 0; t < 16; t += 4)
+            *reinterpret_cast<float4*>(dst + c0 + t) = make_float4(v[t], v[t + 1], v[t + 2], v[t + 3]);
+        }
+        __threadfence();
+        if (!epi_sync()) break;
+        if (threadIdx.x == 64) st_release_gpu(&p.sk_flag[blockIdx.x], 1);
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+        continue;
+      }
+      // stream-K: this CTA holds the tile's first k-block; the CTAs after it
+      // that took the rest have written their partials
+      int c_last = blockIdx.x;
+      if (MODE == kModeW1 && kb1 < nkb) {
+        c_last = ((tile + 1) * nkb - 1) / p.kpc;
+        bool ready = true;
+        for (int c = blockIdx.x + 1; ready && c <= c_last; ++c)
+          ready = wait_flag_bounded(&p.sk_flag[c], abort_flag, p.status);
+        if (!ready) break;
+      }
 #pragma unroll 1
       for (int c0 = 0; epi_ok && c0 < NB; c0 += 16) {
         float v[16];
         tmem_ld16(taddr + c0, v);
+        for (int c = blockIdx.x + 1; c <= c_last; ++c) {
+          const float* src = p.sk_part + ((size_t)c * kTileM + row) * NB + c0;
+#pragma unroll
+          for (int t = 0; t < 16; t += 4) {
+            const float4 q = *reinterpret_cast<const float4*>(src + t);
+            v[t] += q.x;
+            v[t + 1] += q.y;
+            v[t + 2] += q.z;
+            v[t + 3] += q.w;
+          }
+        }
         if (MODE == kModeW1) {
           if (valid) {
             const float bias = __bfloat162float(p.b1[(size_t)head * p.d + r]);
@@ -480,7 +596,7 @@ medusa_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const Ge
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
       cudaSuccess)
     return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(heads_gemm) failed");
-  const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
+  const int grid = p.kpc > 0 ? p.sk_grid : (p.n_tiles < num_sms() ? p.n_tiles : num_sms());
   launch(kern, grid, kGemmThreads, L::kAlloc, stream, a, b, p);
   return check_launch("heads_gemm");
 }
@@ -505,7 +621,7 @@ int round_nb(int cols) {
 }
 
 struct HeadsWs {
-  size_t y_bytes, part_bytes, total;
+  size_t y_bytes, part_bytes, sk_part_bytes, sk_flag_bytes, total;
 };
 
 HeadsWs heads_ws_layout(int B, int d, int V, int K, int kmax, medusa_dtype_t dt) {
@@ -514,7 +630,11 @@ HeadsWs heads_ws_layout(int B, int d, int V, int K, int kmax, medusa_dtype_t dt)
     const size_t tph = (size_t)(V + kTileM - 1) / kTileM;
     w.y_bytes = align256((size_t)K * 2 * B * d * 2);
     w.part_bytes = align256((size_t)B * K * tph * kmax * 4);
-    w.total = w.y_bytes + 2 * w.part_bytes;
+    // stream-K partials of the first GEMM: one [128][NB] fp32 slot and one
+    // flag per CTA
+    w.sk_part_bytes = align256((size_t)num_sms() * kTileM * round_nb(B) * 4);
+    w.sk_flag_bytes = align256((size_t)num_sms() * 4);
+    w.total = w.y_bytes + 2 * w.part_bytes + w.sk_part_bytes + w.sk_flag_bytes;
   } else {
     w.y_bytes = align256((size_t)B * K * d * 4);
     w.part_bytes = align256((size_t)B * K * V * 4);
@@ -578,10 +698,28 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
   p1.b1 = static_cast<const __nv_bfloat16*>(b1);
   p1.Y = Y;
   p1.status = status;
+  // Stream-K for the first GEMM when its few tiles would leave SMs idle for
+  // part of the run: every CTA then takes the same number of k-blocks (at
+  // least 8), and a tile cut between CTAs is finished by the one holding its
+  // first k-block.
+  {
+    const int sms = num_sms();
+    const int nkb = d / kTileK;
+    const long long total_kb = (long long)p1.n_tiles * nkb;
+    if (p1.n_tiles % sms != 0 && p1.n_tiles < 8 * sms && total_kb >= 8LL * sms) {
+      p1.kpc = (int)((total_kb + sms - 1) / sms);
+      p1.sk_grid = (int)((total_kb + p1.kpc - 1) / p1.kpc);
+      p1.sk_part = reinterpret_cast<float*>(wsb + w.y_bytes + 2 * w.part_bytes);
+      p1.sk_flag = reinterpret_cast<int*>(wsb + w.y_bytes + 2 * w.part_bytes + w.sk_part_bytes);
+      if (cudaMemsetAsync(p1.sk_flag, 0, (size_t)p1.sk_grid * sizeof(int), stream) != cudaSuccess)
+        return check_launch("heads stream-K flags");
+    }
+  }
   medusa_status_t st = launch_gemm_nb<kModeW1>(nb1, mA1, mB1, p1, stream);
   if (st != MEDUSA_OK) return st;
 
   GemmParams p2 = p1;
+  p2.kpc = 0;  // the second GEMM has many tiles per CTA: whole tiles round-robin
   p2.rows_per_head = V;
   p2.tiles_per_head = (V + kTileM - 1) / kTileM;
   p2.n_tiles = p2.tiles_per_head * K;
