@@ -1855,12 +1855,12 @@ static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaSt
   p.grid = device_sm_count();  // persistent: one CTA per SM
   p.slot_mul = 1;
   launch(tree_attn_tc_kernel<DH>, p.grid, kAttnThreads, L::kAlloc, stream, mK, mV, mKn, mVn, mKs0,
-                                                                        mVs0, mKs1, mVs1, mQ, p);
+         mVs0, mKs1, mVs1, mQ, p);
   medusa_status_t st = check_launch("tree_attention");
   if (st != MEDUSA_OK) return st;
   const int rows = p.B * p.Hkv * p.R;
-  launch(attn_combine_kernel<DH>, (rows + kCombineRows - 1) / kCombineRows, 256, 0, stream, p,
-         out, out_f32);
+  launch(attn_combine_kernel<DH>, (rows + kCombineRows - 1) / kCombineRows, 256, 0, stream, p, out,
+         out_f32);
   return check_launch("tree_attention_combine");
 }
 
@@ -1902,8 +1902,8 @@ static medusa_status_t launch_pair(AttnParams& p, void* out, int out_f32, cudaSt
   medusa_status_t st = check_launch("tree_attention_pair");
   if (st != MEDUSA_OK) return st;
   const int rows = p.B * p.Hkv * p.R;
-  launch(attn_combine_kernel<DH>, (rows + kCombineRows - 1) / kCombineRows, 256, 0, stream, p,
-         out, out_f32);
+  launch(attn_combine_kernel<DH>, (rows + kCombineRows - 1) / kCombineRows, 256, 0, stream, p, out,
+         out_f32);
   return check_launch("tree_attention_combine");
 }
 
@@ -1929,18 +1929,16 @@ medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_n
   if (dt == MEDUSA_F32) {
     const size_t total = (size_t)B * N * Hkv * dh;
     const int blocks = (int)((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
-    launch(tree_kv_write_f32_kernel, blocks, 256, 0, stream,
-        static_cast<const float*>(k_new), static_cast<const float*>(v_new),
-        static_cast<float*>(Kc), static_cast<float*>(Vc), prefix_len, B, N, Hkv, dh, cap,
-        max_prefix, status);
+    launch(tree_kv_write_f32_kernel, blocks, 256, 0, stream, static_cast<const float*>(k_new),
+           static_cast<const float*>(v_new), static_cast<float*>(Kc), static_cast<float*>(Vc),
+           prefix_len, B, N, Hkv, dh, cap, max_prefix, status);
     medusa_status_t st = check_launch("tree_kv_write_f32");
     if (st != MEDUSA_OK) return st;
     const int rows = B * N * Hq;
-    launch(tree_attn_f32_kernel, (rows + 7) / 8, 256, 0, stream,
-        static_cast<const float*>(q), static_cast<const float*>(k_new),
-        static_cast<const float*>(v_new), static_cast<const float*>(Kc),
-        static_cast<const float*>(Vc), prefix_len, anc_mask, B, N, Hq, Hkv, dh, cap, max_prefix,
-        words, scale, out, out_f32);
+    launch(tree_attn_f32_kernel, (rows + 7) / 8, 256, 0, stream, static_cast<const float*>(q),
+           static_cast<const float*>(k_new), static_cast<const float*>(v_new),
+           static_cast<const float*>(Kc), static_cast<const float*>(Vc), prefix_len, anc_mask, B, N,
+           Hq, Hkv, dh, cap, max_prefix, words, scale, out, out_f32);
     return check_launch("tree_attention_f32");
   }
   const Plan pl = plan(N, Hq, Hkv, max_prefix);

@@ -570,8 +570,8 @@ medusa_status_t topk_merge_lists(const float* vals, const int32_t* ids, int rows
                                  const int32_t* id_offsets, int kmax, int32_t* out_ids,
                                  float* out_vals, cudaStream_t stream) {
   const MergeLayout lay{row_stride, list_stride, list_len, id_offsets};
-  launch(topk_merge_kernel, rows * kMergeCtas, kMergeWarps * 32, 0, stream,
-      vals, ids, (long long)n_lists * list_len, kmax, out_ids, out_vals, lay);
+  launch(topk_merge_kernel, rows * kMergeCtas, kMergeWarps * 32, 0, stream, vals, ids,
+         (long long)n_lists * list_len, kmax, out_ids, out_vals, lay);
   return check_launch("topk_merge");
 }
 
@@ -658,19 +658,17 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
   if (dt == MEDUSA_F32) {
     float* y = reinterpret_cast<float*>(wsb);
     float* z = logits != nullptr ? logits : reinterpret_cast<float*>(wsb + w.y_bytes);
-    launch(heads_f32_w1_kernel, dim3((d + 7) / 8, K), 256, 0, stream,
-        static_cast<const float*>(h), static_cast<const float*>(W1),
-        static_cast<const float*>(b1), B, d, K, y);
+    launch(heads_f32_w1_kernel, dim3((d + 7) / 8, K), 256, 0, stream, static_cast<const float*>(h),
+           static_cast<const float*>(W1), static_cast<const float*>(b1), B, d, K, y);
     medusa_status_t st = check_launch("heads_f32_w1");
     if (st != MEDUSA_OK) return st;
-    launch(heads_f32_w2_kernel, dim3((V + 7) / 8, K), 256, 0, stream,
-        y, static_cast<const float*>(W2), B, d, V, K, z);
+    launch(heads_f32_w2_kernel, dim3((V + 7) / 8, K), 256, 0, stream, y,
+           static_cast<const float*>(W2), B, d, V, K, z);
     st = check_launch("heads_f32_w2");
     if (st != MEDUSA_OK) return st;
     const MergeLayout lay{(long long)V, (long long)V, V, nullptr};
     launch(topk_merge_kernel, B * K * kMergeCtas, kMergeWarps * 32, 0, stream, z, nullptr, V, kmax,
-                                                                            topk_ids, topk_vals,
-                                                                            lay);
+           topk_ids, topk_vals, lay);
     return check_launch("topk_merge");
   }
 
@@ -732,8 +730,8 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
 
   const long long C = (long long)p2.tiles_per_head * kmax;
   const MergeLayout lay{C, C, (int)C, nullptr};
-  launch(topk_merge_kernel, B * K * kMergeCtas, kMergeWarps * 32, 0, stream,
-      part_vals, part_ids, C, kmax, topk_ids, topk_vals, lay);
+  launch(topk_merge_kernel, B * K * kMergeCtas, kMergeWarps * 32, 0, stream, part_vals, part_ids, C,
+         kmax, topk_ids, topk_vals, lay);
   return check_launch("topk_merge");
 }
 

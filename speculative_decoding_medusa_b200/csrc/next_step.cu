@@ -43,8 +43,8 @@ medusa_status_t next_step(const void* node_hidden, int elem_bytes, const int32_t
                           int32_t* status, cudaStream_t stream) {
   const int row_vecs = d * elem_bytes / 16;
   launch(next_step_kernel, B, 128, 0, stream, static_cast<const uint4*>(node_hidden), N, row_vecs,
-                                          accept_len, accepted_nodes, max_depth + 1, bonus,
-                                          static_cast<uint4*>(h_next), root_next, status);
+         accept_len, accepted_nodes, max_depth + 1, bonus, static_cast<uint4*>(h_next), root_next,
+         status);
   return check_launch("next_step");
 }
 

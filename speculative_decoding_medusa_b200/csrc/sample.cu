@@ -159,12 +159,12 @@ medusa_status_t sample_bonus(const void* logits, medusa_dtype_t dt, const int32_
   const uint32_t o0 = (uint32_t)offset, o1 = (uint32_t)(offset >> 32);
   if (dt == MEDUSA_BF16)
     launch(sample_bonus_kernel<__nv_bfloat16>, B, kSampleThreads, 0, stream,
-        static_cast<const __nv_bfloat16*>(logits), accept_len, accepted_nodes, N, V,
-        max_depth + 1, inv_T, s0, s1, o0, o1, bonus, accepted_tokens, status);
+           static_cast<const __nv_bfloat16*>(logits), accept_len, accepted_nodes, N, V,
+           max_depth + 1, inv_T, s0, s1, o0, o1, bonus, accepted_tokens, status);
   else
     launch(sample_bonus_kernel<float>, B, kSampleThreads, 0, stream,
-        static_cast<const float*>(logits), accept_len, accepted_nodes, N, V, max_depth + 1, inv_T,
-        s0, s1, o0, o1, bonus, accepted_tokens, status);
+           static_cast<const float*>(logits), accept_len, accepted_nodes, N, V, max_depth + 1,
+           inv_T, s0, s1, o0, o1, bonus, accepted_tokens, status);
   return check_launch("sample_bonus");
 }
 

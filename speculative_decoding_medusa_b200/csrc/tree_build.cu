@@ -124,9 +124,9 @@ medusa_status_t tree_build(const medusa_tree_t& t, const int32_t* root_tok, cons
                            int K, int kmax, const int32_t* prefix_len, int B, int32_t* cand_ids,
                            int32_t* pos_ids, uint32_t* anc_mask, int32_t* retrieve,
                            int32_t* status, cudaStream_t stream) {
-  launch(tree_build_kernel, B, MEDUSA_MAX_NODES, (size_t)K * kmax * sizeof(int), stream,
-      t.parent, t.depth, t.rank, t.n_nodes, t.max_depth, t.n_leaves, root_tok, topk_ids, K, kmax,
-      prefix_len, cand_ids, pos_ids, anc_mask, retrieve, status);
+  launch(tree_build_kernel, B, MEDUSA_MAX_NODES, (size_t)K * kmax * sizeof(int), stream, t.parent,
+         t.depth, t.rank, t.n_nodes, t.max_depth, t.n_leaves, root_tok, topk_ids, K, kmax,
+         prefix_len, cand_ids, pos_ids, anc_mask, retrieve, status);
   return check_launch("tree_build");
 }
 

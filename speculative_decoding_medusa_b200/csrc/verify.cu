@@ -524,11 +524,10 @@ medusa_status_t verify_path_from_parts(const RowPart* part, int n_chunks,
   const int N = tree.n_nodes;
   const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
   const float inv_T = typical ? 1.0f / temperature : 1.0f;
-  launch(verify_path_kernel<__nv_bfloat16>, B, kPathThreads, 0, stream,
-      nullptr, hidden, lm_head, d, part, n_chunks, n_chunks, 1, path_threads_per_node(N, n_chunks),
-      nullptr, cand_ids,
-      tree.parent, tree.depth, N, tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta,
-      accept_len, accepted_nodes, accepted_tokens, bonus, status);
+  launch(verify_path_kernel<__nv_bfloat16>, B, kPathThreads, 0, stream, nullptr, hidden, lm_head, d,
+         part, n_chunks, n_chunks, 1, path_threads_per_node(N, n_chunks), nullptr, cand_ids,
+         tree.parent, tree.depth, N, tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta,
+         accept_len, accepted_nodes, accepted_tokens, bonus, status);
   return check_launch("verify_path");
 }
 
@@ -610,29 +609,29 @@ medusa_status_t verify_records(const void* logits, medusa_dtype_t dt, const int3
     if (typical) {
       auto k = verify_rows_kernel<__nv_bfloat16, true>;
       launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V_shard, n_chunks, n_items,
-                                                              inv_T, part, status);
+             inv_T, part, status);
     } else {
       auto k = verify_rows_kernel<__nv_bfloat16, false>;
       launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V_shard, n_chunks, n_items,
-                                                              inv_T, part, status);
+             inv_T, part, status);
     }
-    launch(shard_records_kernel<__nv_bfloat16>, grid, 256, 0, stream,
-        lg, part, n_chunks, cand_ids, tree.parent, B, N, V_shard, v_offset, typical ? 1 : 0,
-        inv_T, records, cand_logit, status);
+    launch(shard_records_kernel<__nv_bfloat16>, grid, 256, 0, stream, lg, part, n_chunks, cand_ids,
+           tree.parent, B, N, V_shard, v_offset, typical ? 1 : 0, inv_T, records, cand_logit,
+           status);
   } else {
     const float* lg = static_cast<const float*>(logits);
     if (typical) {
       auto k = verify_rows_kernel<float, true>;
       launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V_shard, n_chunks, n_items,
-                                                              inv_T, part, status);
+             inv_T, part, status);
     } else {
       auto k = verify_rows_kernel<float, false>;
       launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V_shard, n_chunks, n_items,
-                                                              inv_T, part, status);
+             inv_T, part, status);
     }
-    launch(shard_records_kernel<float>, grid, 256, 0, stream,
-        lg, part, n_chunks, cand_ids, tree.parent, B, N, V_shard, v_offset, typical ? 1 : 0,
-        inv_T, records, cand_logit, status);
+    launch(shard_records_kernel<float>, grid, 256, 0, stream, lg, part, n_chunks, cand_ids,
+           tree.parent, B, N, V_shard, v_offset, typical ? 1 : 0, inv_T, records, cand_logit,
+           status);
   }
   return check_launch("verify_records");
 }
@@ -647,11 +646,10 @@ medusa_status_t verify_from_records(const RowPart* records, int G, const float* 
   const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
   const float inv_T = typical ? 1.0f / temperature : 1.0f;
   // records are shard-major: [G][B * N]
-  launch(verify_path_kernel<float>, B, kPathThreads, 0, stream,
-      nullptr, nullptr, nullptr, 0, records, G, 1, (long long)B * N,
-      path_threads_per_node(N, G), cand_logit, cand_ids, tree.parent, tree.depth, N,
-      tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes,
-      accepted_tokens, bonus, status);
+  launch(verify_path_kernel<float>, B, kPathThreads, 0, stream, nullptr, nullptr, nullptr, 0,
+         records, G, 1, (long long)B * N, path_threads_per_node(N, G), cand_logit, cand_ids,
+         tree.parent, tree.depth, N, tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta,
+         accept_len, accepted_nodes, accepted_tokens, bonus, status);
   return check_launch("verify_path");
 }
 
@@ -677,36 +675,36 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
     if (typical) {
       auto k = verify_rows_kernel<__nv_bfloat16, true>;
       launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V, n_chunks, n_items, inv_T,
-                                                              part, status);
+             part, status);
     } else {
       auto k = verify_rows_kernel<__nv_bfloat16, false>;
       launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V, n_chunks, n_items, inv_T,
-                                                              part, status);
+             part, status);
     }
     medusa_status_t st = check_launch("verify_rows");
     if (st != MEDUSA_OK) return st;
-    launch(verify_path_kernel<__nv_bfloat16>, B, kPathThreads, 0, stream,
-        lg, nullptr, nullptr, 0, part, n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
-        typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
-        status);
+    launch(verify_path_kernel<__nv_bfloat16>, B, kPathThreads, 0, stream, lg, nullptr, nullptr, 0,
+           part, n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N,
+           tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes,
+           accepted_tokens, bonus, status);
     return check_launch("verify_path");
   }
   const float* lg = static_cast<const float*>(logits);
   if (typical) {
     auto k = verify_rows_kernel<float, true>;
-    launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V, n_chunks, n_items, inv_T, part,
-                                                            status);
+    launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V, n_chunks, n_items, inv_T,
+           part, status);
   } else {
     auto k = verify_rows_kernel<float, false>;
-    launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V, n_chunks, n_items, inv_T, part,
-                                                            status);
+    launch(k, rows_grid(k, n_items), kRowWarps * 32, 0, stream, lg, V, n_chunks, n_items, inv_T,
+           part, status);
   }
   medusa_status_t st = check_launch("verify_rows");
   if (st != MEDUSA_OK) return st;
-  launch(verify_path_kernel<float>, B, kPathThreads, 0, stream,
-      lg, nullptr, nullptr, 0, part, n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N, tree.max_depth, V,
-      typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
-      status);
+  launch(verify_path_kernel<float>, B, kPathThreads, 0, stream, lg, nullptr, nullptr, 0, part,
+         n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N, tree.max_depth,
+         V, typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
+         status);
   return check_launch("verify_path");
 }
 
