@@ -544,6 +544,30 @@ def main():
               for i, n in enumerate(names)}  # us
     assert int(step.status.item()) == 0
 
+    # ---- the step captured in one CUDA graph and replayed: per-step
+    # percentiles (an event between replays) ----
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            one_step()
+    stream.wait_stream(side)
+    n_rep = min(max(args.steps, 20), 200)
+    rep_evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_rep + 1)]
+    for _ in range(3):
+        graph.replay()
+    rep_evs[0].record(stream)
+    for k in range(n_rep):
+        graph.replay()
+        rep_evs[k + 1].record(stream)
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    per_step = sorted(rep_evs[k].elapsed_time(rep_evs[k + 1]) * 1e3 for k in range(n_rep))
+    step_us = {"graph": True, "replays": n_rep, "p10": per_step[n_rep // 10],
+               "p50": per_step[n_rep // 2], "p90": per_step[(9 * n_rep) // 10]}
+    del graph
+
     # ---- end to end through the public API with host buffers ----
     host_in = {k: v.cpu().pin_memory() for k, v in
                {"h": hin["h"], "root": root, "q": att["q"], "k_new": att["k_new"],
@@ -613,6 +637,7 @@ def main():
             "hbm_roofline_frac_step": step_gbs / hbm_peak,
             "step_bytes": ab["total"],
             "stages_us": stages,
+            "step_us": step_us,
             "roofline": {"bound": "hbm", "kernel": "medusa_heads_topk (W1 GEMM + W2 GEMM + top-k merge)",
                          "achieved": heads_gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": heads_gbs / hbm_peak, "traffic": traffic,
