@@ -49,6 +49,17 @@ def _peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+def workload_of(args, W):
+    """The named workload with the --nodes and --batch overrides applied."""
+    w = W.WORKLOADS[args.workload]
+    over = {}
+    if args.nodes:
+        over["N"] = args.nodes
+    if args.batch:
+        over["B"] = args.batch
+    return W.scaled(w, **over) if over else w
+
+
 def heads_traffic(algorithmic):
     """DRAM bytes of one heads call, scaled from the profiled ratio; None when
     the kernel sources changed since the counters were taken."""
@@ -230,6 +241,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama3_8b")
     ap.add_argument("--nodes", type=int, default=None, help="tree size override (long: 16/64/128)")
+    ap.add_argument("--batch", type=int, default=None, help="batch override (llama3_8b: 1..8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--loop-steps", type=int, default=16,
@@ -253,7 +265,7 @@ def run_loop(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    w = W.WORKLOADS[args.workload]
+    w = workload_of(args, W)
     R = args.loop_steps
     spec = W.tree_for(w)
     N = spec.n_nodes
@@ -326,10 +338,8 @@ def run_stage(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    w = W.WORKLOADS[args.workload]
-    N = args.nodes or w.N
-    if args.nodes:
-        w = W.scaled(w, N=N)
+    w = workload_of(args, W)
+    N = w.N
     spec = W.tree_for(w, n_nodes=N)
     tree = M.Tree.from_spec(spec, dev)
     att = W.attention_inputs(w, seed=0, device=dev, n_nodes=N)
@@ -403,8 +413,8 @@ def run_reference(args):
     if rank != 0:
         return 0
     from speculative_decoding_medusa_b200 import workloads as W
-    w = W.WORKLOADS[args.workload]
-    N = args.nodes or w.N
+    w = workload_of(args, W)
+    N = w.N
     times = []
     for i in range(args.warmup + args.steps):
         r = oracle_sample(w, N, seed=i)
@@ -453,10 +463,8 @@ def main():
                                 device_id=dev)
     M.lib()  # fails loudly when the library is missing
 
-    w = W.WORKLOADS[args.workload]
-    N = args.nodes or w.N
-    if args.nodes:
-        w = W.scaled(w, N=N)
+    w = workload_of(args, W)
+    N = w.N
     spec = W.tree_for(w, n_nodes=N)
     seed = rank
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
