@@ -214,7 +214,9 @@ MEDUSA_API medusa_status_t medusa_tree_build(const medusa_tree_t* tree, const in
  * Workspace: medusa_tree_attention_workspace_size(...) bytes (partial
  *   results of key ranges, merged at the end), 256-byte aligned.
  * Precision: bf16 q/k/v, fp32 scores, fp32 softmax statistics; the softmax
- *   weights enter the value product as two bf16 terms (hi + lo).
+ *   weights (at most 2^8 relative to the running maximum) enter the value
+ *   product as fp16, with V converted to fp16 in shared memory: |v| >= 65536,
+ *   inf or NaN in V is reported as MEDUSA_ERR_DEVICE_CHECK.
  *   dt = MEDUSA_F32 runs an fp32 CUDA-core path.
  * Limits: Hq % Hkv == 0; bf16: dh in {64, 128}, B <= 256, pointers 16-byte
  *   aligned; f32: dh <= 256 and dh % 32 == 0; N <= MEDUSA_MAX_NODES.
