@@ -21,6 +21,7 @@ MEDUSA_ACCEPT_TYPICAL = 1
 MAX_NODES = 256
 MAX_KMAX = 32
 MAX_HEADS = 16
+MAX_BATCH = 128
 
 STATUS_NAMES = {
     0: "MEDUSA_OK", 1: "MEDUSA_ERR_INVALID_ARG", 2: "MEDUSA_ERR_SHAPE",

@@ -199,6 +199,17 @@ def cartesian_tree(widths: Sequence[int], n_nodes: Optional[int] = None) -> Tree
     return _spec_from_paths(paths)
 
 
+def limits_tree(n_nodes: int, depth: int, kmax: int) -> TreeSpec:
+    """A tree at the size limits: the chain of rank-0 nodes down to ``depth``,
+    then, breadth-first, every other rank 1..kmax-1 under each chain node,
+    until ``n_nodes`` nodes.  The deepest node and the largest rank are both
+    present whenever n_nodes >= depth + kmax."""
+    chain = [tuple([0] * t) for t in range(depth + 1)]
+    rest = [tuple([0] * (t - 1)) + (r,) for t in range(1, depth + 1) for r in range(1, kmax)]
+    rest.sort(key=lambda p: (len(p), p))
+    return _spec_from_paths(chain + rest[: n_nodes - len(chain)])
+
+
 def sparse_tree(n_nodes: int, n_heads: int, topk: int, seed: int,
                 max_depth: int = 5) -> TreeSpec:
     """Seeded stand-in for the accuracy-driven sparse tree.

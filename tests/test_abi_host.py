@@ -134,3 +134,12 @@ def test_workspace_queries(L):
     assert M.medusa_tree_attention_workspace_size(8, 64, 32, 8, 128, 8192, 0) > 0
     assert M.medusa_tree_attention_workspace_size(1, 9, 4, 4, 64, 128, 1) == 0  # f32 needs none
     assert M.medusa_verify_accept_workspace_size(8, 64, 128256) > 0
+
+
+def test_python_limits_match_the_header():
+    """The binding's size limits are the header's #defines."""
+    src = open(os.path.join(ROOT, "include", "medusa.h")).read()
+    defs = dict(re.findall(r"#define MEDUSA_(MAX_\w+)\s+(\d+)", src))
+    assert set(defs) == {"MAX_NODES", "MAX_KMAX", "MAX_HEADS", "MAX_BATCH"}, defs
+    for name, value in defs.items():
+        assert getattr(_lib, name) == int(value), name

@@ -93,6 +93,7 @@ def test_tiny_fp32():
     (1, 8, 8, 128, (1500, 1500), "dense256", 4),   # 256 nodes, 8 mask words
     (2, 6, 2, 128, (50, 300), "sparse16", 5),      # G 3: Q rows gathered by threads
     (1, 16, 1, 64, (200, 200), "sparse64", 6),     # G 16: four query groups of 256 rows
+    (256, 2, 1, 64, (0, 40), "sparse16", 7),       # 256 sequences: the schedule table is full
 ])
 @pytest.mark.parametrize("pair", [True, False], ids=["pair", "single"])
 def test_bf16_small(B, Hq, Hkv, dh, ctx, tree, seed, pair, monkeypatch):

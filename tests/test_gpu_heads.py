@@ -52,6 +52,7 @@ def test_tiny_fp32(zero_init):
     (100, 64, 300, 2, 8),       # 256-wide MMA, one k-block
     (4, 2048, 3000, 3, 10),     # stream-K first GEMM: 48 tiles of 32 k-blocks, 11 per CTA
     (20, 2048, 1500, 3, 5),     # the same at 32 columns
+    (128, 128, 700, 16, 32),    # the limits: MAX_BATCH sequences, MAX_HEADS heads, MAX_KMAX
 ])
 def test_bf16_small(B, d, V, K, kmax):
     w = _case("vicuna7b", B=B, d=d, V=V, K=K, kmax=kmax)

@@ -118,3 +118,57 @@ def test_kv_compact_rejects_out_of_range_path():
     torch.cuda.synchronize()
     assert int(status.item()) == 6
     assert torch.equal(Kg[0], before[0]) and int(pl[0].item()) == prefix[0]
+
+
+def test_tree_build_at_the_limits():
+    """MAX_NODES nodes, a depth of K = MAX_HEADS, ranks up to MAX_KMAX - 1 and
+    MAX_BATCH sequences: bit-exact."""
+    spec = W.limits_tree(M.MAX_NODES, M.MAX_HEADS, M.MAX_KMAX)
+    assert spec.max_depth == M.MAX_HEADS and spec.rank.max() == M.MAX_KMAX - 1
+    w = W.scaled(W.WORKLOADS["llama3_8b"], B=M.MAX_BATCH, K=M.MAX_HEADS, kmax=M.MAX_KMAX,
+                 N=spec.n_nodes)
+    root = W.random_root_tokens(w, seed=9)
+    topk_ids = W.random_topk_ids(w, seed=9)
+    prefix = W.prefix_lengths(w, seed=9)
+    got, st = _build(spec, root, topk_ids, prefix)
+    assert st == 0
+    ref = O.tree_build(spec.parent, spec.depth, spec.rank, i64(root), i64(topk_ids), i64(prefix))
+    for k in ("cand", "pos", "retrieve"):
+        np.testing.assert_array_equal(got[k], ref[k], err_msg=k)
+    np.testing.assert_array_equal(got["mask"].view(np.uint32), ref["mask"])
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_kv_compact_deepest_path(dtype):
+    """max_depth = MAX_HEADS - 1, the deepest path compaction takes: every
+    sequence keeps a full-length path, some of them the first nodes (sources
+    that are other steps' destinations)."""
+    max_depth = M.MAX_HEADS - 1
+    B, Hkv, dh, N, cap = 4, 8, 128, 256, 700
+    rng = np.random.default_rng(21)
+    prefix = rng.integers(0, cap - N, size=B).astype(np.int32)
+    g = torch.Generator().manual_seed(21)
+    Kc = torch.randn(B, Hkv, cap, dh, generator=g).to(dtype)
+    Vc = torch.randn(B, Hkv, cap, dh, generator=g).to(dtype)
+    L = np.full(B, max_depth, dtype=np.int32)
+    nodes = np.zeros((B, max_depth + 1), dtype=np.int32)
+    for b in range(B):
+        if b % 2:
+            nodes[b] = np.arange(max_depth + 1)  # node j at slot P + j: stays in place
+            nodes[b, 1:] += 1                    # shifted by one: overlapping chain
+        else:
+            nodes[b, 1:] = np.sort(rng.choice(np.arange(1, N), size=max_depth, replace=False))
+    ref = O.kv_compact(Kc.float().numpy(), Vc.float().numpy(), prefix, nodes, L)
+    dev = "cuda"
+    Kg, Vg = Kc.to(dev), Vc.to(dev)
+    pl = torch.from_numpy(prefix).to(dev)
+    src = torch.full(nodes.shape, -9, dtype=torch.int32, device=dev)
+    status = M.new_status()
+    M.medusa_kv_compact(Kg, Vg, pl, torch.from_numpy(nodes).to(dev), torch.from_numpy(L).to(dev),
+                        src, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    np.testing.assert_array_equal(Kg.float().cpu().numpy(), ref["Kc"])
+    np.testing.assert_array_equal(Vg.float().cpu().numpy(), ref["Vc"])
+    np.testing.assert_array_equal(pl.cpu().numpy(), ref["prefix_len"])
+    np.testing.assert_array_equal(src.cpu().numpy(), ref["compact_src"])

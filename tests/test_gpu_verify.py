@@ -141,3 +141,38 @@ def test_full_size_typical_llama3_70b():
     ref = O.verify_typical(f64(logits), cand, spec.parent, spec.depth, spec.max_depth,
                            w.temperature, w.eps, w.delta)
     _assert_same(got, ref)
+
+
+@pytest.mark.parametrize("mode", ["greedy", "typical"])
+def test_deepest_tree_full_acceptance(mode):
+    """MAX_NODES nodes at depth MAX_HEADS - 1: sequence 0's logits make the
+    whole rank-0 chain the base model's choice, so it keeps the deepest
+    node; the others follow the seeded draw."""
+    spec = W.limits_tree(M.MAX_NODES, M.MAX_HEADS - 1, M.MAX_KMAX)
+    base = W.WORKLOADS["llama3_70b"] if mode == "typical" else W.WORKLOADS["llama3_8b"]
+    w = W.scaled(base, B=3, V=5000, K=M.MAX_HEADS, kmax=M.MAX_KMAX, N=spec.n_nodes)
+    cand = _cands(w, spec, 11)
+    chain = [i for i in range(spec.n_nodes) if all(r == 0 for r in spec.paths[i])]
+    for attempt in range(20):
+        logits = W.verify_logits(w, spec, torch.from_numpy(cand), seed=11, attempt=attempt).float()
+        for a, c in zip(chain[:-1], chain[1:]):
+            logits[0, a, cand[0, c]] = logits[0, a].max() + 8.0
+        logits = logits.to(torch.bfloat16)
+        if mode == "greedy":
+            break
+        # typical: redraw until fp32 and fp64 take the same decisions
+        m = O.typical_log_margin(f64(logits), cand, spec.parent, w.temperature, w.eps, w.delta)
+        if np.abs(m[:, 1:]).min() > TYPICAL_LOG_MARGIN:
+            break
+    else:
+        pytest.skip("no margin-clean draw")
+    if mode == "greedy":
+        got = _run(logits, cand, spec, M.MEDUSA_ACCEPT_GREEDY)
+        ref = O.verify_greedy(f64(logits), cand, spec.parent, spec.depth, spec.max_depth)
+    else:
+        got = _run(logits, cand, spec, M.MEDUSA_ACCEPT_TYPICAL, w.temperature, w.eps, w.delta)
+        ref = O.verify_typical(f64(logits), cand, spec.parent, spec.depth, spec.max_depth,
+                               w.temperature, w.eps, w.delta)
+    _assert_same(got, ref)
+    assert ref["accept_len"][0] == M.MAX_HEADS - 1
+    np.testing.assert_array_equal(ref["accepted_nodes"][0], chain)
