@@ -47,7 +47,7 @@ constexpr int kAttnThreads = 384;    // producer, MMA, two softmax warpgroups, t
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold, log2 units
 constexpr uint32_t kAttnTmemCols = 512;
 constexpr int kAttnMaxB = 256;       // sequences per call (schedule table in shared memory)
-constexpr int kAttnMinTiles = 8;     // smallest tile range a CTA takes
+constexpr int kAttnMinTiles = 4;     // smallest tile range a CTA takes
 
 // 2^x with the SFU instruction (ex2.approx; relative error about 2^-22, -inf -> 0)
 __device__ __forceinline__ float ex2_approx(float x) {
