@@ -64,23 +64,68 @@ struct GemmParams {
   float* sk_part;  // [grid][kTileM][NB] fp32 partial of a CTA's leading tile tail
   int* sk_flag;    // [grid] 1 once that partial is written (zeroed before the launch)
   int sk_grid;     // CTAs of a stream-K launch
+  // second GEMM: tiles handed out by this counter (tiles past the first
+  // grid-full are claimed one at a time); the first GEMM zeroes it.  Null:
+  // whole tiles round-robin.
+  int* tile_counter;
 };
+
+// tile ids a CTA's producer has claimed and not every role has read yet: the
+// producer runs at most S stages ahead of the MMA issuer, which runs at most
+// two tiles ahead of the epilogue, so S + 3 <= 11 slots are ever in use
+constexpr int kTileRing = 16;
 
 // One CTA's work as (tile, first k-block, end k-block) segments, in order.
 // Round-robin: whole tiles blockIdx.x, + gridDim.x, ...  Stream-K: the
 // k-blocks [blockIdx.x * kpc, + kpc) of the tile-major sequence, cut at tile
-// ends; only the first segment can start inside a tile.
+// ends; only the first segment can start inside a tile.  Dynamic (whole
+// tiles): tile blockIdx.x first, then tiles gridDim.x + (counter++) until
+// they run out, so that CTAs which stream faster take more tiles; the
+// producer claims each tile and publishes it in a ring slot with its own
+// mbarrier, which the MMA issuer and the epilogue wait on before reading it.
 struct SegIter {
   int nkb, n_tiles, kpc, tile, g, g_hi;
-  __device__ __forceinline__ void init(const GemmParams& p, int nkb_) {
+  int* counter;        // dynamic mode when set
+  int* ring;           // [kTileRing] tile ids
+  uint64_t* ring_bar;  // [kTileRing]
+  bool producer;
+  int it;
+  volatile int* abort;
+  int32_t* status;
+  __device__ __forceinline__ void init(const GemmParams& p, int nkb_, int* counter_ = nullptr,
+                                       int* ring_ = nullptr, uint64_t* ring_bar_ = nullptr,
+                                       bool producer_ = false, volatile int* abort_ = nullptr) {
     nkb = nkb_;
     n_tiles = p.n_tiles;
     kpc = p.kpc;
     tile = blockIdx.x;
     g = blockIdx.x * kpc;
     g_hi = min(g + kpc, n_tiles * nkb);
+    counter = counter_;
+    ring = ring_;
+    ring_bar = ring_bar_;
+    producer = producer_;
+    it = 0;
+    abort = abort_;
+    status = p.status;
   }
   __device__ __forceinline__ bool next(int& t, int& kb0, int& kb1) {
+    if (counter != nullptr) {
+      const int slot = it % kTileRing;
+      if (producer) {
+        t = it == 0 ? static_cast<int>(blockIdx.x)
+                    : static_cast<int>(gridDim.x) + atomicAdd(counter, 1);
+        ring[slot] = t;
+        mbar_arrive(&ring_bar[slot]);  // release: the id is visible to its waiters
+      } else {
+        if (!mbar_wait_bounded(&ring_bar[slot], (it / kTileRing) & 1, abort, status)) return false;
+        t = ring[slot];
+      }
+      ++it;
+      kb0 = 0;
+      kb1 = nkb;
+      return t < n_tiles;
+    }
     if (kpc > 0) {
       if (g >= g_hi) return false;
       t = g / nkb;
@@ -106,11 +151,12 @@ struct GemmSmem {
   static constexpr int kAOff = 0;
   static constexpr int kBOff = S * kABytes;
   static constexpr int kBarOff = kBOff + S * kBBytes;
-  // full[S], empty[S], tfull[2], tempty[2], drain, epilogue
-  static constexpr int kNumBars = 2 * S + 6;
+  // full[S], empty[S], tfull[2], tempty[2], drain, epilogue, ring[kTileRing]
+  static constexpr int kNumBars = 2 * S + 6 + kTileRing;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kRingOff = kMiscOff + 16;  // [kTileRing] claimed tile ids
   // per-warp sorted lists of the W2 epilogue: [4 quads][8 sequences][32] (value, index)
-  static constexpr int kListOff = kMiscOff + 16;
+  static constexpr int kListOff = kRingOff + kTileRing * 4;
   static constexpr int kListBytes = 4 * 8 * 32 * 8;
   static constexpr int kBytes = kListOff + kListBytes;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base
@@ -156,6 +202,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                       const __grid_constant__ CUtensorMap tmB, GemmParams p) {
   grid_dep_wait();
   grid_dep_launch();
+  // the first GEMM resets the second GEMM's tile counter (the second GEMM
+  // reads it only after waiting for this kernel)
+  if (MODE == kModeW1 && p.tile_counter != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
+    *p.tile_counter = 0;
   using L = GemmSmem<NB, S>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -166,8 +216,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tempty = bars + 2 * S + 2;
   uint64_t* drain = bars + 2 * S + 4;
   uint64_t* epi = bars + 2 * S + 5;
+  uint64_t* ring_bar = bars + 2 * S + 6;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  int* ring = reinterpret_cast<int*>(smem + L::kRingOff);
+  // the second GEMM hands out tiles dynamically when given a counter
+  int* const dyn_counter = MODE == kModeW2 ? p.tile_counter : nullptr;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -184,6 +238,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(drain, 1);
     mbar_init(epi, 128);
+    for (int i = 0; i < kTileRing; ++i) mbar_init(&ring_bar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -206,7 +261,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int g = 0;
       bool ok = true;
       SegIter seg;
-      seg.init(p, nkb);
+      seg.init(p, nkb, dyn_counter, ring, ring_bar, true, abort_flag);
       int tile, kb0, kb1;
       while (ok && seg.next(tile, kb0, kb1)) {
         const int head = tile / p.tiles_per_head;
@@ -239,7 +294,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int g = 0, it = 0;
       bool ok = true;
       SegIter seg;
-      seg.init(p, nkb);
+      seg.init(p, nkb, dyn_counter, ring, ring_bar, false, abort_flag);
       int tile, kb0, kb1;
       for (; ok && seg.next(tile, kb0, kb1); ++it) {
         const int acc = it & 1;
@@ -287,7 +342,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     };
     int it = 0;
     SegIter seg;
-    seg.init(p, nkb);
+    seg.init(p, nkb, dyn_counter, ring, ring_bar, false, abort_flag);
     int tile, kb0, kb1;
     for (; epi_ok && seg.next(tile, kb0, kb1); ++it) {
       const int acc = it & 1;
@@ -621,7 +676,7 @@ int round_nb(int cols) {
 }
 
 struct HeadsWs {
-  size_t y_bytes, part_bytes, sk_part_bytes, sk_flag_bytes, total;
+  size_t y_bytes, part_bytes, sk_part_bytes, sk_flag_bytes, counter_bytes, total;
 };
 
 HeadsWs heads_ws_layout(int B, int d, int V, int K, int kmax, medusa_dtype_t dt) {
@@ -634,7 +689,9 @@ HeadsWs heads_ws_layout(int B, int d, int V, int K, int kmax, medusa_dtype_t dt)
     // flag per CTA
     w.sk_part_bytes = align256((size_t)num_sms() * kTileM * round_nb(B) * 4);
     w.sk_flag_bytes = align256((size_t)num_sms() * 4);
-    w.total = w.y_bytes + 2 * w.part_bytes + w.sk_part_bytes + w.sk_flag_bytes;
+    // the second GEMM's tile counter
+    w.counter_bytes = 256;
+    w.total = w.y_bytes + 2 * w.part_bytes + w.sk_part_bytes + w.sk_flag_bytes + w.counter_bytes;
   } else {
     w.y_bytes = align256((size_t)B * K * d * 4);
     w.part_bytes = align256((size_t)B * K * V * 4);
@@ -696,6 +753,8 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
   p1.b1 = static_cast<const __nv_bfloat16*>(b1);
   p1.Y = Y;
   p1.status = status;
+  p1.tile_counter = reinterpret_cast<int*>(wsb + w.y_bytes + 2 * w.part_bytes + w.sk_part_bytes +
+                                           w.sk_flag_bytes);
   // Stream-K for the first GEMM when its few tiles would leave SMs idle for
   // part of the run: every CTA then takes the same number of k-blocks (at
   // least 8), and a tile cut between CTAs is finished by the one holding its
@@ -717,7 +776,7 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
   if (st != MEDUSA_OK) return st;
 
   GemmParams p2 = p1;
-  p2.kpc = 0;  // the second GEMM has many tiles per CTA: whole tiles round-robin
+  p2.kpc = 0;  // the second GEMM has many tiles per CTA: whole tiles, handed out dynamically
   p2.rows_per_head = V;
   p2.tiles_per_head = (V + kTileM - 1) / kTileM;
   p2.n_tiles = p2.tiles_per_head * K;
