@@ -68,6 +68,10 @@ struct GemmParams {
   // grid-full are claimed one at a time); the first GEMM zeroes it.  Null:
   // whole tiles round-robin.
   int* tile_counter;
+  // second GEMM: 1 = each CTA keeps a best-32 list per (head, sequence) in
+  // shared memory across its tiles and writes one list per row at the end
+  // (list blockIdx.x of gridDim.x); 0 = one list per tile (list tile_in_head)
+  int run_lists;
 };
 
 // tile ids a CTA's producer has claimed and not every role has read yet: the
@@ -160,7 +164,14 @@ struct GemmSmem {
   static constexpr int kListBytes = 4 * 8 * 32 * 8;
   static constexpr int kBytes = kListOff + kListBytes;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base
+  // running lists (second GEMM, run_lists): [K*B][32] values, then ids,
+  // after kBytes; K*B*256 bytes more at launch
 };
+
+// a (head, sequence) row's running list takes 32 values and 32 ids
+constexpr int kRunRowBytes = 32 * 8;
+constexpr int kRunMaxRows = 128;  // K * B up to which the running lists are used
+constexpr int kSmemLimit = 227 * 1024;
 
 template <int NB>
 __host__ __device__ constexpr uint32_t tmem_cols() {
@@ -340,6 +351,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       epi_phase ^= 1u;
       return epi_ok;
     };
+    // running lists of the second GEMM: warp quad owns the sequences b with
+    // b % 4 == quad (the warp that merges them in every tile below), so a
+    // row's list is only ever touched by one warp
+    const bool run = MODE == kModeW2 && p.run_lists != 0;
+    const int run_rows = p.n_heads * p.B;
+    float* run_v = reinterpret_cast<float*>(smem + L::kBytes);
+    int* run_i = reinterpret_cast<int*>(smem + L::kBytes + (size_t)run_rows * 32 * 4);
+    if (run) {
+      for (int e = threadIdx.x - 64; e < run_rows * 32; e += 128) {
+        run_v[e] = -INFINITY;
+        run_i[e] = 0x7fffffff;
+      }
+      epi_sync();
+    }
     int it = 0;
     SegIter seg;
     seg.init(p, nkb, dyn_counter, ring, ring_bar, false, abort_flag);
@@ -443,7 +468,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int q2 = 1; q2 < 4; ++q2)
               warp_merge_top32(rv, ri, lv[(q2 * 8 + t) * 32 + lane], li[(q2 * 8 + t) * 32 + lane]);
-            if (lane < p.kmax) {
+            if (run) {
+              const int at = (head * p.B + b) * 32 + lane;
+              warp_merge_top32(rv, ri, run_v[at], run_i[at]);
+              run_v[at] = rv;
+              run_i[at] = ri;
+            } else if (lane < p.kmax) {
               const size_t row_bk = (size_t)b * p.n_heads + head;
               const size_t o = (row_bk * p.tiles_per_head + tile_in_head) * p.kmax + lane;
               p.part_vals[o] = rv;
@@ -455,6 +485,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
+    }
+    // one list per (sequence, head) row: list blockIdx.x of gridDim.x
+    if (run && epi_ok) {
+      for (int rr = 0; rr < run_rows; ++rr) {
+        const int head = rr / p.B, b = rr - head * p.B;
+        if ((b & 3) != quad) continue;  // the warp that owns the row
+        if (lane < p.kmax) {
+          const size_t o = (((size_t)b * p.n_heads + head) * gridDim.x + blockIdx.x) * p.kmax + lane;
+          p.part_vals[o] = run_v[rr * 32 + lane];
+          p.part_ids[o] = run_i[rr * 32 + lane];
+        }
+      }
     }
   }
 
@@ -643,17 +685,34 @@ bool make_map_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim
 
 int num_sms() { return device_sm_count(); }
 
+int gemm_grid(const GemmParams& p) {
+  return p.kpc > 0 ? p.sk_grid : (p.n_tiles < num_sms() ? p.n_tiles : num_sms());
+}
+
 template <int NB, int S, int MODE>
 medusa_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
                             cudaStream_t stream) {
   using L = GemmSmem<NB, S>;
   auto kern = heads_gemm_kernel<NB, S, MODE>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
+  const size_t smem =
+      L::kAlloc + (p.run_lists ? (size_t)p.n_heads * p.B * kRunRowBytes : (size_t)0);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(heads_gemm) failed");
-  const int grid = p.kpc > 0 ? p.sk_grid : (p.n_tiles < num_sms() ? p.n_tiles : num_sms());
-  launch(kern, grid, kGemmThreads, L::kAlloc, stream, a, b, p);
+  launch(kern, gemm_grid(p), kGemmThreads, smem, stream, a, b, p);
   return check_launch("heads_gemm");
+}
+
+// shared memory of the GEMM at width nb before any running lists
+size_t gemm_alloc_bytes(int nb) {
+  switch (nb) {
+    case 16: return GemmSmem<16, 8>::kAlloc;
+    case 32: return GemmSmem<32, 8>::kAlloc;
+    case 64: return GemmSmem<64, 8>::kAlloc;
+    case 128: return GemmSmem<128, 4>::kAlloc;
+    case 256: return GemmSmem<256, 3>::kAlloc;
+  }
+  return 0;
 }
 
 template <int MODE>
@@ -684,7 +743,9 @@ HeadsWs heads_ws_layout(int B, int d, int V, int K, int kmax, medusa_dtype_t dt)
   if (dt == MEDUSA_BF16) {
     const size_t tph = (size_t)(V + kTileM - 1) / kTileM;
     w.y_bytes = align256((size_t)K * 2 * B * d * 2);
-    w.part_bytes = align256((size_t)B * K * tph * kmax * 4);
+    // candidate lists per row: one per tile, or one per CTA (running lists)
+    const size_t lists = tph > (size_t)num_sms() ? tph : (size_t)num_sms();
+    w.part_bytes = align256((size_t)B * K * lists * kmax * 4);
     // stream-K partials of the first GEMM: one [128][NB] fp32 slot and one
     // flag per CTA
     w.sk_part_bytes = align256((size_t)num_sms() * kTileM * round_nb(B) * 4);
@@ -784,10 +845,16 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
   p2.logits = logits;
   p2.part_vals = part_vals;
   p2.part_ids = part_ids;
+  // running lists when they fit: the merge then reads one list per CTA
+  // instead of one per tile
+  p2.run_lists = (K * B <= kRunMaxRows &&
+                  gemm_alloc_bytes(nb2) + (size_t)K * B * kRunRowBytes <= (size_t)kSmemLimit)
+                     ? 1
+                     : 0;
   st = launch_gemm_nb<kModeW2>(nb2, mA2, mB2, p2, stream);
   if (st != MEDUSA_OK) return st;
 
-  const long long C = (long long)p2.tiles_per_head * kmax;
+  const long long C = (long long)(p2.run_lists ? gemm_grid(p2) : p2.tiles_per_head) * kmax;
   const MergeLayout lay{C, C, (int)C, nullptr};
   launch(topk_merge_kernel, B * K * kMergeCtas, kMergeWarps * 32, 0, stream, part_vals, part_ids, C,
          kmax, topk_ids, topk_vals, lay);
