@@ -9,12 +9,17 @@
 //      sequence into Y [K, 2B, d] so that y enters the next GEMM at ~16-bit
 //      mantissa precision.
 //   2. W2 stage: Z = W2 * Y^T (rows = K*V tokens, columns = 2B); the epilogue
-//      adds the hi/lo columns, optionally stores the fp32 logits and keeps a
-//      per-warp top-kmax of every 32-row slice (warp bitonic sort).
-//   3. topk_merge: per (sequence, head), the best kmax of all slices.
+//      adds the hi/lo columns, optionally stores the fp32 logits, sorts every
+//      32-row slice (warp bitonic sort) and merges them into the tile's best
+//      list, which joins a running best list per (head, sequence) that the
+//      CTA keeps in shared memory across its tiles (one list per tile when
+//      those lists do not fit).  Tiles are handed out by an atomic counter.
+//   3. topk_merge: per (sequence, head), the best kmax of all the lists.
 // The weights are the only large operand (K*(d^2 + V*d) bf16): every CTA
 // streams 128-row weight tiles through a TMA -> shared memory -> tcgen05.mma
 // pipeline; the batch sits in the MMA's N dimension (weight rows fill M=128).
+// The first GEMM's few tiles are split evenly by k-blocks over the CTAs
+// (stream-K) when whole tiles would leave SMs idle.
 //
 // fp32 path (small shapes): warp-per-row CUDA-core dot products, same merge.
 #include <cuda.h>
