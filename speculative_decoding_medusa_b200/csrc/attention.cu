@@ -15,13 +15,15 @@
 //   warp 1      MMA issuer: S = Q K^T into TMEM (one S/P buffer per M tile),
 //               then O += P V with P as packed fp16 in TMEM (over the S
 //               columns) and V as an M/N-major shared-memory operand;
-//   warps 2..9  two softmax warpgroups, one query row per thread: the row's
-//               scores come out of TMEM, max and sum stay in the thread,
-//               O is rescaled in TMEM only when the row maximum grows by more
-//               than 2^8 (the stale maximum cancels in the final O / l);
-//   warps 10,11 V converters: each landed V tile is rewritten in place from
+//   warps 2,3   V converters: each landed V tile is rewritten in place from
 //               bf16 to fp16; for the tree tiles of query group 0 they first
-//               store the tree K/V into cache slots P + i.
+//               store the tree K/V into cache slots P + i;
+//   warps 4..11 two softmax warpgroups, one query row per thread, holding a
+//               whole 128-key tile of scores (warpgroup 0 gives up registers
+//               to them): the row's scores come out of TMEM, max and sum stay
+//               in the thread, O is rescaled in TMEM only when the row
+//               maximum grows by more than 2^8 (the stale maximum cancels in
+//               the final O / l).
 // Each piece of a range writes its normalised partial output and log2-sum-exp;
 // a combine kernel merges the pieces.
 //
@@ -43,7 +45,9 @@ constexpr int kAttnBN = 128;         // keys per tile (UMMA N of S = Q K^T)
 constexpr int kAttnMT = 128;         // query rows per M tile (UMMA M)
 constexpr int kAttnRows = 256;       // query rows per segment (two M tiles)
 constexpr int kAttnStages = 2;       // K/V ring depth (64 KB per stage)
-constexpr int kAttnThreads = 384;    // producer, MMA, two softmax warpgroups, two V converters
+constexpr int kAttnThreads = 384;    // producer, MMA, two V converters, two softmax warpgroups
+constexpr int kAttnRegsLow = 96;     // registers a thread in warpgroup 0
+constexpr int kAttnRegsHigh = 200;   // registers a thread in the softmax warpgroups
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold, log2 units
 constexpr uint32_t kAttnTmemCols = 512;
 constexpr int kAttnMaxB = 256;       // sequences per call (schedule table in shared memory)
@@ -54,6 +58,18 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Register budget of a warpgroup (all four warps execute it together).  The
+// shares must add up to no more than the registers the CTA was launched with
+// (threads x registers per thread), or the increase waits for ever.
+template <int N>
+__device__ __forceinline__ void warpgroup_regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void warpgroup_regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // 5-D tiled load (no multicast), c0 innermost
@@ -520,6 +536,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem_o = tmem_base;           // O[m]: columns m*DH .. m*DH+DH-1
   const uint32_t tmem_s = tmem_base + 2 * DH;  // S[m] then P[m]: 128 columns each
 
+  // Warpgroup 0 (producer, MMA issuer, V converters) needs few registers;
+  // the softmax warpgroups 1 and 2 hold a whole 128-key tile of scores.
+  // 128 x kAttnRegsLow + 256 x kAttnRegsHigh <= 384 x 168, the allocation of
+  // the launch (the kernel is built at 168 registers a thread).
+  static_assert(128 * kAttnRegsLow + 256 * kAttnRegsHigh <= kAttnThreads * 168,
+                "register split exceeds the launch's allocation");
+  if (warp < 4) {
+  warpgroup_regs_dec<kAttnRegsLow>();
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
@@ -669,14 +693,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int dummy_abort = 0;
       mbar_wait_bounded(drain, 0, &dummy_abort, p.status);
     }
-  } else if (warp >= 10) {
-    // ---------------- V converters (warps 10, 11) ----------------
+  } else {
+    // ---------------- V converters (warps 2, 3) ----------------
     // Each landed V tile is rewritten in place from bf16 to fp16 (the value
     // product runs on fp16 P and V); rows past the prefix end of a partial
     // tile are cleared (their weights are zero, but 0 * NaN is not).  A V
     // entry of magnitude 65536 or more, inf or NaN is reported as a
     // device-check error.
-    const int ct = (warp - 10) * 32 + lane;
+    const int ct = (warp - 2) * 32 + lane;
     bool range_ok = true;
     uint32_t copy_par = 0;  // bit s: parity of the copies made from stage s
     for (int j = 0; j < n; ++j) {
@@ -743,9 +767,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     if (ct == 0) bulk_wait_all();
     if (!range_ok) report(p.status, MEDUSA_ERR_DEVICE_CHECK);
+  }
   } else {
-    // ---------------- softmax warpgroups ----------------
-    const int m = (warp - 2) >> 2;
+    warpgroup_regs_inc<kAttnRegsHigh>();
+    // ---------------- softmax warpgroups (M tile 0: warps 4-7, 1: 8-11) ----------------
+    const int m = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int rl = quad * 32 + lane;  // row within the M tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
@@ -782,20 +808,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(&q_full[m]);
-    };
-    // 64 scores of half h of the tile, waited
-    auto load_half = [&](int h, float (&sv)[64]) {
-      uint32_t r0[32], r1[32];
-      tmem_ld32_raw(srow + h * 64, r0);
-      tmem_ld32_raw(srow + h * 64 + 32, r1);
-      tmem_ld_wait();
-      tmem_regs_after_wait(r0);
-      tmem_regs_after_wait(r1);
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        sv[c] = __uint_as_float(r0[c]);
-        sv[32 + c] = __uint_as_float(r1[c]);
-      }
     };
 
     int tcount = 0;
@@ -848,94 +860,93 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) tw[q] = upper ? mw[4 + q] : mw[q];
       }
-      // One pass over the tile, in two halves of 64 keys: the exponent base is
-      // the running maximum m_used (log2 units); a half whose maximum exceeds
-      // it by more than 2^8 (or the first half of a piece) moves the base,
-      // rescaling O, l and the half already written, so that every stored
-      // weight stays <= 2^8 (well inside fp16).
-      float sum_tile = 0.f;
-      bool moved = false;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float sv[64];
-        load_half(h, sv);
-        if (!full_tile) {
-          // visible keys of this half as a 64-bit mask: below the key end and
-          // set in the ancestor bitmask (the half's words are selected, not
-          // indexed, so the mask stays in registers)
-          const int nv = min(max(key_end - kbase - h * 64, 0), 64);
-          const uint64_t in_range = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
-          const uint32_t lo = h ? tw[2] : tw[0], hi = h ? tw[3] : tw[1];
-          const uint64_t vis = in_range & ((static_cast<uint64_t>(hi) << 32) | lo);
+      // One pass over the whole tile: all 128 scores of the row come out of
+      // TMEM with one wait.  The exponent base is the running maximum m_used
+      // (log2 units); a tile whose maximum exceeds it by more than 2^8 (or the
+      // first tile of a piece) moves the base and rescales O and l, so that
+      // every stored weight stays <= 2^8 (well inside fp16).
+      float sv[kAttnBN];
+      {
+        uint32_t r[4][32];
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (!((vis >> c) & 1ull)) sv[c] = -INFINITY;
+        for (int q = 0; q < 4; ++q) tmem_ld32_raw(srow + q * 32, r[q]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          tmem_regs_after_wait(r[q]);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) sv[q * 32 + c] = __uint_as_float(r[q][c]);
         }
-        // row maximum of the half: three-input max in four independent chains
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      }
+      if (!full_tile) {
+        // visible keys, 32 at a time: below the key end and set in the
+        // ancestor bitmask (the words are selected, not indexed, so the mask
+        // stays in registers)
+        const int nv = min(max(key_end - kbase, 0), kAttnBN);
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], sv[c], sv[c + 1]);
-        const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * p.scale_log2;
-        const bool need = (m_used == -INFINITY) ? (mx != -INFINITY) : (mx > m_used + kRescaleLog2);
-        if (__any_sync(0xffffffffu, need)) {
-          const float new_m = need ? mx : m_used;
-          const float corr = (need && m_used != -INFINITY) ? ex2_approx(m_used - new_m) : 1.f;
-          if (jj > 0) {
-            // O holds earlier tiles (their PV is done: this tile's QK was
-            // issued after it)
-#pragma unroll 1
-            for (int ch = 0; ch < DH / 32; ++ch) {
-              float o[32];
-              const uint32_t ta = tmem_o + lane_off + m * DH + ch * 32;
-              tmem_ld32(ta, o);
+        for (int q = 0; q < 4; ++q) {
+          const int nq = min(max(nv - q * 32, 0), 32);
+          const uint32_t vis = (nq >= 32 ? 0xffffffffu : ((1u << nq) - 1u)) & tw[q];
 #pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] *= corr;
-              tmem_st32(ta, o);
-            }
-          }
-          if (h == 1) {
-            // half 0 of this tile is already stored as fp16 pairs
-            uint32_t r0[32];
-            tmem_ld32_raw(srow, r0);
-            tmem_ld_wait();
-            tmem_regs_after_wait(r0);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r0[c]));
-              const __half2 h2 = __floats2half2_rn(f.x * corr, f.y * corr);
-              r0[c] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-            tmem_st32_u(srow, r0);
-          }
-          l_run *= corr;
-          sum_tile *= corr;
-          m_used = new_m;
-          moved = true;
+          for (int c = 0; c < 32; ++c)
+            if (!((vis >> c) & 1u)) sv[q * 32 + c] = -INFINITY;
         }
-        const float nbase = m_used == -INFINITY ? 0.f : -m_used;
-        // weights 2^(s * scale - m) on key pairs: the exponent argument and the
-        // running sums use the paired fp32 instructions; four partial sums
-        const uint64_t scale2 = f32x2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nbase2 = f32x2_pack(nbase, nbase);
-        uint64_t part[4] = {0ull, 0ull, 0ull, 0ull};
+      }
+      // row maximum: three-input max in four independent chains
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < kAttnBN; c += 2)
+        m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], sv[c], sv[c + 1]);
+      const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * p.scale_log2;
+      const bool need = (m_used == -INFINITY) ? (mx != -INFINITY) : (mx > m_used + kRescaleLog2);
+      if (__any_sync(0xffffffffu, need)) {
+        const float new_m = need ? mx : m_used;
+        const float corr = (need && m_used != -INFINITY) ? ex2_approx(m_used - new_m) : 1.f;
+        if (jj > 0) {
+          // O holds earlier tiles (their PV is done: this tile's QK was
+          // issued after it)
+#pragma unroll 1
+          for (int ch = 0; ch < DH / 32; ++ch) {
+            float o[32];
+            const uint32_t ta = tmem_o + lane_off + m * DH + ch * 32;
+            tmem_ld32(ta, o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] *= corr;
+            tmem_st32(ta, o);
+          }
+        }
+        l_run *= corr;
+        m_used = new_m;
+      }
+      // weights 2^(s * scale - m) on key pairs: the exponent argument and the
+      // running sums use the paired fp32 instructions; four partial sums.  P
+      // (packed fp16 pairs, 64 columns) overwrites the first half of S, which
+      // is already in registers.
+      const float nbase = m_used == -INFINITY ? 0.f : -m_used;
+      const uint64_t scale2 = f32x2_pack(p.scale_log2, p.scale_log2);
+      const uint64_t nbase2 = f32x2_pack(nbase, nbase);
+      uint64_t part[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int hq = 0; hq < 2; ++hq) {
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
+          const int c = hq * 64 + 2 * e;
           float x0, x1;
-          f32x2_unpack(f32x2_fma(f32x2_pack(sv[2 * e], sv[2 * e + 1]), scale2, nbase2), x0, x1);
+          f32x2_unpack(f32x2_fma(f32x2_pack(sv[c], sv[c + 1]), scale2, nbase2), x0, x1);
           const float a0 = ex2_approx(x0);
           const float a1 = ex2_approx(x1);
           part[e & 3] = f32x2_add(part[e & 3], f32x2_pack(a0, a1));
           const __half2 h2 = __floats2half2_rn(a0, a1);
           pk[e] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-        tmem_st32_u(srow + h * 32, pk);
+        tmem_st32_u(srow + hq * 32, pk);
+      }
+      {
         float s0, s1;
         f32x2_unpack(f32x2_add(f32x2_add(part[0], part[1]), f32x2_add(part[2], part[3])), s0, s1);
-        sum_tile += s0 + s1;
+        l_run += s0 + s1;
       }
-      (void)moved;
-      l_run += sum_tile;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[m]);
@@ -1852,6 +1863,20 @@ static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaSt
   if (cudaFuncSetAttribute(tree_attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            L::kAlloc) != cudaSuccess)
     return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(tree_attention) failed");
+  // the warpgroups' register shares must fit in what the launch allocates,
+  // or the softmax warpgroups' increase would wait for ever: checked against
+  // the registers the kernel was built with
+  {
+    static int regs = 0;
+    if (regs == 0) {
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, tree_attn_tc_kernel<DH>) != cudaSuccess)
+        return fail(MEDUSA_ERR_CUDA, "cudaFuncGetAttributes(tree_attention) failed");
+      regs = fa.numRegs;
+    }
+    if (128 * kAttnRegsLow + 256 * kAttnRegsHigh > kAttnThreads * regs)
+      return fail(MEDUSA_ERR_UNSUPPORTED, "tree_attention: register split exceeds the build's");
+  }
   p.grid = device_sm_count();  // persistent: one CTA per SM
   p.slot_mul = 1;
   launch(tree_attn_tc_kernel<DH>, p.grid, kAttnThreads, L::kAlloc, stream, mK, mV, mKn, mVn, mKs0,
