@@ -38,3 +38,16 @@ def test_planner_glossary_tree_and_errors():
     with pytest.raises(M.MedusaError) as e:
         M.medusa_tree_from_accuracies(acc * 2.0, 5, 2)
     assert e.value.status == 1
+
+
+def test_limits_tree_shape():
+    """The size-limit tree of the parity tests: the rank-0 chain reaches the
+    requested depth, ranks reach kmax - 1, every node's parent precedes it,
+    and nodes are in breadth-first order."""
+    spec = W.limits_tree(M.MAX_NODES, M.MAX_HEADS, M.MAX_KMAX)
+    assert spec.n_nodes == M.MAX_NODES
+    assert spec.max_depth == M.MAX_HEADS and spec.rank.max() == M.MAX_KMAX - 1
+    assert all(spec.parent[i] < i for i in range(1, spec.n_nodes))
+    assert list(spec.depth) == sorted(spec.depth)
+    chain = [i for i in range(spec.n_nodes) if all(r == 0 for r in spec.paths[i])]
+    assert len(chain) == M.MAX_HEADS + 1
