@@ -580,3 +580,28 @@ def test_sample_bonus_closed_forms():
     # different offsets give different draws
     us = {O.bonus_uniform(7, off, 0) for off in range(8)}
     assert len(us) == 8
+
+
+def test_bonus_uniform_literals():
+    """The uniform number of a sequence, pinned by literals.
+
+    Counter 0 and key 0 give the first word 0x6627E8D5 (known-answer vector
+    above), so the top 24 bits of word 0 give 0x6627E8 * 2^-24: taking
+    another word (0xE169C58D) or the low 24 bits (0x27E8D5) fails here.
+    The second literal is the generator's first word, 0xE1E5F2BB, for key
+    (0x89ABCDEF, 0x01234567) and counter (0x76543210, 0xFEDCBA98, 5, 0),
+    computed from the published round function by a separate C program; it
+    fixes the counter/key layout of seed, offset and sequence index."""
+    assert O.bonus_uniform(0, 0, 0) == 0x6627E8 * 2.0 ** -24
+    seed, offset, b = 0x0123456789ABCDEF, 0xFEDCBA9876543210, 5
+    assert O.bonus_uniform(seed, offset, b) == 0xE1E5F2 * 2.0 ** -24
+    # every plausible misreading of the layout gives another number
+    lo, hi = offset & 0xFFFFFFFF, offset >> 32
+    klo, khi = seed & 0xFFFFFFFF, seed >> 32
+    wrong = [
+        O.philox4x32_10([b, hi, lo, 0], [klo, khi])[0],     # offset and b swapped
+        O.philox4x32_10([hi, lo, b, 0], [klo, khi])[0],     # offset halves swapped
+        O.philox4x32_10([lo, hi, b, 0], [khi, klo])[0],     # key halves swapped
+        O.philox4x32_10([lo, hi, 0, b], [klo, khi])[0],     # b in the last word
+    ]
+    assert all((w >> 8) != 0xE1E5F2 for w in wrong)
