@@ -157,77 +157,141 @@ def _gpu_index(local_rank: int) -> str:
 # ---------------------------------------------------------------------------
 # CPU oracle on a bounded sample
 # ---------------------------------------------------------------------------
-def oracle_sample(w, n_nodes=None, seed=0):
-    """Time the CPU oracle on a bounded sample of one step and extrapolate to a
-    whole step.  Sample: head 0 on a 16384-token slice of its vocabulary for
-    every sequence (scaled by K * V / 16384); tree attention of 4 (sequence,
-    node) query rows with all heads (scaled by B*N/4); verification statistics
-    of 8 rows (scaled by B*N/8); tree build and KV compaction in full."""
-    from oracle import medusa_oracle as O
-    from speculative_decoding_medusa_b200 import workloads as W
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
-    N = n_nodes or w.N
-    spec = W.tree_for(w, n_nodes=N)
-    f64 = lambda t: t.to(torch.float64).numpy()
-    rows_v = min(16384, w.V)
-    h = f64(W.randn((w.B, w.d), seed, 1, 1.0, w.dtype))
-    W1 = f64(W.randn((1, w.d, w.d), seed, 2, 0.02, w.dtype))
-    b1 = f64(W.randn((1, w.d), seed, 3, 0.02, w.dtype))
-    W2 = f64(W.randn((1, rows_v, w.d), seed, 4, 0.02, w.dtype))
-    P = W.prefix_lengths(w, seed).numpy().astype(np.int64)
-    cap = w.ctx_hi + N
-    b0 = int(np.argmax(P))
-    q = f64(W.randn((1, N, w.Hq, w.dh), seed, 11, 1.0, w.dtype))
-    kn = f64(W.randn((1, N, w.Hkv, w.dh), seed, 12, 1.0, w.dtype))
-    vn = f64(W.randn((1, N, w.Hkv, w.dh), seed, 13, 1.0, w.dtype))
-    Kc = f64(W.randn((1, w.Hkv, cap, w.dh), seed, 14, 1.0, w.dtype))
-    Vc = f64(W.randn((1, w.Hkv, cap, w.dh), seed, 15, 1.0, w.dtype))
-    logits = f64(W.randn((1, 9, w.V), seed, 21, 1.0, w.dtype))
 
-    t = {}
-    t0 = time.perf_counter()
-    z = O.head_logits(h, W1, b1, W2)
-    O.topk(z, w.kmax)
-    t["heads"] = (time.perf_counter() - t0) * w.K * (w.V / rows_v)
-    t0 = time.perf_counter()
-    ids = np.zeros((w.B, w.K, w.kmax), dtype=np.int64)
-    tb = O.tree_build(spec.parent, spec.depth, spec.rank, np.zeros(w.B, np.int64), ids, P)
-    t["tree_build"] = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    # 4 query nodes (all heads) of the longest sequence: the oracle over a
-    # 4-node chain (root + 3 descendants) of that sequence
-    chain = [0]
-    while len(chain) < 4 and any(spec.parent[c] == chain[-1] for c in range(1, N)):
-        chain.append(next(c for c in range(1, N) if spec.parent[c] == chain[-1]))
-    mm = np.zeros((len(chain), 1), dtype=np.uint32)
-    for r in range(len(chain)):
-        mm[r, 0] = (1 << (r + 1)) - 1
-    O.tree_attention(q[:, chain], kn[:, chain], vn[:, chain], Kc, Vc, P[b0:b0 + 1], mm,
-                     1.0 / math.sqrt(w.dh))
-    t["attention"] = (time.perf_counter() - t0) * w.B * N / len(chain) * \
-        (float(np.mean(P)) + N / 2) / (float(P[b0]) + len(chain) / 2)
-    t0 = time.perf_counter()
-    O.row_argmax(logits[:, :8])
-    if w.accept == "typical":  # a 9-node chain: statistics of its first 8 rows
-        O.typical_log_margin(logits, np.zeros((1, 9), np.int64), np.arange(-1, 8),
-                             w.temperature, w.eps, w.delta)
-    t["verify"] = (time.perf_counter() - t0) * w.B * N / 8
-    t0 = time.perf_counter()
-    nodes = np.full((1, spec.max_depth + 1), -1, dtype=np.int64)
-    nodes[0, 0] = 0
-    O.kv_compact(Kc, Vc, P[b0:b0 + 1], nodes, np.array([0]))
-    t["kv_compact"] = (time.perf_counter() - t0) * w.B
-    sec = sum(t.values())
+def _oracle_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        return int(max([i.get("num_threads", 1) for i in threadpool_info()] + [1]))
     except Exception:
-        cores = os.cpu_count() or 1
-    sample = (f"head 0 on {rows_v} of {w.V} vocab rows x {w.B} sequences (x{w.K * w.V / rows_v:.1f}); "
-              f"{len(chain)} query nodes x {w.Hq} heads of one sequence (x{w.B * N / len(chain):.0f}, "
-              f"scaled by mean prefix); verify stats of 8 rows (x{w.B * N / 8:.0f}); tree build and "
-              f"compaction in full; fp64 numpy")
-    return {"seconds_per_step": sec, "stages": t, "cores": int(cores), "sample": sample}
+        return os.cpu_count() or 1
+
+
+class OracleSample:
+    """A bounded sample of one decode-verify step, run by the CPU oracle and
+    extrapolated to the whole step.
+
+    Sample (``frac`` = 1): head 0 on a 16384-token slice of its vocabulary for
+    every sequence (scaled by K * V / 16384); tree attention of 4 (sequence,
+    node) query rows with all heads (scaled by B*N/4 and the mean prefix);
+    verification statistics of 8 rows (scaled by B*N/8); tree build and KV
+    compaction in full.  ``frac`` < 1 shrinks the vocabulary slice (to at
+    least 256 tokens) so that long runs stay within a few minutes.  Inputs
+    are drawn once, outside the timed calls."""
+
+    def __init__(self, w, n_nodes=None, seed=0, frac=1.0):
+        from speculative_decoding_medusa_b200 import workloads as W
+
+        self.w = w
+        self.N = N = n_nodes or w.N
+        self.spec = spec = W.tree_for(w, n_nodes=N)
+        f64 = lambda t: t.to(torch.float64).numpy()
+        self.rows_v = min(w.V, max(256, int(16384 * frac)))
+        self.h = f64(W.randn((w.B, w.d), seed, 1, 1.0, w.dtype))
+        self.W1 = f64(W.randn((1, w.d, w.d), seed, 2, 0.02, w.dtype))
+        self.b1 = f64(W.randn((1, w.d), seed, 3, 0.02, w.dtype))
+        self.W2 = f64(W.randn((1, self.rows_v, w.d), seed, 4, 0.02, w.dtype))
+        self.P = W.prefix_lengths(w, seed).numpy().astype(np.int64)
+        cap = w.ctx_hi + N
+        self.b0 = int(np.argmax(self.P))
+        self.q = f64(W.randn((1, N, w.Hq, w.dh), seed, 11, 1.0, w.dtype))
+        self.kn = f64(W.randn((1, N, w.Hkv, w.dh), seed, 12, 1.0, w.dtype))
+        self.vn = f64(W.randn((1, N, w.Hkv, w.dh), seed, 13, 1.0, w.dtype))
+        self.Kc = f64(W.randn((1, w.Hkv, cap, w.dh), seed, 14, 1.0, w.dtype))
+        self.Vc = f64(W.randn((1, w.Hkv, cap, w.dh), seed, 15, 1.0, w.dtype))
+        self.logits = f64(W.randn((1, 9, w.V), seed, 21, 1.0, w.dtype))
+        # 4 query nodes (all heads) of the longest sequence: a 4-node chain
+        chain = [0]
+        while len(chain) < 4 and any(spec.parent[c] == chain[-1] for c in range(1, N)):
+            chain.append(next(c for c in range(1, N) if spec.parent[c] == chain[-1]))
+        self.chain = chain
+        self.mm = np.zeros((len(chain), 1), dtype=np.uint32)
+        for r in range(len(chain)):
+            self.mm[r, 0] = (1 << (r + 1)) - 1
+        B, K, V = w.B, w.K, w.V
+        self.scale = {
+            "heads": K * V / self.rows_v, "tree_build": 1.0,
+            "attention": B * N / len(chain) * (float(np.mean(self.P)) + N / 2)
+            / (float(self.P[self.b0]) + len(chain) / 2),
+            "verify": B * N / 8, "kv_compact": float(B)}
+
+    def run(self):
+        """Time the oracle on the sample once: (measured seconds, extrapolated
+        seconds of one whole step, extrapolated seconds per stage)."""
+        from oracle import medusa_oracle as O
+
+        w, spec, N = self.w, self.spec, self.N
+        t = {}
+        t0 = time.perf_counter()
+        z = O.head_logits(self.h, self.W1, self.b1, self.W2)
+        O.topk(z, w.kmax)
+        t["heads"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        ids = np.zeros((w.B, w.K, w.kmax), dtype=np.int64)
+        O.tree_build(spec.parent, spec.depth, spec.rank, np.zeros(w.B, np.int64), ids, self.P)
+        t["tree_build"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        b0, ch = self.b0, self.chain
+        O.tree_attention(self.q[:, ch], self.kn[:, ch], self.vn[:, ch], self.Kc, self.Vc,
+                         self.P[b0:b0 + 1], self.mm, 1.0 / math.sqrt(w.dh))
+        t["attention"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        O.row_argmax(self.logits[:, :8])
+        if w.accept == "typical":  # a 9-node chain: statistics of its first 8 rows
+            O.typical_log_margin(self.logits, np.zeros((1, 9), np.int64), np.arange(-1, 8),
+                                 w.temperature, w.eps, w.delta)
+        t["verify"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        nodes = np.full((1, spec.max_depth + 1), -1, dtype=np.int64)
+        nodes[0, 0] = 0
+        O.kv_compact(self.Kc, self.Vc, self.P[b0:b0 + 1], nodes, np.array([0]))
+        t["kv_compact"] = time.perf_counter() - t0
+        measured = sum(t.values())
+        stages = {k: v * self.scale[k] for k, v in t.items()}
+        return measured, sum(stages.values()), stages
+
+    def describe(self) -> str:
+        w = self.w
+        return (f"head 0 on {self.rows_v} of {w.V} vocab rows x {w.B} sequences "
+                f"(x{self.scale['heads']:.1f}); {len(self.chain)} query nodes x {w.Hq} heads of "
+                f"one sequence (x{w.B * self.N / len(self.chain):.0f}, scaled by mean prefix); "
+                f"verify stats of 8 rows (x{self.scale['verify']:.0f}); tree build and "
+                f"compaction in full; fp64 numpy")
+
+
+def oracle_sample(w, n_nodes=None, seed=0, frac=1.0):
+    """One timed oracle sample of a step: extrapolated seconds per step, the
+    measured seconds, stages, threads used and the sample's description."""
+    s = OracleSample(w, n_nodes, seed, frac)
+    measured, sec, stages = s.run()
+    return {"seconds_per_step": sec, "sample_s": measured, "stages": stages,
+            "cores": _oracle_threads(), "sample": s.describe(),
+            "scale": sec / measured if measured > 0 else None}
+
+
+def single_core_figures():
+    """Steps/s of the oracle on one host thread (Tiny and Vicuna-7B shapes,
+    bounded samples as above)."""
+    from threadpoolctl import threadpool_limits
+
+    from speculative_decoding_medusa_b200 import workloads as W
+    out = {}
+    with threadpool_limits(limits=1):
+        for name in ("tiny", "vicuna7b"):
+            r = oracle_sample(W.WORKLOADS[name])
+            out[name] = {"value": 1.0 / r["seconds_per_step"], "unit": UNIT, "cores": 1,
+                         "sample_s": r["sample_s"]}
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -409,29 +473,47 @@ def run_stage(args):
 
 
 def run_reference(args):
+    """The CPU oracle as the reference arm: warmup + steps timed samples of
+    the workload's step, each extrapolated to the whole step.  ms_per_step is
+    what was measured (oracle seconds of one sample); value is the
+    extrapolated whole-step rate; the sample is sized so the whole run takes
+    a few minutes at most."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from speculative_decoding_medusa_b200 import workloads as W
     w = workload_of(args, W)
     N = w.N
-    times = []
-    for i in range(args.warmup + args.steps):
-        r = oracle_sample(w, N, seed=i)
+    n_total = args.warmup + args.steps
+    # size the sample: one full sample first (untimed), then shrink the
+    # vocabulary slice so that all steps take about 120 s of oracle time
+    probe = OracleSample(w, N, seed=0)
+    t_full, _, _ = probe.run()
+    frac = min(1.0, 120.0 / max(n_total * t_full, 1e-9))
+    sample = OracleSample(w, N, seed=0, frac=frac) if frac < 1.0 else probe
+    measured, extrap = [], []
+    for i in range(n_total):
+        m, sec, _ = sample.run()
         if i >= args.warmup:
-            times.append(r["seconds_per_step"])
-        if sum(times) > 120:  # keep the whole run within a few minutes
-            break
-    sec = statistics.mean(times)
+            measured.append(m)
+            extrap.append(sec)
+    sec = statistics.mean(extrap)
     value = 1.0 / sec
+    sample_s = statistics.mean(measured)
+    cores = _oracle_threads()
     line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
-            "n_gpus": args.gpus, "steps": len(times), "warmup": args.warmup,
-            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "n_gpus": args.gpus, "steps": len(measured), "warmup": args.warmup,
+            "ms_per_step": sample_s * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "value_basis": "extrapolated: each timed step is a bounded sample of the step "
+                           "(ms_per_step = its measured oracle time), scaled to the whole step",
+            "sample_s": sample_s, "scale": sec / sample_s if sample_s > 0 else None,
+            "ms_per_step_extrapolated": sec * 1e3,
             "config": {"workload": args.workload, "global_batch": w.B, "n_nodes": N,
                        "prefix": [w.ctx_lo, w.ctx_hi], "parallelism": "none (CPU oracle)"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
-                             "sample": r["sample"]},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample.describe(), "cpu_model": _cpu_model(),
+                             "sample_s": sample_s},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
@@ -646,12 +728,25 @@ def main():
     traffic, traffic_src = heads_traffic(ab["heads"])
     step_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
     value = world * args.steps / (ms_total / 1e3)
+    # tree attention (attention kernel + combine): HBM and tensor rooflines
+    _, tc_peak, _ = _peaks()
+    attn_s = stages["tree_attention"] * 1e-6
+    attn_flops = 4.0 * w.Hq * w.dh * N * sum(P + N for P in prefix_list)
+    attention = {"us": stages["tree_attention"], "bytes": ab["attention"], "flops": attn_flops,
+                 "achieved_gbs": ab["attention"] / attn_s / 1e9,
+                 "frac_hbm": ab["attention"] / attn_s / 1e9 / hbm_peak,
+                 "achieved_tflops": attn_flops / attn_s / 1e12,
+                 "frac_tensor": attn_flops / attn_s / 1e12 / tc_peak,
+                 "peaks": f"{peak_kind} hbm_gbs {hbm_peak:.0f}, bf16_tflops {tc_peak:.0f} (burst)",
+                 "flops_def": "4 Hq dh N sum_b (P_b + N): QK and PV over prefix and tree tiles"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r = oracle_sample(w, N)
         cpu = {"value": 1.0 / r["seconds_per_step"], "unit": UNIT, "cores": r["cores"],
-               "kind": "oracle", "sample": r["sample"]}
+               "kind": "oracle", "sample": r["sample"], "sample_s": r["sample_s"],
+               "scale": r["scale"], "basis": "extrapolated from the timed sample",
+               "cpu_model": _cpu_model(), "single_core": single_core_figures()}
 
     if rank == 0:
         line = {
@@ -673,6 +768,7 @@ def main():
                          "frac": heads_gbs / hbm_peak, "traffic": traffic,
                          "traffic_source": "ncu dram bytes ratio, " + traffic_src,
                          "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": ab["heads"]},
+            "attention": attention,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": n_e2e,

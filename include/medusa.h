@@ -18,7 +18,8 @@
  * medusa_sample_bonus (a drawn bonus token), medusa_tree_from_accuracies
  * (the sparse tree of the most accurate combinations, host only), the
  * vocabulary-sharding calls (medusa_topk_merge, medusa_verify_records,
- * medusa_verify_from_records) and medusa_verify_accept_noalloc.
+ * medusa_verify_from_records), medusa_verify_accept_noalloc and
+ * medusa_wait_flag (a check of the bounded device waits).
  *
  * Sources (page title, then section):
  *   "Medusa Heads" glossary - "Comment les têtes prédisent les tokens
@@ -308,12 +309,16 @@ MEDUSA_API medusa_status_t medusa_kv_compact(void* Kc, void* Vc, medusa_dtype_t 
  * ws/ws_bytes: the row statistics go to a 4 MiB array compiled into the
  * library (every GPU that loads the library holds it until the process
  * exits).  Requests needing more, i.e. B * n_nodes * ceil(V / 4096) * 16 bytes
- * > 4 MiB, are rejected with MEDUSA_ERR_WORKSPACE before any launch.  Nothing
- * is allocated.  The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.  All calls share the one array and it keeps
- * the last call's contents: calls whose kernels overlap on the GPU (e.g. on
- * two streams at once) race and give wrong results.
+ * > 4 MiB, are rejected with MEDUSA_ERR_WORKSPACE before any launch, after
+ * the argument checks medusa_verify_accept makes (so a bad tree or shape gets
+ * the same error as there).  Nothing is allocated.  Every call looks up the
+ * array's device address (cudaGetSymbolAddress, a host-side query) with the
+ * caller's device and context current, so the address stays right after a
+ * device reset or in another context; the first call on a device may load
+ * the library's device code there, so make it before any stream capture.
+ * All calls share the one array and it keeps the last call's contents:
+ * calls whose kernels overlap on the GPU (e.g. on two streams at once) race
+ * and give wrong results.
  * ---------------------------------------------------------------------- */
 MEDUSA_API medusa_status_t medusa_verify_accept_noalloc(
     const void* logits, medusa_dtype_t dt, const int32_t* cand_ids, const medusa_tree_t* tree,
@@ -512,6 +517,30 @@ MEDUSA_API medusa_status_t medusa_tree_from_accuracies(const float* acc, int n_h
                                                        int32_t* parent, int32_t* depth,
                                                        int32_t* rank,
                                                        double* expected_accept_len);
+
+/* ------------------------------------------------------------------------
+ * medusa_wait_flag
+ *
+ * No counterpart on the pages: a check of this library's failure handling.
+ * Every wait inside the library's kernels (on a shared-memory barrier, or on
+ * a flag another block raises) is bounded: when it runs out it writes
+ * MEDUSA_ERR_TIMEOUT into *dev_status and the kernel returns, instead of
+ * holding the GPU.  This call runs that same bounded flag wait (the one the
+ * heads' first GEMM uses for its stream-K partials) in one thread on a
+ * caller's flag: it waits until *flag == value (acquire, device scope) or
+ * until budget_cycles SM clock cycles have passed, and in the second case
+ * writes MEDUSA_ERR_TIMEOUT into *dev_status.  The budget is checked every
+ * 64 polls of about 64 ns, so the wait lasts at least a few microseconds.
+ * budget_cycles <= 0 takes the library's own bound (2e9 cycles, one to two
+ * seconds).  A flag that nothing sets thus shows, on a given device and
+ * driver, that a stalled wait ends with a status the host can read and
+ * leaves the context usable.
+ * Inputs (device): flag, 4-byte aligned.  Output (device): dev_status.
+ * Errors: MEDUSA_ERR_SHAPE for budget_cycles above the library's bound.
+ * ---------------------------------------------------------------------- */
+MEDUSA_API medusa_status_t medusa_wait_flag(const int32_t* flag, int32_t value,
+                                            long long budget_cycles, int32_t* dev_status,
+                                            void* stream);
 
 #ifdef __cplusplus
 }

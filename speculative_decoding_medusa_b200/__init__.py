@@ -13,6 +13,6 @@ from ._lib import (  # noqa: F401
     medusa_verify_from_records, medusa_verify_records, medusa_verify_records_workspace_size,
     medusa_tree_attention, medusa_tree_attention_workspace_size,
     medusa_tree_build, medusa_verify_accept, medusa_verify_accept_noalloc,
-    medusa_verify_accept_workspace_size, new_status,
+    medusa_verify_accept_workspace_size, medusa_wait_flag, new_status,
     workspace,
 )

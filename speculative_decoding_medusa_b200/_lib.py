@@ -40,6 +40,7 @@ EXPORTS = (
     "medusa_lmhead_verify_workspace_size", "medusa_lmhead_verify", "medusa_next_step",
     "medusa_tree_from_accuracies", "medusa_sample_bonus", "medusa_topk_merge",
     "medusa_verify_records_workspace_size", "medusa_verify_records", "medusa_verify_from_records",
+    "medusa_wait_flag",
 )
 
 
@@ -115,6 +116,8 @@ def lib() -> ctypes.CDLL:
     L.medusa_tree_from_accuracies.argtypes = [_V, _I, _I, _I, _I, _V, _V, _V, _V]
     L.medusa_next_step.restype = _I
     L.medusa_next_step.argtypes = [_V, _I, _V, _V, _V, _I, _I, _I, _I, _V, _V, _V, _V]
+    L.medusa_wait_flag.restype = _I
+    L.medusa_wait_flag.argtypes = [_V, ctypes.c_int32, ctypes.c_longlong, _V, _V]
     L.medusa_lmhead_verify.restype = _I
     L.medusa_lmhead_verify.argtypes = [_V, _V, _I, _V, ctypes.POINTER(medusa_tree_t), _I, _I, _I,
                                        _I, _F, _F, _F, _V, _V, _V, _V, _V, _V, _Z, _V, _V]
@@ -406,3 +409,12 @@ def medusa_verify_from_records(records, cand_logit, cand_ids, tree: Tree, V: int
                                             float(eps), float(delta), _p(accept_len),
                                             _p(accepted_nodes), _p(accepted_tokens), _p(bonus),
                                             _p(dev_status), _stream(stream)))
+
+
+def medusa_wait_flag(flag, value: int, budget_cycles: int, dev_status, stream=None) -> None:
+    """Run the library's bounded flag wait on ``flag`` (device int32): returns
+    once *flag == value, or writes MEDUSA_ERR_TIMEOUT into dev_status after
+    budget_cycles SM clock cycles (<= 0: the library's own bound)."""
+    _req(flag, "flag")
+    _check(lib().medusa_wait_flag(_p(flag), int(value), int(budget_cycles), _p(dev_status),
+                                  _stream(stream)))

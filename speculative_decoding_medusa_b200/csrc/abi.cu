@@ -169,12 +169,18 @@ size_t medusa_verify_accept_workspace_size(int B, int N, int V) {
   return medusa::verify_accept_workspace_size(B, N, V);
 }
 
-medusa_status_t medusa_verify_accept(const void* logits, medusa_dtype_t dt,
-                                     const int32_t* cand_ids, const medusa_tree_t* tree, int B,
-                                     int V, medusa_accept_t mode, float temperature, float eps,
-                                     float delta, int32_t* accept_len, int32_t* accepted_nodes,
-                                     int32_t* accepted_tokens, int32_t* bonus, void* ws,
-                                     size_t ws_bytes, int32_t* dev_status, void* stream) {
+}  // extern "C"
+
+// Every check of medusa_verify_accept except the workspace's (shared with
+// medusa_verify_accept_noalloc, whose scratch limit is checked after these).
+medusa_status_t medusa::check_verify_accept_args(const void* logits, medusa_dtype_t dt,
+                                                 const int32_t* cand_ids,
+                                                 const medusa_tree_t* tree, int B, int V,
+                                                 medusa_accept_t mode, float temperature,
+                                                 float eps, float delta, const int32_t* accept_len,
+                                                 const int32_t* accepted_nodes,
+                                                 const int32_t* accepted_tokens,
+                                                 const int32_t* bonus) {
   medusa_status_t st = check_tree(tree);
   if (st != MEDUSA_OK) return st;
   if (!logits || !cand_ids || !accept_len || !accepted_nodes || !accepted_tokens || !bonus)
@@ -187,6 +193,21 @@ medusa_status_t medusa_verify_accept(const void* logits, medusa_dtype_t dt,
   if (mode == MEDUSA_ACCEPT_TYPICAL && (!(temperature > 0.f) || !(eps >= 0.f) || !(delta >= 0.f)))
     return fail(MEDUSA_ERR_INVALID_ARG, "verify_accept: need temperature > 0, eps >= 0, delta >= 0");
   if (!aligned16(logits)) return fail(MEDUSA_ERR_ALIGNMENT, "verify_accept: logits not 16-byte aligned");
+  return MEDUSA_OK;
+}
+
+extern "C" {
+
+medusa_status_t medusa_verify_accept(const void* logits, medusa_dtype_t dt,
+                                     const int32_t* cand_ids, const medusa_tree_t* tree, int B,
+                                     int V, medusa_accept_t mode, float temperature, float eps,
+                                     float delta, int32_t* accept_len, int32_t* accepted_nodes,
+                                     int32_t* accepted_tokens, int32_t* bonus, void* ws,
+                                     size_t ws_bytes, int32_t* dev_status, void* stream) {
+  medusa_status_t st = medusa::check_verify_accept_args(logits, dt, cand_ids, tree, B, V, mode,
+                                                        temperature, eps, delta, accept_len,
+                                                        accepted_nodes, accepted_tokens, bonus);
+  if (st != MEDUSA_OK) return st;
   const size_t need = medusa::verify_accept_workspace_size(B, tree->n_nodes, V);
   if (ws == nullptr || ws_bytes < need || !aligned256(ws))
     return fail(MEDUSA_ERR_WORKSPACE, "verify_accept: workspace null, misaligned or too small");

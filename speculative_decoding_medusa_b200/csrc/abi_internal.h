@@ -19,6 +19,14 @@ medusa_status_t check_launch(const char* what);
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// the argument checks of medusa_verify_accept, all but the workspace's
+medusa_status_t check_verify_accept_args(const void* logits, medusa_dtype_t dt,
+                                         const int32_t* cand_ids, const medusa_tree_t* tree,
+                                         int B, int V, medusa_accept_t mode, float temperature,
+                                         float eps, float delta, const int32_t* accept_len,
+                                         const int32_t* accepted_nodes,
+                                         const int32_t* accepted_tokens, const int32_t* bonus);
+
 // bf16 tensor of `rank` dims (dims[0] contiguous; byte_strides[i] is the
 // stride of dims[i+1]), tile `box`, 128-byte swizzle, zero fill outside
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,

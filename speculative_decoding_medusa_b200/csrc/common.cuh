@@ -127,6 +127,39 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 // ----------------------------------------------------------------------------
+// flags in global memory that one CTA raises and another waits on
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Wait until *flag == value (acquire).  Gives up (false) when *abort is
+// raised or `budget` clock cycles have passed; on running out it raises
+// *abort and reports MEDUSA_ERR_TIMEOUT.
+__device__ __forceinline__ bool wait_flag_bounded(const int* flag, int value,
+                                                  volatile int* abort, int32_t* status,
+                                                  long long budget) {
+  if (ld_acquire_gpu(flag) == value) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) == value) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort) return false;
+      if (clock64() - t0 > budget) {
+        *abort = 1;
+        report(status, MEDUSA_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
 // TMA (bulk tensor copies, no multicast)
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -183,35 +183,6 @@ __host__ __device__ constexpr uint32_t tmem_cols() {
   return (2 * NB) < 32 ? 32u : static_cast<uint32_t>(2 * NB);
 }
 
-// release / acquire of a flag another CTA waits on
-__device__ __forceinline__ void st_release_gpu(int* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-// Wait until *flag == 1; gives up (false) when *abort is raised or the spin
-// budget runs out, reporting MEDUSA_ERR_TIMEOUT in that case.
-__device__ __forceinline__ bool wait_flag_bounded(const int* flag, volatile int* abort,
-                                                  int32_t* status) {
-  if (ld_acquire_gpu(flag) == 1) return true;
-  const long long t0 = clock64();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(64);
-    if (ld_acquire_gpu(flag) == 1) return true;
-    if ((it & 63u) == 0u) {
-      if (*abort) return false;
-      if (clock64() - t0 > kSpinBudgetCycles) {
-        *abort = 1;
-        report(status, MEDUSA_ERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
 template <int NB, int S, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     heads_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -410,7 +381,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         c_last = ((tile + 1) * nkb - 1) / p.kpc;
         bool ready = true;
         for (int c = blockIdx.x + 1; ready && c <= c_last; ++c)
-          ready = wait_flag_bounded(&p.sk_flag[c], abort_flag, p.status);
+          ready = wait_flag_bounded(&p.sk_flag[c], 1, abort_flag, p.status, kSpinBudgetCycles);
         if (!ready) break;
       }
 #pragma unroll 1

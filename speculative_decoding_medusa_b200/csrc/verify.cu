@@ -17,7 +17,6 @@
 #include <math.h>
 #include <stdint.h>
 
-#include <atomic>
 #include <type_traits>
 
 #include "abi_internal.h"
@@ -726,9 +725,6 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) unsigned char g_verify_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kNoAllocMaxDevices = 64;
-std::atomic<void*> g_verify_noalloc_ptr[kNoAllocMaxDevices];
-
 }  // namespace
 
 extern "C" medusa_status_t medusa_verify_accept_noalloc(
@@ -736,29 +732,27 @@ extern "C" medusa_status_t medusa_verify_accept_noalloc(
     int B, int V, medusa_accept_t mode, float temperature, float eps, float delta,
     int32_t* accept_len, int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
     int32_t* dev_status, void* stream) {
-  if (tree == nullptr)
-    return medusa::fail(MEDUSA_ERR_INVALID_ARG, "verify_accept_noalloc: null tree");
-  if (B >= 1 && V >= 1 && tree->n_nodes >= 1 &&
-      medusa::verify_accept_workspace_size(B, tree->n_nodes, V) > kNoAllocScratchBytes)
+  // the checks of medusa_verify_accept first, so that a bad tree or shape
+  // gets the same error here as there; then the scratch limit
+  medusa_status_t st = medusa::check_verify_accept_args(logits, dt, cand_ids, tree, B, V, mode,
+                                                        temperature, eps, delta, accept_len,
+                                                        accepted_nodes, accepted_tokens, bonus);
+  if (st != MEDUSA_OK) return st;
+  if (medusa::verify_accept_workspace_size(B, tree->n_nodes, V) > kNoAllocScratchBytes)
     return medusa::fail(MEDUSA_ERR_WORKSPACE,
                         "verify_accept_noalloc: B * n_nodes * ceil(V / 4096) * 16 bytes exceeds "
                         "the 4 MiB static scratch; use medusa_verify_accept with a workspace");
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
-    return medusa::fail(MEDUSA_ERR_CUDA, "verify_accept_noalloc: cudaGetDevice failed");
-  if (dev >= kNoAllocMaxDevices)
-    return medusa::fail(MEDUSA_ERR_UNSUPPORTED, "verify_accept_noalloc: device index >= 64");
-  // host code sees only a stand-in for the device array: its device address
-  // is looked up once per device, with that device current
-  void* scratch = g_verify_noalloc_ptr[dev].load(std::memory_order_acquire);
-  if (scratch == nullptr) {
-    const cudaError_t e = cudaGetSymbolAddress(&scratch, g_verify_noalloc_scratch);
-    if (e != cudaSuccess || scratch == nullptr) {
-      cudaGetLastError();
-      return medusa::fail(MEDUSA_ERR_CUDA,
-                          "verify_accept_noalloc: cudaGetSymbolAddress of the scratch failed");
-    }
-    g_verify_noalloc_ptr[dev].store(scratch, std::memory_order_release);
+  // Host code sees only a stand-in for the device array.  Its device address
+  // is looked up on every call, with the caller's device and context current:
+  // the lookup is a host-side query (no synchronisation), and an address kept
+  // from an earlier call could belong to a module that a device reset or
+  // another context has since replaced.
+  void* scratch = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&scratch, g_verify_noalloc_scratch);
+  if (e != cudaSuccess || scratch == nullptr) {
+    cudaGetLastError();
+    return medusa::fail(MEDUSA_ERR_CUDA,
+                        "verify_accept_noalloc: cudaGetSymbolAddress of the scratch failed");
   }
   // every row record is written by the row kernel before the path kernel
   // reads it, so the scratch needs no clearing between calls

@@ -7,9 +7,14 @@ row records and merges them; this module only moves those few kilobytes
 between ranks (one all-gather each, plus a max all-reduce of the candidate
 logits for typical acceptance).  No collective touches the weights or the
 logits, and no device buffer of another GPU is read by a kernel.
+
+The exchanges run on the stream the library calls were enqueued on.  Over
+NCCL they stay on the device; over gloo (host collectives) the few KB go
+through host memory.
 """
 from __future__ import annotations
 
+import contextlib
 from typing import List, Tuple
 
 import torch
@@ -30,18 +35,45 @@ def shard_offsets(V: int, world: int) -> List[int]:
     return [shard_range(V, world, r)[0] for r in range(world)]
 
 
+def _host_staged(t: torch.Tensor, group) -> bool:
+    """A device tensor exchanged over a backend without device collectives
+    (gloo gathers host tensors only) goes through host memory."""
+    return t.is_cuda and dist.get_backend(group) != "nccl"
+
+
 def gather_stacked(t: torch.Tensor, group=None) -> torch.Tensor:
-    """[world, *t.shape]: every rank's ``t`` in rank order (all-gather)."""
+    """[world, *t.shape]: every rank's ``t`` in rank order (all-gather).
+
+    Runs on the current stream: NCCL orders the collective after the work
+    already queued there; a host-staged exchange copies ``t`` to the host
+    with a copy that waits for that work."""
     world = dist.get_world_size(group)
+    if _host_staged(t, group):
+        h = t.to("cpu")
+        parts = [torch.empty_like(h) for _ in range(world)]
+        dist.all_gather(parts, h.contiguous(), group=group)
+        return torch.stack(parts).to(t.device)
     parts = [torch.empty_like(t) for _ in range(world)]
     dist.all_gather(parts, t.contiguous(), group=group)
     return torch.stack(parts)
 
 
 def max_over_ranks(t: torch.Tensor, group=None) -> torch.Tensor:
-    """Element-wise maximum over the ranks, in place."""
+    """Element-wise maximum over the ranks, in place (current stream)."""
+    if _host_staged(t, group):
+        h = t.to("cpu")
+        dist.all_reduce(h, op=dist.ReduceOp.MAX, group=group)
+        t.copy_(h)
+        return t
     dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
     return t
+
+
+def _on(stream):
+    """Context making ``stream`` (if given) torch's current stream, so that
+    the exchange is ordered after the library calls enqueued on it and the
+    calls after the exchange are ordered after it."""
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
 
 
 class ShardedHeads:
@@ -71,8 +103,9 @@ class ShardedHeads:
     def run(self, h, W1, b1, W2_shard, stream=None):
         M.medusa_heads_topk(h, W1, b1, W2_shard, self.kmax, self.local_ids, self.local_vals, None,
                             self.ws, self.status, stream)
-        vals = gather_stacked(self.local_vals, self.group)
-        ids = gather_stacked(self.local_ids, self.group)
+        with _on(stream):
+            vals = gather_stacked(self.local_vals, self.group)
+            ids = gather_stacked(self.local_ids, self.group)
         rows = self.B * self.K
         M.medusa_topk_merge(vals, ids, rows, self.world, self.kmax, self.kmax,
                             rows * self.kmax, self.offsets, self.kmax, self.topk_ids,
@@ -111,9 +144,10 @@ class ShardedVerify:
         M.medusa_verify_records(logits_shard, cand_ids, self.tree, self.v0, self.records,
                                 self.cand_logit, self.mode, self.temperature, self.ws,
                                 self.status, stream)
-        records = gather_stacked(self.records, self.group)
-        if self.mode == M.MEDUSA_ACCEPT_TYPICAL:
-            max_over_ranks(self.cand_logit, self.group)
+        with _on(stream):
+            records = gather_stacked(self.records, self.group)
+            if self.mode == M.MEDUSA_ACCEPT_TYPICAL:
+                max_over_ranks(self.cand_logit, self.group)
         M.medusa_verify_from_records(records, self.cand_logit, cand_ids, self.tree, self.V,
                                      self.accept_len, self.accepted_nodes, self.accepted_tokens,
                                      self.bonus, self.mode, self.temperature, self.eps,

@@ -118,6 +118,23 @@ def test_attention_verify_compact_checks(L):
     assert verify(logits=v(1032)) == 8
     assert verify(ws=None) == 7
 
+    # the workspace-free variant: same argument checks first, then its 4 MiB
+    # limit of B * n_nodes * ceil(V / 4096) 16-byte records, before any launch
+    tree128 = _lib.medusa_tree_t(128, 4, 64, 1024, 1024, 1024)
+
+    def noalloc(B=64, V=131073, logits=v(1024), t=tree128):
+        return L.medusa_verify_accept_noalloc(logits, 0, v(1024), ctypes.byref(t), B, V, 0, 1.0,
+                                              0.09, 0.3, v(1024), v(1024), v(1024), v(1024), None,
+                                              None)
+
+    assert noalloc() == 7                          # 64 x 128 x 33 = 270336 records
+    assert b"4 MiB" in L.medusa_last_error()
+    assert noalloc(V=131072) != 7                  # 64 x 128 x 32 = 262144: exactly fits
+    assert noalloc(B=1024) == 2                    # B * n_nodes > 65535, as medusa_verify_accept
+    assert noalloc(logits=None) == 1
+    assert noalloc(logits=v(1032)) == 8
+    assert noalloc(t=_lib.medusa_tree_t(300, 4, 64, 1024, 1024, 1024)) == 2
+
     def compact(max_depth=4, dh=128, Kc=v(1024)):
         return L.medusa_kv_compact(Kc, v(1024), 0, v(1024), v(1024), v(1024), 1, 2, dh, 100,
                                    max_depth, v(1024), None, None)
@@ -126,6 +143,14 @@ def test_attention_verify_compact_checks(L):
     assert compact(max_depth=16) == 2
     assert compact(dh=4) == 2                     # 8-byte rows are not 16-byte multiples
     assert compact(Kc=v(1032)) == 8
+
+    def wait(flag=v(1024), budget=1000, status=v(2048)):
+        return L.medusa_wait_flag(flag, 1, budget, status, None)
+
+    assert wait(flag=None) == 1
+    assert wait(status=None) == 1
+    assert wait(flag=v(1026)) == 8
+    assert wait(budget=2000000001) == 2           # above the library's own bound
 
 
 def test_workspace_queries(L):

@@ -59,8 +59,9 @@ def _assert_same(got, ref):
 
 def _check_logits(got, z):
     """The GEMM's fp32 logits against the fp64 oracle, and its argmax (taken
-    by the kernel on those fp32 values) against the oracle's: equal, or a
-    near-tie within the logit tolerance."""
+    by the kernel on those fp32 values) against the oracle's: the same token
+    on every row whose oracle top-2 gap exceeds twice the logit tolerance,
+    a near-tie within that tolerance elsewhere."""
     zg = got["logits"]
     assert np.abs(zg - z).max() < LOGIT_ABS
     g_gpu = np.argmax(zg, axis=-1)
@@ -68,7 +69,33 @@ def _check_logits(got, z):
     zmax = z.max(axis=-1)
     z_at = np.take_along_axis(z, g_gpu[..., None], axis=-1)[..., 0]
     assert (z_at >= zmax - 2 * LOGIT_ABS).all()
-    assert (g_gpu == g_ora).mean() > 0.98
+    top2 = np.sort(z, axis=-1)[..., -2:]
+    clear = top2[..., 1] - top2[..., 0] > 2 * LOGIT_ABS
+    np.testing.assert_array_equal(g_gpu[clear], g_ora[clear])
+
+
+def _without_near_ties(hidden, lm, z, seed):
+    """Redraw, from N(0, 1), the hidden state of every tree node whose oracle
+    top-2 logit gap is at most twice the logit tolerance, until no such node
+    is left (a planted node's top token stands about 8 above the rest, so
+    only unplanted nodes are redrawn).  The argmax of every row is then
+    unambiguous at the kernel's fp32 accuracy, and the acceptance from the
+    hidden states can be compared with the oracle's unconditionally.
+    Returns the new hidden states and their oracle logits."""
+    gen = torch.Generator().manual_seed(104729 + seed)
+    hidden = hidden.clone()
+    z = z.copy()
+    lmd = f64(lm)
+    d = hidden.shape[-1]
+    for _ in range(20):
+        top2 = np.sort(z, axis=-1)[..., -2:]
+        bad = np.argwhere(top2[..., 1] - top2[..., 0] <= 2 * LOGIT_ABS)
+        if len(bad) == 0:
+            return hidden, z
+        for b, i in bad:
+            hidden[b, i] = torch.randn(d, generator=gen).to(hidden.dtype)
+            z[b, i] = O.lm_head_logits(f64(hidden[b, i])[None], lmd)[0]
+    raise AssertionError("rows with a near-tie argmax remain after 20 redraws")
 
 
 @pytest.mark.parametrize("B,n_nodes,V,d,seed", [
@@ -83,19 +110,16 @@ def test_logits_and_greedy_decisions(B, n_nodes, V, d, seed):
     spec = W.tree_for(w)
     cand = _cands(w, spec, seed)
     hidden, lm = W.lmhead_inputs(w, spec, torch.from_numpy(cand), seed=seed)
-    z = _oracle_logits(hidden, lm)
+    hidden, z = _without_near_ties(hidden, lm, _oracle_logits(hidden, lm), seed)
     got = _run(hidden, lm, cand, spec, M.MEDUSA_ACCEPT_GREEDY, want_logits=True)
     _check_logits(got, z)
     # acceptance: bit-exact on the kernel's own logits ...
     ref = O.verify_greedy(got["logits"], cand, spec.parent, spec.depth, spec.max_depth)
     _assert_same(got, ref)
-    # ... and equal to the oracle's from the hidden states whenever no row
-    # has a near-tie argmax
-    top2 = np.sort(z, axis=-1)[..., -2:]
-    if (top2[..., 1] - top2[..., 0]).min() > 2 * LOGIT_ABS:
-        ref2 = O.lmhead_verify(f64(hidden), f64(lm), cand, spec.parent, spec.depth,
-                               spec.max_depth)
-        _assert_same(got, ref2)
+    # ... and equal to the oracle's from the hidden states (every argmax is
+    # unambiguous after the redraw)
+    ref2 = O.lmhead_verify(f64(hidden), f64(lm), cand, spec.parent, spec.depth, spec.max_depth)
+    _assert_same(got, ref2)
 
 
 @pytest.mark.parametrize("B,V,d,seed", [(2, 4000, 512, 4), (3, 1300, 1024, 5)])
@@ -107,7 +131,7 @@ def test_typical_decisions(B, V, d, seed):
     for attempt in range(20):
         hidden, lm = W.lmhead_inputs(w, spec, torch.from_numpy(cand), seed=seed, attempt=attempt,
                                      plant=4.0)
-        z = _oracle_logits(hidden, lm)
+        hidden, z = _without_near_ties(hidden, lm, _oracle_logits(hidden, lm), seed + attempt)
         m = O.typical_log_margin(z, cand, spec.parent, w.temperature, w.eps, w.delta)
         if np.abs(m[:, 1:]).min() > TYPICAL_LOG_MARGIN:
             break
@@ -121,7 +145,7 @@ def test_typical_decisions(B, V, d, seed):
     _assert_same(got, ref)
     ref2 = O.lmhead_verify(f64(hidden), f64(lm), cand, spec.parent, spec.depth, spec.max_depth,
                            "typical", w.temperature, w.eps, w.delta)
-    np.testing.assert_array_equal(got["accepted_nodes"], ref2["accepted_nodes"])
+    _assert_same(got, ref2)
     assert 0 < ref["accept_len"].sum()
 
 
@@ -180,12 +204,15 @@ def test_full_size_greedy_llama3_8b():
     spec = W.tree_for(w)
     cand = _cands(w, spec, 0)
     hidden, lm = W.lmhead_inputs(w, spec, torch.from_numpy(cand), seed=0, device="cuda")
-    got = _run(hidden, lm, cand, spec, M.MEDUSA_ACCEPT_GREEDY, want_logits=True)
     h = f64(hidden.cpu()).reshape(-1, w.d)
     z = np.empty((h.shape[0], w.V))
     for v0 in range(0, w.V, 8192):
         z[:, v0:v0 + 8192] = O.lm_head_logits(h, f64(lm[v0:v0 + 8192].cpu()))
     z = z.reshape(w.B, spec.n_nodes, w.V)
+    hidden, z = _without_near_ties(hidden.cpu(), lm.cpu(), z, 0)
+    got = _run(hidden, lm, cand, spec, M.MEDUSA_ACCEPT_GREEDY, want_logits=True)
     _check_logits(got, z)
     ref = O.verify_greedy(got["logits"], cand, spec.parent, spec.depth, spec.max_depth)
     _assert_same(got, ref)
+    ref2 = O.verify_greedy(z, cand, spec.parent, spec.depth, spec.max_depth)
+    _assert_same(got, ref2)

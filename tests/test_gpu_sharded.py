@@ -1,6 +1,7 @@
 """GPU: vocabulary-sharded heads and verification, the G shards computed one
 after another on one GPU and stacked as an all-gather would, against the
-unsharded calls (same kernels, same per-token arithmetic)."""
+oracle and against the unsharded calls (same kernels, same per-token
+arithmetic)."""
 import numpy as np
 import pytest
 import torch
@@ -9,7 +10,8 @@ import speculative_decoding_medusa_b200 as M
 from oracle import medusa_oracle as O
 from speculative_decoding_medusa_b200 import sharded as S
 from speculative_decoding_medusa_b200 import workloads as W
-from tests.helpers import TYPICAL_LOG_MARGIN, f64, i64
+from tests.helpers import (TYPICAL_LOG_MARGIN, check_topk, f64, i64,
+                           oracle_head_logits_chunked)
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +50,12 @@ def test_sharded_heads_equal_unsharded(G, V):
     M.medusa_topk_merge(gv, gi, rows, G, w.kmax, w.kmax, rows * w.kmax, offs, w.kmax, out_i,
                         out_v)
     torch.cuda.synchronize()
+    # the merged shard lists against the oracle's logits of the whole
+    # vocabulary ...
+    z = oracle_head_logits_chunked(inp["h"].cpu(), inp["W1"].cpu(), inp["b1"].cpu(),
+                                   inp["W2"].cpu())
+    check_topk(out_i.cpu().numpy(), out_v.cpu().numpy(), z, w.kmax)
+    # ... and equal to the unsharded call bit for bit
     assert torch.equal(out_i, ids)
     assert torch.equal(out_v, vals)
 
@@ -110,7 +118,8 @@ def test_sharded_greedy_equals_unsharded(G, V, dtype):
     for a, b in zip(got, ref):
         np.testing.assert_array_equal(a, b)
     oracle = O.verify_greedy(f64(logits.cpu()), cand, spec.parent, spec.depth, spec.max_depth)
-    np.testing.assert_array_equal(got[0], oracle["accept_len"])
+    for k, a in zip(("accept_len", "accepted_nodes", "accepted_tokens", "bonus"), got):
+        np.testing.assert_array_equal(a, oracle[k], err_msg=k)
 
 
 @pytest.mark.parametrize("G,V", [(2, 6000), (4, 30000)])
