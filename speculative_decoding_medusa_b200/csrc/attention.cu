@@ -24,8 +24,12 @@
 //               in the thread, O is rescaled in TMEM only when the row
 //               maximum grows by more than 2^8 (the stale maximum cancels in
 //               the final O / l).
-// Each piece of a range writes its normalised partial output and log2-sum-exp;
-// a combine kernel merges the pieces.
+// A piece that covers a whole segment writes its output rows directly.  Any
+// other piece writes its normalised partial output and log2-sum-exp, then
+// counts itself in a per-row counter; the row's last piece to arrive merges
+// all of the row's partials (log-sum-exp weights) and writes the output row,
+// so no separate merge pass follows the kernel.  The counters are zeroed by a
+// small kernel before each launch.
 //
 // fp32 path: one warp per query row on CUDA cores (small shapes).
 #include <cuda_bf16.h>
@@ -33,8 +37,6 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
-#include <stdlib.h>
-#include <string.h>
 
 #include "abi_internal.h"
 #include "common.cuh"
@@ -130,152 +132,6 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// ----------------------------------------------------------------------------
-// CTA pairs (cluster of two, tcgen05 cta_group::2)
-// ----------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// shared::cluster address of this shared-memory location in CTA `rank`
-__device__ __forceinline__ uint32_t cluster_addr(const void* ptr, uint32_t rank) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(ptr)), "r"(rank));
-  return a;
-}
-// arrive on a barrier of CTA 0 of the pair: a plain local arrive in CTA 0, an
-// arrive through the cluster window (given by its shared::cluster address)
-// in CTA 1.  What it publishes is ordered by the caller's tcgen05 or proxy
-// fence, so the arrive keeps the default (CTA-scope release) semantics.
-__device__ __forceinline__ void mbar_arrive_cta0(uint64_t* bar, uint32_t caddr, uint32_t rank) {
-  if (rank == 0) {
-    mbar_arrive(bar);
-  } else {
-    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
-  }
-}
-__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// bounded wait on a barrier that the peer CTA also arrives on (acquire at
-// cluster scope); same give-up rules as mbar_wait_bounded
-__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                             int32_t* status) {
-  if (mbar_try_wait_cl(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cl(bar, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (*abort) return false;
-      if (clock64() - t0 > kSpinBudgetCycles) {
-        *abort = 1;
-        report(status, MEDUSA_ERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-// 16 consecutive 32-bit columns of this thread's lane
-__device__ __forceinline__ void tmem_st16_u(uint32_t taddr, const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-      "r"(v[15])
-      : "memory");
-}
-// every thread of both CTAs
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(dst_smem)),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem] over the pair: M = 256 rows, CTA r holding
-// rows 128r.. of A and D in its tensor memory and half of B's N columns in
-// its shared memory (same addresses in both CTAs).  Issued by CTA 0.
-__device__ __forceinline__ void umma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// same with A from shared memory (each CTA's 128 rows of A in its own)
-__device__ __forceinline__ void umma_pair_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// the barrier at this shared-memory offset in both CTAs gets one arrival once
-// every pair MMA issued so far has completed
-__device__ __forceinline__ void umma_pair_commit_both(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(smem_u32(bar)),
-      "h"(static_cast<uint16_t>(3))
-      : "memory");
-}
-// tiled loads into this CTA's shared memory whose completion is counted on a
-// barrier of either CTA of the pair (given by its shared::cluster address);
-// no multicast
-__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map,
-                                                 uint32_t bar_caddr, int c0, int c1, int c2,
-                                                 uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar_caddr),
-      "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_5d_pair(void* dst, const CUtensorMap* map,
-                                                 uint32_t bar_caddr, int c0, int c1, int c2,
-                                                 int c3, int c4) {
-  asm volatile(
-      "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
-      "r"(bar_caddr)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map,
-                                                 uint32_t bar_caddr, int c0, int c1, int c2,
-                                                 int c3, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar_caddr),
-      "l"(policy)
-      : "memory");
-}
-
 struct AttnParams {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k_new;
@@ -286,10 +142,11 @@ struct AttnParams {
   const uint32_t* anc_mask;
   float* o_part;    // [n_seg, slots, DH / 4, 256] groups of 4 floats
   float* lse_part;  // [n_seg, slots, 256]
+  unsigned int* row_count;  // [n_seg, 256] pieces of the row written so far (zeroed per call)
+  void* out;        // [B, N, Hq, DH], bf16 or fp32
+  int out_f32;
   int B, N, Hq, Hkv, G, R, n_qg, T_tree, slots, cap, max_prefix, words, grid;
   int q_tma;  // Q tiles by bulk tensor loads (G divides 128)
-  int copy_tree;  // the combine kernel stores the tree K/V into the caches
-  int slot_mul;   // partial results per piece (one per softmax stream)
   float scale_log2;
   int32_t* status;
 };
@@ -452,6 +309,123 @@ __device__ __forceinline__ bool build_schedule(const AttnParams& p, int* cumT, i
 __device__ __forceinline__ int tiles_per_cta(int total, int grid) {
   const int per = (total + grid - 1) / grid;
   return per < kAttnMinTiles ? kAttnMinTiles : per;
+}
+
+// 32 output values of query row r (within the segment's query rows) from
+// column c0: row r is query head kvh * G + g of node r / G
+struct OutRow {
+  void* out;
+  int out_f32, N, Hq, G;
+};
+
+template <int DH>
+__device__ __forceinline__ void store_out_row32(const OutRow& q, int b, int kvh, int r, int c0,
+                                                const float (&v)[32]) {
+  const int node = r / q.G, g = r - node * q.G;
+  const size_t base = (((size_t)b * q.N + node) * q.Hq + kvh * q.G + g) * DH + c0;
+  if (q.out_f32) {
+    float4* o = reinterpret_cast<float4*>(static_cast<float*>(q.out) + base);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) o[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  } else {
+    uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(q.out) + base);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * c + 2 * q], v[8 * c + 2 * q + 1]);
+        w[q] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      o[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+// The merge of a query row's pieces by the last one to arrive: weights
+// 2^(lse_k - max lse), the partials (normalised O of each key range) summed
+// with them and divided by the weights' sum.  The partials of other CTAs are
+// read past L1 (they were released by a fence before their row count).
+template <int DH>
+__device__ __noinline__ void merge_row(const float* o_part, const float* lse_part, OutRow q,
+                                       int b, int kvh, int r, size_t pbase, int row,
+                                       unsigned int n_pieces) {
+  constexpr int kFast = 4;  // pieces whose loads are all in flight together
+  const float4* src0 = reinterpret_cast<const float4*>(o_part) + pbase * kAttnRows * (DH / 4) + row;
+  const size_t piece_stride = (size_t)kAttnRows * (DH / 4);
+  if (n_pieces <= kFast) {
+    float lse[kFast];
+#pragma unroll
+    for (int k = 0; k < kFast; ++k)
+      lse[k] = k < (int)n_pieces ? __ldcg(lse_part + (pbase + k) * kAttnRows + row) : -INFINITY;
+    const float M = fmaxf(fmaxf(lse[0], lse[1]), fmaxf(lse[2], lse[3]));
+    float w[kFast], wsum = 0.f;
+#pragma unroll
+    for (int k = 0; k < kFast; ++k) {
+      w[k] = lse[k] == -INFINITY ? 0.f : exp2f(lse[k] - M);
+      wsum += w[k];
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+    for (int k = 0; k < kFast; ++k) w[k] *= inv;
+#pragma unroll 1
+    for (int ch = 0; ch < DH / 32; ++ch) {
+      float4 v[kFast][8];
+#pragma unroll
+      for (int k = 0; k < kFast; ++k)
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          v[k][c] = k < (int)n_pieces ? __ldcg(src0 + k * piece_stride + (ch * 8 + c) * kAttnRows)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      float acc[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        acc[4 * c] = w[0] * v[0][c].x + w[1] * v[1][c].x + w[2] * v[2][c].x + w[3] * v[3][c].x;
+        acc[4 * c + 1] = w[0] * v[0][c].y + w[1] * v[1][c].y + w[2] * v[2][c].y + w[3] * v[3][c].y;
+        acc[4 * c + 2] = w[0] * v[0][c].z + w[1] * v[1][c].z + w[2] * v[2][c].z + w[3] * v[3][c].z;
+        acc[4 * c + 3] = w[0] * v[0][c].w + w[1] * v[1][c].w + w[2] * v[2][c].w + w[3] * v[3][c].w;
+      }
+      store_out_row32<DH>(q, b, kvh, r, ch * 32, acc);
+    }
+    return;
+  }
+  float M = -INFINITY;
+  for (unsigned int k = 0; k < n_pieces; ++k)
+    M = fmaxf(M, __ldcg(lse_part + (pbase + k) * kAttnRows + row));
+  float wsum = 0.f;
+  for (unsigned int k = 0; k < n_pieces; ++k) {
+    const float lse = __ldcg(lse_part + (pbase + k) * kAttnRows + row);
+    wsum += lse == -INFINITY ? 0.f : exp2f(lse - M);
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll 1
+  for (int ch = 0; ch < DH / 32; ++ch) {
+    float acc[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+    for (unsigned int k = 0; k < n_pieces; ++k) {
+      const float lse = __ldcg(lse_part + (pbase + k) * kAttnRows + row);
+      const float w = lse == -INFINITY ? 0.f : exp2f(lse - M) * inv;
+      const float4* src = src0 + k * piece_stride;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 v = __ldcg(src + (ch * 8 + c) * kAttnRows);
+        acc[4 * c] += w * v.x;
+        acc[4 * c + 1] += w * v.y;
+        acc[4 * c + 2] += w * v.z;
+        acc[4 * c + 3] += w * v.w;
+      }
+    }
+    store_out_row32<DH>(q, b, kvh, r, ch * 32, acc);
+  }
+}
+
+// Row counters of the in-kernel merge, zeroed before every attention launch.
+__global__ void attn_zero_kernel(unsigned int* __restrict__ cnt, size_t n) {
+  grid_dep_wait();
+  grid_dep_launch();
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    cnt[i] = 0u;
 }
 
 template <int DH>
@@ -816,6 +790,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float m_used = -INFINITY, l_run = 0.f;
     uint32_t mw[8];
     int jj = 0;
+    int piece_lt0 = 0;  // the segment tile the current piece starts at
+    const OutRow out_row{p.out, p.out_f32, p.N, p.Hq, p.G};
     TileCursor cur;
     cur.init(t0, t0, t1, per, cumT, pref, p);
     for (int j = 0; ok && j < n; ++j, cur.advance()) {
@@ -833,6 +809,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         m_used = -INFINITY;
         l_run = 0.f;
         jj = 0;
+        piece_lt0 = x.lt;
       }
       if (!mbar_wait_bounded(&s_full[m], tcount & 1, abort_flag, p.status)) {
         ok = false;
@@ -951,31 +928,59 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       mbar_arrive(&p_full[m]);
       if (x.last) {
-        // the piece ends: wait for its last PV, then write the partial
+        // the piece ends: wait for its last PV
         if (!mbar_wait_bounded(&p_empty[m], tcount & 1, abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const size_t piece = (size_t)x.seg * p.slots + x.slot;
-        const size_t prow = piece * kAttnRows + m * kAttnMT + rl;
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        // column-group-major partial: a warp's 32 rows of one group of 4
-        // columns are 512 contiguous bytes
-        float4* dst = reinterpret_cast<float4*>(p.o_part) + piece * kAttnRows * (DH / 4) +
-                      m * kAttnMT + rl;
+        if (piece_lt0 == 0 && x.lt == x.ntiles - 1) {
+          // the piece is the whole segment: O / l is the row's output
 #pragma unroll 1
-        for (int ch = 0; ch < DH / 32; ++ch) {
-          float o[32];
-          tmem_ld32(tmem_o + lane_off + m * DH + ch * 32, o);
-          if (valid) {
+          for (int ch = 0; ch < DH / 32; ++ch) {
+            float o[32];
+            tmem_ld32(tmem_o + lane_off + m * DH + ch * 32, o);
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              dst[(ch * 8 + c) * kAttnRows] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv,
-                                                          o[4 * c + 2] * inv, o[4 * c + 3] * inv);
+            for (int c = 0; c < 32; ++c) o[c] *= inv;
+            if (valid) store_out_row32<DH>(out_row, x.b, x.kvh, r, ch * 32, o);
+          }
+        } else {
+          // a normalised partial O and its log2-sum-exp; the row's last piece
+          // to arrive (counted per row) merges all of them
+          const size_t pbase = (size_t)x.seg * p.slots;
+          const size_t piece = pbase + x.slot;
+          // column-group-major partial: a warp's 32 rows of one group of 4
+          // columns are 512 contiguous bytes
+          float4* dst = reinterpret_cast<float4*>(p.o_part) + piece * kAttnRows * (DH / 4) +
+                        m * kAttnMT + rl;
+#pragma unroll 1
+          for (int ch = 0; ch < DH / 32; ++ch) {
+            float o[32];
+            tmem_ld32(tmem_o + lane_off + m * DH + ch * 32, o);
+            if (valid) {
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                dst[(ch * 8 + c) * kAttnRows] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv,
+                                                            o[4 * c + 2] * inv, o[4 * c + 3] * inv);
+            }
+          }
+          if (valid) {
+            const int row = m * kAttnMT + rl;
+            p.lse_part[piece * kAttnRows + row] = l_run > 0.f ? m_used + log2f(l_run) : -INFINITY;
+            const int seg_t0 = t0 + j - x.lt;  // the segment's first tile (global index)
+            const unsigned int n_pieces =
+                static_cast<unsigned int>((seg_t0 + x.ntiles - 1) / per - seg_t0 / per + 1);
+            // release this piece, count it; the counter wraps to 0 at the last
+            __threadfence();
+            const unsigned int before =
+                atomicInc(&p.row_count[(size_t)x.seg * kAttnRows + row], n_pieces - 1);
+            if (before == n_pieces - 1) {
+              __threadfence();
+              merge_row<DH>(p.o_part, p.lse_part, out_row, x.b, x.kvh, r, pbase, row, n_pieces);
+            }
           }
         }
-        if (valid) p.lse_part[prow] = l_run > 0.f ? m_used + log2f(l_run) : -INFINITY;
         tc_fence_before();
       }
       ++tcount;
@@ -988,675 +993,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kAttnTmemCols);
-  }
-}
-
-// ----------------------------------------------------------------------------
-// Pair kernel (dh = 128, G dividing 128): a cluster of two CTAs runs the 256
-// query rows of a segment as one M = 256 tile of cta_group::2 MMAs.  CTA r
-// holds M tile r (its 128 rows of Q in shared memory; S, P and O in its own
-// tensor memory) and half of every K/V tile: keys 64r..64r+63 of K (the N
-// half of S = Q K^T) and head dims 64r..64r+63 of V (the N half of O = P V).
-// So each CTA loads, converts and feeds to the tensor core half a tile per
-// step.  S is double-buffered (QK of tile j+1 runs while the softmax works on
-// tile j), Q is double-buffered (the next piece's Q arrives by TMA while the
-// current piece runs) and so is O (a finished piece is read out while the
-// next one accumulates).  Tensor memory per CTA: O buffers [0,128) and
-// [128,256), S/P buffers [256,384) and [384,512).
-// ----------------------------------------------------------------------------
-constexpr int kPairStages = 4;     // K/V ring depth (32 KB per stage and CTA)
-constexpr int kPairThreads = 384;  // producer, MMA, 8 softmax warps, two V converters
-
-struct PairSmem {
-  static constexpr int DH = 128;
-  static constexpr int kKPanel = 64 * 128;           // 64 keys x 64 dims (128 B rows)
-  static constexpr int kKHalf = 2 * kKPanel;         // 64 keys x 128 dims
-  static constexpr int kVHalf = kAttnBN * 128;       // 128 keys x 64 dims
-  static constexpr int kQPanel = kAttnMT * 128;      // 128 rows x 64 dims
-  static constexpr int kQBytes = 2 * kQPanel;        // one M tile of Q
-  static constexpr int kQOff = 0;                    // Q buffers [2]
-  static constexpr int kKOff = kQOff + 2 * kQBytes;
-  static constexpr int kVOff = kKOff + kPairStages * kKHalf;
-  static constexpr int kBarOff = kVOff + kPairStages * kVHalf;
-  // k_full[S], v_land[S], v_ready[S], kv_empty[S], q_full[2], q_empty[2],
-  // s_full[2], p_full[2], p_empty[2], o_free[2], drain
-  static constexpr int kNumBars = 4 * kPairStages + 11;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kInfoOff = kMiscOff + 16;                   // int info[S]
-  static constexpr int kCumOff = (kInfoOff + 4 * kPairStages + 15) / 16 * 16;  // int cumT[kAttnMaxB + 1]
-  static constexpr int kPrefOff = kCumOff + (kAttnMaxB + 1) * 4;   // int P[kAttnMaxB]
-  static constexpr int kBytes = kPrefOff + kAttnMaxB * 4;
-  static constexpr int kAlloc = kBytes + 1024;
-  static_assert(kKOff % 1024 == 0 && kVOff % 1024 == 0, "swizzled tiles need 1024-B alignment");
-};
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
-    tree_attn_pair_kernel(const __grid_constant__ CUtensorMap tmKh,
-                          const __grid_constant__ CUtensorMap tmV,
-                          const __grid_constant__ CUtensorMap tmKnh,
-                          const __grid_constant__ CUtensorMap tmVn,
-                          const __grid_constant__ CUtensorMap tmQ, AttnParams p) {
-  grid_dep_wait();
-  grid_dep_launch();
-  constexpr int DH = PairSmem::DH;
-  using L = PairSmem;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  int* cumT = reinterpret_cast<int*>(smem + L::kCumOff);
-  int* pref = reinterpret_cast<int*>(smem + L::kPrefOff);
-  volatile int* sched_ok = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
-  if (warp == 0) {
-    const bool ok = build_schedule(p, cumT, pref);
-    if (lane == 0) *sched_ok = ok ? 1 : 0;
-  }
-  __syncthreads();
-  // both CTAs of a pair read the same prefix lengths, so they take the same
-  // early exits
-  if (!*sched_ok) {
-    if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, MEDUSA_ERR_DEVICE_CHECK);
-    return;
-  }
-  const int total = cumT[p.B];
-  const int pair = static_cast<int>(blockIdx.x >> 1);
-  const int per = tiles_per_cta(total, p.grid);
-  const int t0 = pair * per;
-  const int t1 = min(t0 + per, total);
-  if (t0 >= total) return;
-  const int n = t1 - t0;
-
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* k_full = bars;                        // [S] (CTA 0's): both K halves landed
-  uint64_t* v_land = bars + kPairStages;          // [S] this CTA's V half landed
-  uint64_t* v_ready = bars + 2 * kPairStages;     // [S] (CTA 0's): both V halves in fp16
-  uint64_t* kv_empty = bars + 3 * kPairStages;    // [S] the stage's MMAs are done
-  uint64_t* q_full = bars + 4 * kPairStages;      // [2] (CTA 0's): both Q tiles landed
-  uint64_t* q_empty = q_full + 2;                 // [2] the piece's last QK is done
-  uint64_t* s_full = q_empty + 2;                 // [2]
-  uint64_t* p_full = s_full + 2;                  // [2] (CTA 0's): both P tiles in TMEM
-  uint64_t* p_empty = p_full + 2;                 // [2] the PV that read P is done
-  uint64_t* o_free = p_empty + 2;                 // [2] (CTA 0's): O buffer read out
-  uint64_t* drain = o_free + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
-  int* stage_info = reinterpret_cast<int*>(smem + L::kInfoOff);
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kPairStages; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&v_land[i], 1);
-      mbar_init(&v_ready[i], 2 * 64);
-      mbar_init(&kv_empty[i], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&q_full[b], 1);
-      mbar_init(&q_empty[b], 1);
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 2 * 128);
-      mbar_init(&p_empty[b], 1);
-      mbar_init(&o_free[b], 2 * 128);
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(tmem_holder, kAttnTmemCols);
-    tmem_relinquish_pair();
-  }
-  // barriers initialised and tensor memory allocated in both CTAs before
-  // either touches the other's
-  tc_fence_before();
-  cluster_sync_all();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_holder;
-  const uint32_t tmem_o = tmem_base;                 // O buffer ob at + ob * 128
-  const uint32_t tmem_s = tmem_base + 2 * DH;        // S/P buffer b at + b * 128
-
-  if (warp == 0) {
-    // ---------------- TMA producer (this CTA's Q tile and K/V halves) ----------------
-    if (lane == 0) {
-      tma_prefetch_desc(&tmKh);
-      tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmKnh);
-      tma_prefetch_desc(&tmVn);
-      tma_prefetch_desc(&tmQ);
-      // each K/V byte is read by one CTA only, so it need not stay in L2
-      // unless other query groups read it again
-      const uint64_t pol = p.n_qg > 1 ? l2_policy_evict_last() : l2_policy_evict_first();
-      const uint32_t kfull0 = cluster_addr(&k_full[0], 0);  // CTA 0's k_full[0]
-      const uint32_t qfull0 = cluster_addr(&q_full[0], 0);
-      const int kr = static_cast<int>(rank) * 64;           // this CTA's keys of K, dims of V
-      TileCursor cur;
-      cur.init(t0, t0, t1, per, cumT, pref, p);
-      int j = 0, pieces = 0;
-      for (; j < n; ++j, cur.advance()) {
-        const TileInfo& x = cur.x;
-        const int st = j % kPairStages;
-        if (x.first) {
-          // the piece's Q tile (rows 128r.. of its query group, node-major
-          // (node, g) pairs) into Q buffer pieces % 2, once the piece that
-          // used that buffer before has issued its last QK
-          const int qb = pieces & 1;
-          if (!mbar_wait_bounded(&q_empty[qb], ((pieces >> 1) & 1) ^ 1u, abort_flag, p.status))
-            break;
-          if (rank == 0) mbar_arrive_expect_tx(&q_full[qb], 2 * L::kQBytes);
-          const int node0 = (x.qg * kAttnRows + static_cast<int>(rank) * kAttnMT) / p.G;
-          uint8_t* qdst = smem + L::kQOff + qb * L::kQBytes;
-#pragma unroll
-          for (int pn = 0; pn < 2; ++pn)
-            tma_load_5d_pair(qdst + pn * L::kQPanel, &tmQ, qfull0 + qb * 8, pn * 64, 0, x.kvh,
-                             node0, x.b);
-          ++pieces;
-        }
-        if (!mbar_wait_bounded(&kv_empty[st], ((j / kPairStages) & 1) ^ 1u, abort_flag, p.status))
-          break;
-        // published with the stage: the converters (and in CTA 0 the MMA
-        // thread) read it instead of walking the schedule
-        stage_info[st] = pack_stage_info(x);
-        if (rank == 0) mbar_arrive_expect_tx(&k_full[st], 2 * L::kKHalf);
-        mbar_arrive_expect_tx(&v_land[st], L::kVHalf);
-        uint8_t* kdst = smem + L::kKOff + st * L::kKHalf;
-        uint8_t* vdst = smem + L::kVOff + st * L::kVHalf;
-        const int bh = x.b * p.Hkv + x.kvh;
-        const uint32_t kbar = kfull0 + st * 8;
-        if (x.lt < x.tpre) {
-          const int key = x.lt * kAttnBN;
-#pragma unroll
-          for (int pn = 0; pn < 2; ++pn)
-            tma_load_3d_pair(kdst + pn * L::kKPanel, &tmKh, kbar, pn * 64, key + kr, bh, pol);
-          tma_load_3d(vdst, &tmV, &v_land[st], kr, key, bh, pol);
-        } else {
-          const int node = (x.lt - x.tpre) * kAttnBN;
-#pragma unroll
-          for (int pn = 0; pn < 2; ++pn)
-            tma_load_4d_pair(kdst + pn * L::kKPanel, &tmKnh, kbar, pn * 64, x.kvh, node + kr, x.b,
-                             pol);
-          tma_load_4d(vdst, &tmVn, &v_land[st], kr, x.kvh, node, x.b, pol);
-        }
-      }
-      // before the CTA leaves: its loads have landed (they may still be in
-      // flight after an abort) and the MMA thread has released every stage
-      // (the releases are arrivals on this CTA's barriers)
-      const int first = j > kPairStages ? j - kPairStages : 0;
-      for (int t = first; t < j; ++t) {
-        int dummy_abort = 0;
-        const int st = t % kPairStages;
-        const uint32_t ph = (t / kPairStages) & 1;
-        mbar_wait_bounded(&v_land[st], ph, &dummy_abort, p.status);
-        if (rank == 0) mbar_wait_cl(&k_full[st], ph, &dummy_abort, p.status);
-        mbar_wait_bounded(&kv_empty[st], ph, abort_flag, p.status);
-      }
-      for (int k = pieces > 2 ? pieces - 2 : 0; k < pieces; ++k) {
-        int dummy_abort = 0;
-        if (rank == 0) mbar_wait_cl(&q_full[k & 1], (k >> 1) & 1, &dummy_abort, p.status);
-        mbar_wait_bounded(&q_empty[k & 1], (k >> 1) & 1, abort_flag, p.status);
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (CTA 0 only) ----------------
-    // Per tile j: QK(j+1) into the other S buffer as soon as its K halves
-    // (and, for a piece's first tile, its Q tiles) have landed, then PV(j)
-    // once both CTAs' P(j) and V halves are ready.  QK(j+1) overwrites the
-    // buffer PV(j-1) read; both come from this thread, so the tensor core
-    // runs them in that order.
-    if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc_qk = umma_idesc_bf16(2 * kAttnMT, kAttnBN, 0);
-      constexpr uint32_t idesc_pv = umma_idesc_f16(2 * kAttnMT, DH, 1);
-      // shared-memory descriptors built once; advancing one only adds to its
-      // start-address field (16-byte units)
-      const uint64_t dq0 = umma_desc_sw128(smem_u32(smem + L::kQOff));
-      const uint64_t dk0 = umma_desc_sw128(smem_u32(smem + L::kKOff));
-      const uint64_t dv0 = umma_desc_sw128_lbo(smem_u32(smem + L::kVOff), L::kVHalf, 1024);
-      // S[b] = Q K^T: A = this CTA's 128 Q rows, B = its 64 keys, both
-      // K-major with two 64-dim panels
-      auto issue_qk = [&](int b, int st, int qb) {
-        const uint64_t dq = dq0 + (uint64_t)((qb * L::kQBytes) >> 4);
-        const uint64_t dk = dk0 + (uint64_t)((st * L::kKHalf) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk)
-          umma_pair_ss(tmem_s + b * kAttnBN,
-                       dq + (uint64_t)((kk >> 2) * (L::kQPanel >> 4) + (kk & 3) * 2),
-                       dk + (uint64_t)((kk >> 2) * (L::kKPanel >> 4) + (kk & 3) * 2), idesc_qk,
-                       kk > 0 ? 1u : 0u);
-        umma_pair_commit_both(&s_full[b]);
-      };
-      // O[ob] (+)= P[b] V (stream b = j & 1 owns S/P buffer b and O buffer b):
-      // A = P (packed fp16 pairs, 16 keys = 8 columns per
-      // step), B = this CTA's 64 dims of V (fp16 after conversion),
-      // M/N-major, 16 keys = two 8-row groups of 1024 B
-      auto issue_pv = [&](int b, int st, int ob, uint32_t acc0) {
-        const uint64_t dv = dv0 + (uint64_t)((st * L::kVHalf) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < kAttnBN / 16; ++kk)
-          umma_pair_ts(tmem_o + ob * DH, tmem_s + b * kAttnBN + kk * 8,
-                       dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
-        umma_pair_commit_both(&p_empty[b]);
-        umma_pair_commit_both(&kv_empty[st]);
-      };
-      uint32_t nq = 0;            // pieces whose Q was awaited (their QKs issued)
-      uint32_t npc0 = 0, npc1 = 0;  // pieces each stream has started accumulating
-      int qb = 0;                 // Q buffer of the piece being multiplied
-      bool prev_first = false;    // tile j-1 started a piece
-      bool ok = n > 0 && mbar_wait_cl(&k_full[0], 0, abort_flag, p.status);
-      int cur = ok ? stage_info[0] : 0;
-      if (ok) ok = mbar_wait_cl(&q_full[0], 0, abort_flag, p.status);
-      if (ok) {
-        nq = 1;
-        tc_fence_after();
-        issue_qk(0, 0, 0);
-        if (info_last(cur)) umma_pair_commit_both(&q_empty[0]);
-      }
-      for (int j = 0; ok && j < n; ++j) {
-        const int st = j % kPairStages;
-        const int b = j & 1;
-        int nxt = 0;
-        if (j + 1 < n) {
-          const int sn = (j + 1) % kPairStages;
-          if (!mbar_wait_cl(&k_full[sn], ((j + 1) / kPairStages) & 1, abort_flag, p.status)) break;
-          nxt = stage_info[sn];
-          if (info_first(nxt)) {
-            qb = nq & 1;
-            if (!mbar_wait_cl(&q_full[qb], (nq >> 1) & 1, abort_flag, p.status)) break;
-            ++nq;
-          }
-          tc_fence_after();
-          issue_qk(b ^ 1, sn, qb);
-          // the piece's last QK frees its Q buffer for the piece after next
-          if (info_last(nxt)) umma_pair_commit_both(&q_empty[qb]);
-        }
-        if (!mbar_wait_cl(&v_ready[st], (j / kPairStages) & 1, abort_flag, p.status) ||
-            !mbar_wait_cl(&p_full[b], (j >> 1) & 1, abort_flag, p.status))
-          break;
-        // stream b's first tile of a piece starts its O over, once the
-        // stream's previous piece has been read out of it
-        const bool sfirst = info_first(cur) || prev_first;
-        if (sfirst) {
-          const uint32_t k = b ? npc1 : npc0;
-          if (k >= 1 && !mbar_wait_cl(&o_free[b], (k - 1) & 1, abort_flag, p.status)) break;
-          if (b) ++npc1;
-          else ++npc0;
-        }
-        tc_fence_after();
-        issue_pv(b, st, b, sfirst ? 0u : 1u);
-        prev_first = info_first(cur);
-        cur = nxt;
-      }
-      umma_pair_commit_both(drain);
-    }
-    // every MMA (and so every arrival it makes on this CTA's barriers) is
-    // done before the CTA leaves
-    if (lane == 0) {
-      int dummy_abort = 0;
-      mbar_wait_bounded(drain, 0, &dummy_abort, p.status);
-    }
-  } else if (warp >= 10) {
-    // ---------------- V converters (warps 10, 11) ----------------
-    // This CTA's V half (128 keys x 64 dims) is rewritten in place from bf16
-    // to fp16; rows past the prefix end of a partial tile are cleared (their
-    // weights are zero, but 0 * NaN is not).  |v| >= 65536, inf or NaN is
-    // reported as a device-check error.
-    const int ct = (warp - 10) * 32 + lane;
-    const uint32_t vready0 = cluster_addr(&v_ready[0], 0);
-    bool range_ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int st = j % kPairStages;
-      if (!mbar_wait_bounded(&v_land[st], (j / kPairStages) & 1, abort_flag, p.status)) break;
-      const int zero_from = info_zero_from(stage_info[st]);
-      uint4* vt = reinterpret_cast<uint4*>(smem + L::kVOff + st * L::kVHalf);
-      constexpr int kChunks = L::kVHalf / 16;  // 8 chunks of 16 B per key row
-      constexpr int kUnroll = 8;
-      static_assert(kChunks % (64 * kUnroll) == 0, "V half must split evenly over the converters");
-      uint32_t vmax = 0u;
-#pragma unroll 1
-      for (int e0 = ct; e0 < kChunks; e0 += 64 * kUnroll) {
-        uint4 v[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) v[u] = vt[e0 + u * 64];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int row = (e0 + u * 64) >> 3;
-          uint32_t* w = &v[u].x;
-          const bool keep = row < zero_from;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (keep) vmax = __vmaxu2(vmax, w[q] & 0x7FFF7FFFu);
-            const __half2 h2 = __floats2half2_rn(__uint_as_float(w[q] << 16),
-                                                 __uint_as_float(w[q] & 0xffff0000u));
-            w[q] = keep ? *reinterpret_cast<const uint32_t*>(&h2) : 0u;
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) vt[e0 + u * 64] = v[u];
-      }
-      if (__vcmpgtu2(vmax, 0x477F477Fu)) range_ok = false;
-      fence_proxy_async_smem();
-      mbar_arrive_cta0(&v_ready[st], vready0 + st * 8, rank);
-    }
-    if (!range_ok) report(p.status, MEDUSA_ERR_DEVICE_CHECK);
-  } else {
-    // ---------------- softmax: two streams of one thread per row ----------------
-    // Stream s (warps 2..5: s = 0, warps 6..9: s = 1) takes the tiles j with
-    // j % 2 == s, which use S/P buffer s, and accumulates them into O buffer
-    // s with its own running maximum and sum.  The streams never wait for
-    // each other: their tiles' QKs finish one tile apart, so one stream
-    // computes exponentials while the other loads scores.  Each stream
-    // writes its own partial result of a piece (slot 2 * slot + s); the
-    // combine kernel merges them like any two pieces.
-    const int sm = (warp - 2) >> 2;   // stream
-    const int quad = warp & 3;
-    const int rl = quad * 32 + lane;  // row within this CTA's M tile = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t srow = tmem_s + sm * kAttnBN + lane_off;
-    const uint32_t orow = tmem_o + sm * DH + lane_off;
-    const uint32_t pfull0 = cluster_addr(&p_full[sm], 0);
-    const uint32_t ofree0 = cluster_addr(&o_free[sm], 0);
-
-    bool ok = true;
-    float m_used = -INFINITY, l_run = 0.f;
-    uint32_t mw[8];
-    int jj = 0;                // this stream's tiles of the current piece so far
-    bool prev_first = sm == 1;  // tile j-1 started a piece (tile 0 always does)
-    TileCursor cur;
-    cur.init(t0 + sm, t0, t1, per, cumT, pref, p);
-    for (int j = sm; ok && j < n; j += 2) {
-      const TileInfo& x = cur.x;
-      const bool sfirst = x.first || prev_first;  // this stream's first tile of the piece
-      const int r = x.qg * kAttnRows + static_cast<int>(rank) * kAttnMT + rl;
-      const bool valid = r < p.R;
-      if (sfirst) {
-        const int node = valid ? r / p.G : 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w)
-          mw[w] = (valid && w < p.words) ? p.anc_mask[(size_t)node * p.words + w] : 0xffffffffu;
-        m_used = -INFINITY;
-        l_run = 0.f;
-        jj = 0;
-      }
-      if (!mbar_wait_bounded(&s_full[sm], (j >> 1) & 1, abort_flag, p.status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const bool tree_tile = x.lt >= x.tpre;
-      const int kbase = tree_tile ? (x.lt - x.tpre) * kAttnBN : x.lt * kAttnBN;
-      const int key_end = tree_tile ? p.N : x.P;
-      const bool full_tile = !tree_tile && kbase + kAttnBN <= key_end;
-      uint32_t tw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-      if (tree_tile) {
-        const bool upper = x.lt > x.tpre;  // second tree tile: nodes 128..255
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tw[q] = upper ? mw[4 + q] : mw[q];
-      }
-      // One pass over the tile in two halves of 64 keys: the exponent base
-      // is the stream's running maximum; a half whose maximum exceeds it by
-      // more than 2^8 (or the stream's first half of a piece) moves it,
-      // rescaling O, l and the half already written, so that every stored
-      // weight stays <= 2^8 (well inside fp16).
-      float sum_tile = 0.f;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float sv[64];
-        {
-          uint32_t r0[32], r1[32];
-          tmem_ld32_raw(srow + h * 64, r0);
-          tmem_ld32_raw(srow + h * 64 + 32, r1);
-          tmem_ld_wait();
-          tmem_regs_after_wait(r0);
-          tmem_regs_after_wait(r1);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            sv[c] = __uint_as_float(r0[c]);
-            sv[32 + c] = __uint_as_float(r1[c]);
-          }
-        }
-        if (!full_tile) {
-          const int nv = min(max(key_end - kbase - h * 64, 0), 64);
-          const uint64_t in_range = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
-          const uint32_t lo = h ? tw[2] : tw[0], hi = h ? tw[3] : tw[1];
-          const uint64_t vis = in_range & ((static_cast<uint64_t>(hi) << 32) | lo);
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (!((vis >> c) & 1ull)) sv[c] = -INFINITY;
-        }
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], sv[c], sv[c + 1]);
-        const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * p.scale_log2;
-        const bool need = (m_used == -INFINITY) ? (mx != -INFINITY) : (mx > m_used + kRescaleLog2);
-        if (__any_sync(0xffffffffu, need)) {
-          const float new_m = need ? mx : m_used;
-          const float corr = (need && m_used != -INFINITY) ? ex2_approx(m_used - new_m) : 1.f;
-          if (jj > 0) {
-            // O must hold this stream's previous tile (j - 2) before it is
-            // rescaled
-            if (!mbar_wait_bounded(&p_empty[sm], ((j >> 1) - 1) & 1, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-#pragma unroll 1
-            for (int ch = 0; ch < DH / 32; ++ch) {
-              float o[32];
-              tmem_ld32(orow + ch * 32, o);
-#pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] *= corr;
-              tmem_st32(orow + ch * 32, o);
-            }
-          }
-          if (h == 1) {
-            // half 0 of this tile is already stored as fp16 pairs
-            uint32_t r0[32];
-            tmem_ld32_raw(srow, r0);
-            tmem_ld_wait();
-            tmem_regs_after_wait(r0);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r0[c]));
-              const __half2 h2 = __floats2half2_rn(f.x * corr, f.y * corr);
-              r0[c] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-            tmem_st32_u(srow, r0);
-          }
-          l_run *= corr;
-          sum_tile *= corr;
-          m_used = new_m;
-        }
-        const float nbase = m_used == -INFINITY ? 0.f : -m_used;
-        const uint64_t scale2 = f32x2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nbase2 = f32x2_pack(nbase, nbase);
-        uint64_t part[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-        for (int q16 = 0; q16 < 2; ++q16) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c = q16 * 32 + 2 * e;
-            float x0, x1;
-            f32x2_unpack(f32x2_fma(f32x2_pack(sv[c], sv[c + 1]), scale2, nbase2), x0, x1);
-            const float a0 = ex2_approx(x0);
-            const float a1 = ex2_approx(x1);
-            part[e & 3] = f32x2_add(part[e & 3], f32x2_pack(a0, a1));
-            const __half2 h2 = __floats2half2_rn(a0, a1);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&h2);
-          }
-          tmem_st16_u(srow + h * 32 + q16 * 16, pk);
-        }
-        float s0, s1;
-        f32x2_unpack(f32x2_add(f32x2_add(part[0], part[1]), f32x2_add(part[2], part[3])), s0, s1);
-        sum_tile += s0 + s1;
-      }
-      if (!ok) break;
-      l_run += sum_tile;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive_cta0(&p_full[sm], pfull0, rank);
-      // this stream's last tile of the piece: the piece's last tile, or the
-      // one before it
-      const bool slast = x.last || (cur.t + 2 == cur.t1) || (x.lt + 2 == x.ntiles);
-      if (slast) {
-        // wait for the stream's last PV of the piece, then write its partial
-        if (!mbar_wait_bounded(&p_empty[sm], (j >> 1) & 1, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const size_t piece = (size_t)x.seg * p.slots + 2 * x.slot + sm;
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        float4* dst = reinterpret_cast<float4*>(p.o_part) + piece * kAttnRows * (DH / 4) +
-                      rank * kAttnMT + rl;
-#pragma unroll 1
-        for (int ch = 0; ch < DH / 32; ++ch) {
-          float o[32];
-          tmem_ld32(orow + ch * 32, o);
-          if (valid) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              dst[(ch * 8 + c) * kAttnRows] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv,
-                                                          o[4 * c + 2] * inv, o[4 * c + 3] * inv);
-          }
-        }
-        const size_t lrow = rank * kAttnMT + rl;
-        if (valid) {
-          p.lse_part[piece * kAttnRows + lrow] = l_run > 0.f ? m_used + log2f(l_run) : -INFINITY;
-          // a one-tile piece has nothing from the other stream
-          if (x.first && x.last)
-            p.lse_part[(piece + 1 - 2 * sm) * kAttnRows + lrow] = -INFINITY;
-        }
-        tc_fence_before();
-        mbar_arrive_cta0(&o_free[sm], ofree0, rank);
-      }
-      ++jj;
-      // on to this stream's next tile, noting whether the other stream's
-      // tile in between starts a piece
-      cur.advance();
-      prev_first = cur.x.first;
-      cur.advance();
-    }
-  }
-
-  // no CTA leaves (or frees its tensor memory) while the other may still
-  // arrive on its barriers or read its tensor / shared memory
-  tc_fence_before();
-  cluster_sync_all();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc_pair(tmem_base, kAttnTmemCols);
-}
-
-// Merge the pieces of every query row.  A CTA takes 32 consecutive query rows
-// (global row = (b * Hkv + kvh) * R + r): lane = row while the partials are
-// read (each warp reads whole 512-byte runs of one column group), then the
-// rows go through shared memory so that each output row is written by 8
-// threads in contiguous pieces.
-constexpr int kCombineRows = 32;
-
-template <int DH>
-__global__ void __launch_bounds__(256)
-    attn_combine_kernel(AttnParams p, void* __restrict__ out, int out_f32) {
-  grid_dep_wait();
-  grid_dep_launch();
-  constexpr int C4 = DH / 4;  // column groups of 4 floats
-  __shared__ int cumT[kAttnMaxB + 1];
-  __shared__ int sched_ok;
-  __shared__ float4 tile[kCombineRows][C4 + 1];
-  if (threadIdx.x < 32) {
-    const bool ok = build_schedule(p, cumT, nullptr);
-    if (threadIdx.x == 0) sched_ok = ok ? 1 : 0;
-  }
-  __syncthreads();
-  if (!sched_ok) return;  // reported by the attention kernel
-  if (p.copy_tree) {
-    // the tree K/V into cache slots P + i (the prefix lengths were checked
-    // against the capacity above)
-    constexpr int kVec = DH / 8;  // 16-byte pieces per row
-    const long long n_vec = (long long)p.B * p.N * p.Hkv * kVec;
-    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n_vec;
-         e += (long long)gridDim.x * blockDim.x) {
-      const int c = static_cast<int>(e % kVec);
-      const long long row = e / kVec;  // (b, i, kvh), kvh fastest
-      const int kvh = static_cast<int>(row % p.Hkv);
-      const long long bi = row / p.Hkv;
-      const int i = static_cast<int>(bi % p.N);
-      const int b = static_cast<int>(bi / p.N);
-      const size_t src = (size_t)row * DH;
-      const size_t dst = (((size_t)b * p.Hkv + kvh) * p.cap + p.prefix_len[b] + i) * DH;
-      reinterpret_cast<uint4*>(p.Kc + dst)[c] = reinterpret_cast<const uint4*>(p.k_new + src)[c];
-      reinterpret_cast<uint4*>(p.Vc + dst)[c] = reinterpret_cast<const uint4*>(p.v_new + src)[c];
-    }
-  }
-  const int per = tiles_per_cta(cumT[p.B], p.grid);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int total_rows = p.B * p.Hkv * p.R;
-  const int gr = blockIdx.x * kCombineRows + lane;
-  if (gr < total_rows) {
-    const int bh = gr / p.R;
-    const int r = gr - bh * p.R;
-    const int b = bh / p.Hkv;
-    const int kvh = bh - b * p.Hkv;
-    const int qg = r / kAttnRows, row = r - qg * kAttnRows;
-    const int P = p.prefix_len[b];
-    const int ntiles = (P + kAttnBN - 1) / kAttnBN + p.T_tree;
-    const int seg_start = cumT[b] + (kvh * p.n_qg + qg) * ntiles;
-    // pieces of the segment, each with slot_mul partial results
-    const int n_pieces = ((seg_start + ntiles - 1) / per - seg_start / per + 1) * p.slot_mul;
-    const size_t pbase = ((size_t)bh * p.n_qg + qg) * p.slots;
-    float M = -INFINITY;
-    for (int k = 0; k < n_pieces; ++k) M = fmaxf(M, p.lse_part[(pbase + k) * kAttnRows + row]);
-    constexpr int PER = C4 / 8;  // column groups per warp
-    float4 acc[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    float wsum = 0.f;
-    for (int k = 0; k < n_pieces; ++k) {
-      const float lse = p.lse_part[(pbase + k) * kAttnRows + row];
-      const float w = lse == -INFINITY ? 0.f : exp2f(lse - M);
-      wsum += w;
-      const float4* src = reinterpret_cast<const float4*>(p.o_part) +
-                          (pbase + k) * kAttnRows * C4 + row;
-#pragma unroll
-      for (int e = 0; e < PER; ++e) {
-        const float4 v = src[(warp + 8 * e) * kAttnRows];
-        acc[e].x += w * v.x;
-        acc[e].y += w * v.y;
-        acc[e].z += w * v.z;
-        acc[e].w += w * v.w;
-      }
-    }
-    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-#pragma unroll
-    for (int e = 0; e < PER; ++e)
-      tile[lane][warp + 8 * e] =
-          make_float4(acc[e].x * inv, acc[e].y * inv, acc[e].z * inv, acc[e].w * inv);
-  }
-  __syncthreads();
-  // writer: 8 threads per row, C4 / 8 consecutive column groups each
-  const int wr = threadIdx.x >> 3, part = threadIdx.x & 7;
-  const int ogr = blockIdx.x * kCombineRows + wr;
-  if (ogr >= total_rows) return;
-  const int bh = ogr / p.R;
-  const int r = ogr - bh * p.R;
-  const int b = bh / p.Hkv;
-  const int kvh = bh - b * p.Hkv;
-  const int node = r / p.G, g = r - node * p.G;
-  constexpr int PER = C4 / 8;
-  const size_t obase = (((size_t)b * p.N + node) * p.Hq + kvh * p.G + g) * DH + part * PER * 4;
-  if (out_f32) {
-    float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + obase);
-#pragma unroll
-    for (int e = 0; e < PER; ++e) o[e] = tile[wr][part * PER + e];
-  } else {
-    uint2* o = reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + obase);
-#pragma unroll
-    for (int e = 0; e < PER; ++e) {
-      const float4 v = tile[wr][part * PER + e];
-      const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
-      const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
-      o[e] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
-                        *reinterpret_cast<const uint32_t*>(&hi));
-    }
   }
 }
 
@@ -1812,8 +1148,8 @@ Plan plan(int N, int Hq, int Hkv, int max_prefix) {
   pl.n_qg = (R + kAttnRows - 1) / kAttnRows;
   pl.T_tree = (N + kAttnBN - 1) / kAttnBN;
   const int max_seg_tiles = (max_prefix + kAttnBN - 1) / kAttnBN + pl.T_tree;
-  // room for two partial results per piece (the pair kernel's two streams)
-  pl.slots = 2 * ((max_seg_tiles + kAttnMinTiles - 1) / kAttnMinTiles + 1);
+  // the pieces a segment can be cut into
+  pl.slots = (max_seg_tiles + kAttnMinTiles - 1) / kAttnMinTiles + 1;
   return pl;
 }
 
@@ -1823,8 +1159,9 @@ size_t tree_attention_workspace_size(int B, int N, int Hq, int Hkv, int dh, int 
                                      medusa_dtype_t dt) {
   if (dt == MEDUSA_F32) return 0;
   const Plan pl = plan(N, Hq, Hkv, max_prefix);
-  const size_t rows = (size_t)B * Hkv * pl.n_qg * pl.slots * kAttnRows;
-  return align256(rows * dh * 4) + align256(rows * 4);
+  const size_t seg_rows = (size_t)B * Hkv * pl.n_qg * kAttnRows;
+  const size_t rows = seg_rows * pl.slots;
+  return align256(rows * dh * 4) + align256(rows * 4) + align256(seg_rows * 4);
 }
 
 template <int DH>
@@ -1878,70 +1215,16 @@ static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaSt
       return fail(MEDUSA_ERR_UNSUPPORTED, "tree_attention: register split exceeds the build's");
   }
   p.grid = device_sm_count();  // persistent: one CTA per SM
-  p.slot_mul = 1;
+  p.out = out;
+  p.out_f32 = out_f32;
+  const size_t n_count = (size_t)p.B * p.Hkv * p.n_qg * kAttnRows;
+  launch(attn_zero_kernel, (int)((n_count + 255) / 256 < 1024 ? (n_count + 255) / 256 : 1024), 256,
+         0, stream, p.row_count, n_count);
+  medusa_status_t st = check_launch("tree_attention_counters");
+  if (st != MEDUSA_OK) return st;
   launch(tree_attn_tc_kernel<DH>, p.grid, kAttnThreads, L::kAlloc, stream, mK, mV, mKn, mVn, mKs0,
          mVs0, mKs1, mVs1, mQ, p);
-  medusa_status_t st = check_launch("tree_attention");
-  if (st != MEDUSA_OK) return st;
-  const int rows = p.B * p.Hkv * p.R;
-  launch(attn_combine_kernel<DH>, (rows + kCombineRows - 1) / kCombineRows, 256, 0, stream, p, out,
-         out_f32);
-  return check_launch("tree_attention_combine");
-}
-
-// dh = 128 on CTA pairs (cta_group::2); the combine kernel also stores the
-// tree K/V into the caches
-static medusa_status_t launch_pair(AttnParams& p, void* out, int out_f32, cudaStream_t stream) {
-  constexpr int DH = PairSmem::DH;
-  // caches [B*Hkv][cap][DH]; tree K/V [B][N][Hkv][DH].  K boxes: 64 dims x
-  // 64 keys (a CTA's key half, one swizzled panel); V boxes: 64 dims x 128 keys
-  // (a CTA's dim half of the whole tile)
-  CUtensorMap mKh, mV, mKnh, mVn;
-  const uint64_t dc[3] = {DH, (uint64_t)p.cap, (uint64_t)p.B * p.Hkv};
-  const uint64_t sc[2] = {DH * 2, (uint64_t)p.cap * DH * 2};
-  const uint32_t bkh[3] = {64, 64, 1};
-  const uint32_t bv[3] = {64, kAttnBN, 1};
-  const uint64_t dn[4] = {DH, (uint64_t)p.Hkv, (uint64_t)p.N, (uint64_t)p.B};
-  const uint64_t sn[3] = {DH * 2, (uint64_t)p.Hkv * DH * 2, (uint64_t)p.N * p.Hkv * DH * 2};
-  const uint32_t bknh[4] = {64, 1, 64, 1};
-  const uint32_t bvn[4] = {64, 1, kAttnBN, 1};
-  // queries as [B][N][Hkv][G][DH]: a box of 64 dims x G heads x 128 / G nodes
-  // is one CTA's M tile (G divides 128)
-  CUtensorMap mQ;
-  const uint64_t dq[5] = {DH, (uint64_t)p.G, (uint64_t)p.Hkv, (uint64_t)p.N, (uint64_t)p.B};
-  const uint64_t sq[4] = {DH * 2, (uint64_t)p.G * DH * 2, (uint64_t)p.Hq * DH * 2,
-                          (uint64_t)p.N * p.Hq * DH * 2};
-  const uint32_t bq[5] = {64, (uint32_t)p.G, 1, (uint32_t)(kAttnMT / p.G), 1};
-  if (!make_tmap_bf16(&mKh, p.Kc, 3, dc, sc, bkh) || !make_tmap_bf16(&mV, p.Vc, 3, dc, sc, bv) ||
-      !make_tmap_bf16(&mKnh, p.k_new, 4, dn, sn, bknh) ||
-      !make_tmap_bf16(&mVn, p.v_new, 4, dn, sn, bvn) || !make_tmap_bf16(&mQ, p.q, 5, dq, sq, bq))
-    return fail(MEDUSA_ERR_CUDA, "tree_attention: cuTensorMapEncodeTiled failed");
-  if (cudaFuncSetAttribute(tree_attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           PairSmem::kAlloc) != cudaSuccess)
-    return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(tree_attention pair) failed");
-  p.grid = device_sm_count() / 2;  // persistent: one pair per two SMs
-  p.copy_tree = 1;
-  p.slot_mul = 2;
-  launch(tree_attn_pair_kernel, 2 * p.grid, kPairThreads, PairSmem::kAlloc, stream, mKh, mV, mKnh,
-         mVn, mQ, p);
-  medusa_status_t st = check_launch("tree_attention_pair");
-  if (st != MEDUSA_OK) return st;
-  const int rows = p.B * p.Hkv * p.R;
-  launch(attn_combine_kernel<DH>, (rows + kCombineRows - 1) / kCombineRows, 256, 0, stream, p, out,
-         out_f32);
-  return check_launch("tree_attention_combine");
-}
-
-// The pair kernel is opt-in: MEDUSA_ATTN_PAIR=1 (read at every call) selects
-// it for dh = 128 when the query-group size G divides 128 (a CTA's Q tile is
-// one bulk tensor box).  On the Llama-3-8B-shaped step it measures slower
-// than the single-CTA kernel (its two streams double the partials the
-// combine merges, and each pair starts later), so the single-CTA kernel is
-// the default.
-static bool use_pair(int dh, int G) {
-  if (dh != 128 || kAttnMT % G != 0) return false;
-  const char* v = getenv("MEDUSA_ATTN_PAIR");
-  return v != nullptr && strcmp(v, "1") == 0;
+  return check_launch("tree_attention");
 }
 
 medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_new, void* Kc,
@@ -1975,9 +1258,12 @@ medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_n
   p.Vc = static_cast<__nv_bfloat16*>(Vc);
   p.prefix_len = prefix_len;
   p.anc_mask = anc_mask;
-  const size_t rows = (size_t)B * Hkv * pl.n_qg * pl.slots * kAttnRows;
+  const size_t seg_rows = (size_t)B * Hkv * pl.n_qg * kAttnRows;
+  const size_t rows = seg_rows * pl.slots;
   p.o_part = static_cast<float*>(ws);
   p.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(rows * dh * 4));
+  p.row_count = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + align256(rows * dh * 4) +
+                                                align256(rows * 4));
   p.B = B;
   p.N = N;
   p.Hq = Hq;
@@ -1992,7 +1278,6 @@ medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_n
   p.words = words;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = status;
-  if (use_pair(dh, p.G)) return launch_pair(p, out, out_f32, stream);
   if (dh == 128) return launch_bf16<128>(p, out, out_f32, stream);
   return launch_bf16<64>(p, out, out_f32, stream);
 }

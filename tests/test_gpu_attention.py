@@ -95,14 +95,7 @@ def test_tiny_fp32():
     (1, 16, 1, 64, (200, 200), "sparse64", 6),     # G 16: four query groups of 256 rows
     (256, 2, 1, 64, (0, 40), "sparse16", 7),       # 256 sequences: the schedule table is full
 ])
-@pytest.mark.parametrize("pair", [True, False], ids=["pair", "single"])
-def test_bf16_small(B, Hq, Hkv, dh, ctx, tree, seed, pair, monkeypatch):
-    # MEDUSA_ATTN_PAIR=1 opts into the CTA-pair (cta_group::2) kernel, which
-    # serves dh 128 when G divides 128; other shapes fall back to the
-    # single-CTA kernel, which the "single" cases cover
-    if pair and (dh != 128 or 128 % (Hq // Hkv) != 0):
-        pytest.skip("the pair kernel serves dh 128 with G dividing 128 only")
-    monkeypatch.setenv("MEDUSA_ATTN_PAIR", "1" if pair else "0")
+def test_bf16_small(B, Hq, Hkv, dh, ctx, tree, seed):
     if tree == "sparse64":
         spec = W.sparse_tree(64, 4, 10, seed, max_depth=4)
     elif tree == "sparse16":
@@ -128,19 +121,5 @@ def test_full_size_sampled_rows(name):
     inp = W.attention_inputs(w, seed=0)
     rng = np.random.default_rng(0)
     rows = [(int(rng.integers(w.B)), int(rng.integers(w.N))) for _ in range(24)]
-    rows += [(0, 0), (w.B - 1, w.N - 1)]
-    _compare(inp, spec, w.ctx_hi, rows=rows)
-
-
-@pytest.mark.slow
-def test_pair_kernel_full_size_sampled_rows(monkeypatch):
-    # the opt-in CTA-pair kernel on the Llama-3-70B shape: 256 nodes, G = 8,
-    # eight query groups, two tree tiles
-    monkeypatch.setenv("MEDUSA_ATTN_PAIR", "1")
-    w = W.WORKLOADS["llama3_70b"]
-    spec = W.tree_for(w)
-    inp = W.attention_inputs(w, seed=1)
-    rng = np.random.default_rng(1)
-    rows = [(int(rng.integers(w.B)), int(rng.integers(w.N))) for _ in range(16)]
     rows += [(0, 0), (w.B - 1, w.N - 1)]
     _compare(inp, spec, w.ctx_hi, rows=rows)
