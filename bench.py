@@ -36,8 +36,9 @@ import torch  # noqa: E402
 
 METRIC = "Medusa decode-verify steps/s (heads+tree attn+accept); % of HBM roofline"
 UNIT = "steps/s"
-KERNELS_PER_STEP = 9  # W1 GEMM, W2 GEMM, top-k merge, tree build, attention, combine,
-#                       verify rows, verify path, KV compaction
+KERNELS_PER_STEP = 10  # W1 GEMM, W2 GEMM, top-k merge, tree build, attention counters,
+#                        attention, attention exact pass (empty list: reads a count),
+#                        verify rows, verify path, KV compaction
 
 
 def _peaks():

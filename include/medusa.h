@@ -216,8 +216,12 @@ MEDUSA_API medusa_status_t medusa_tree_build(const medusa_tree_t* tree, const in
  *   results of key ranges, merged at the end), 256-byte aligned.
  * Precision: bf16 q/k/v, fp32 scores, fp32 softmax statistics; the softmax
  *   weights (at most 2^8 relative to the running maximum) enter the value
- *   product as fp16, with V converted to fp16 in shared memory: |v| >= 65536,
- *   inf or NaN in V is reported as MEDUSA_ERR_DEVICE_CHECK.
+ *   product as fp16, with V converted to fp16 in shared memory.  A V tile
+ *   that fp16 cannot carry (some |v| >= 65536, or every |v| < 2^-6, where fp16
+ *   would lose mantissa bits) puts its kv head's query rows on a list that an
+ *   exact pass recomputes afterwards on CUDA cores in fp32, so any finite bf16
+ *   V is supported; with no such tile the pass only reads an empty list.  Inf
+ *   or NaN in V is reported as MEDUSA_ERR_DEVICE_CHECK.
  *   dt = MEDUSA_F32 runs an fp32 CUDA-core path.
  * Limits: Hq % Hkv == 0; bf16: dh in {64, 128}, B <= 256, pointers 16-byte
  *   aligned; f32: dh <= 256 and dh % 32 == 0; N <= MEDUSA_MAX_NODES.

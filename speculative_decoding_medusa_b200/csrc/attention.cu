@@ -31,6 +31,9 @@
 // so no separate merge pass follows the kernel.  The counters are zeroed by a
 // small kernel before each launch.
 //
+// A V tile fp16 cannot carry flags its segment; an exact CUDA-core pass
+// after the kernel recomputes the flagged segments' rows in fp32.
+//
 // fp32 path: one warp per query row on CUDA cores (small shapes).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -143,6 +146,11 @@ struct AttnParams {
   float* o_part;    // [n_seg, slots, DH / 4, 256] groups of 4 floats
   float* lse_part;  // [n_seg, slots, 256]
   unsigned int* row_count;  // [n_seg, 256] pieces of the row written so far (zeroed per call)
+  // segments whose V has a tile fp16 cannot carry, recomputed by the exact
+  // pass: a flag per segment, their count and list (zeroed per call)
+  int* seg_flag;
+  int* n_flag;
+  int* flag_list;
   void* out;        // [B, N, Hq, DH], bf16 or fp32
   int out_f32;
   int B, N, Hq, Hkv, G, R, n_qg, T_tree, slots, cap, max_prefix, words, grid;
@@ -166,7 +174,7 @@ struct AttnSmem {
   static constexpr int kNumBars = 4 * kAttnStages + 2 + 2 + 2 + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kInfoOff = kMiscOff + 16;           // int info[kAttnStages]
-  static constexpr int kAuxOff = kInfoOff + 16;            // int {bh, row0}[kAttnStages]
+  static constexpr int kAuxOff = kInfoOff + 16;  // int {bh, cache row0, segment, -}[kAttnStages]
   static constexpr int kCumOff = kAuxOff + 32;             // int cumT[kAttnMaxB + 1]
   static constexpr int kPrefOff = kCumOff + (kAttnMaxB + 1) * 4;  // int P[kAttnMaxB]
   static constexpr int kBytes = kPrefOff + kAttnMaxB * 4;
@@ -420,12 +428,79 @@ __device__ __noinline__ void merge_row(const float* o_part, const float* lse_par
   }
 }
 
-// Row counters of the in-kernel merge, zeroed before every attention launch.
+// Row counters of the in-kernel merge and the exact pass's segment flags and
+// count, zeroed before every attention launch (one contiguous range).
 __global__ void attn_zero_kernel(unsigned int* __restrict__ cnt, size_t n) {
   grid_dep_wait();
   grid_dep_launch();
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
     cnt[i] = 0u;
+}
+
+// The exact pass: every query row of every listed segment recomputed on CUDA
+// cores from the bf16 inputs with fp32 arithmetic (one warp per row, lanes
+// splitting dh, eight prefix keys per online-softmax update), overwriting the
+// tensor-core kernel's output rows.  With no segment listed it only reads the
+// count.
+template <int DH>
+__global__ void __launch_bounds__(256) tree_attn_exact_kernel(AttnParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int nf = *reinterpret_cast<volatile int*>(p.n_flag);
+  if (nf == 0) return;
+  constexpr int PER = DH / 32;
+  const int lane = threadIdx.x & 31;
+  const long long n_rows = (long long)nf * kAttnRows;
+  const float scale = p.scale_log2 * 0.6931471805599453f;  // back to natural units
+  for (long long e = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); e < n_rows;
+       e += (long long)gridDim.x * 8) {
+    const int seg = p.flag_list[e / kAttnRows];
+    const int r = (seg % p.n_qg) * kAttnRows + static_cast<int>(e % kAttnRows);
+    if (r >= p.R) continue;
+    const int bh = seg / p.n_qg, b = bh / p.Hkv, kvh = bh - b * p.Hkv;
+    const int node = r / p.G, g = r - node * p.G;
+    const int P = p.prefix_len[b];
+    float qv[PER], acc[PER];
+    const __nv_bfloat16* qp = p.q + (((size_t)b * p.N + node) * p.Hq + kvh * p.G + g) * DH;
+#pragma unroll
+    for (int c = 0; c < PER; ++c) {
+      qv[c] = __bfloat162float(qp[lane * PER + c]);
+      acc[c] = 0.f;
+    }
+    float m = -INFINITY, l = 0.f;
+    auto visit = [&](const __nv_bfloat16* kp, const __nv_bfloat16* vp) {
+      float d = 0.f;
+#pragma unroll
+      for (int c = 0; c < PER; ++c) d += qv[c] * __bfloat162float(kp[lane * PER + c]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      const float sc = d * scale;
+      const float mn = fmaxf(m, sc);
+      const float corr = expf(m - mn), w = expf(sc - mn);
+      l = l * corr + w;
+#pragma unroll
+      for (int c = 0; c < PER; ++c) acc[c] = acc[c] * corr + w * __bfloat162float(vp[lane * PER + c]);
+      m = mn;
+    };
+    const size_t hb = ((size_t)b * p.Hkv + kvh) * p.cap;
+    for (int t = 0; t < P; ++t) visit(p.Kc + (hb + t) * DH, p.Vc + (hb + t) * DH);
+    for (int jn = 0; jn < p.N; ++jn) {
+      if ((p.anc_mask[(size_t)node * p.words + (jn >> 5)] >> (jn & 31)) & 1u) {
+        const size_t off = (((size_t)b * p.N + jn) * p.Hkv + kvh) * DH;
+        visit(p.k_new + off, p.v_new + off);
+      }
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const size_t ob = (((size_t)b * p.N + node) * p.Hq + kvh * p.G + g) * DH;
+    if (p.out_f32) {
+#pragma unroll
+      for (int c = 0; c < PER; ++c) static_cast<float*>(p.out)[ob + lane * PER + c] = acc[c] * inv;
+    } else {
+#pragma unroll
+      for (int c = 0; c < PER; ++c)
+        static_cast<__nv_bfloat16*>(p.out)[ob + lane * PER + c] = __float2bfloat16_rn(acc[c] * inv);
+    }
+  }
 }
 
 template <int DH>
@@ -538,8 +613,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // MMA and converter warps read it instead of walking the schedule
         const int bh = x.b * p.Hkv + x.kvh;
         stage_info[st] = pack_stage_info(x);
-        stage_aux[2 * st] = bh;
-        stage_aux[2 * st + 1] = x.P + (x.lt - x.tpre) * kAttnBN;
+        stage_aux[4 * st] = bh;
+        stage_aux[4 * st + 1] = x.P + (x.lt - x.tpre) * kAttnBN;
+        stage_aux[4 * st + 2] = x.seg;
         mbar_arrive_expect_tx(&kv_full[st], 2 * L::kKVBytes);
         uint8_t* kdst = smem + L::kKOff + st * L::kKVBytes;
         uint8_t* vdst = smem + L::kVOff + st * L::kKVBytes;
@@ -671,9 +747,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ---------------- V converters (warps 2, 3) ----------------
     // Each landed V tile is rewritten in place from bf16 to fp16 (the value
     // product runs on fp16 P and V); rows past the prefix end of a partial
-    // tile are cleared (their weights are zero, but 0 * NaN is not).  A V
-    // entry of magnitude 65536 or more, inf or NaN is reported as a
-    // device-check error.
+    // tile are cleared (their weights are zero, but 0 * NaN is not).  A tile
+    // fp16 cannot carry - some |v| of 65536 or more, or all of a warp's |v|
+    // below 2^-6, where fp16 loses mantissa bits - puts its segment on the
+    // list of the exact pass that follows the kernel.  Inf or NaN in V is
+    // reported as a device-check error.
     const int ct = (warp - 2) * 32 + lane;
     bool range_ok = true;
     uint32_t copy_par = 0;  // bit s: parity of the copies made from stage s
@@ -691,7 +769,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const bool second = info_second_tree(info);
           const CUtensorMap* mk = second ? &tmKs1 : &tmKs0;
           const CUtensorMap* mv = second ? &tmVs1 : &tmVs0;
-          const int bh = stage_aux[2 * st], row0 = stage_aux[2 * st + 1];
+          const int bh = stage_aux[4 * st], row0 = stage_aux[4 * st + 1];
           const uint8_t* ks = smem + L::kKOff + st * L::kKVBytes;
 #pragma unroll
           for (int pn = 0; pn < L::kPanels; ++pn) {
@@ -733,9 +811,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) vt[e0 + u * 64] = v[u];
       }
-      // |v| of 65536 and above (0x4780: the first bf16 past fp16's 65504),
-      // inf or NaN cannot be carried by the fp16 value product
-      if (__vcmpgtu2(vmax, 0x477F477Fu)) range_ok = false;
+      // 0x4780: the first bf16 past fp16's largest value 65504; 0x3C80: 2^-6;
+      // 0x7F80 and above: inf or NaN
+      const uint32_t vm = max(vmax & 0xffffu, vmax >> 16);
+      if (vm >= 0x7F80u) range_ok = false;
+      const uint32_t wmax = __reduce_max_sync(0xffffffffu, vm);
+      if (lane == 0 && wmax < 0x7F80u && (wmax >= 0x4780u || (wmax != 0u && wmax < 0x3C80u))) {
+        const int seg = stage_aux[4 * st + 2];
+        if (atomicCAS(&p.seg_flag[seg], 0, 1) == 0) p.flag_list[atomicAdd(p.n_flag, 1)] = seg;
+      }
       fence_proxy_async_smem();
       mbar_arrive(&v_ready[st]);
     }
@@ -1159,9 +1243,13 @@ size_t tree_attention_workspace_size(int B, int N, int Hq, int Hkv, int dh, int 
                                      medusa_dtype_t dt) {
   if (dt == MEDUSA_F32) return 0;
   const Plan pl = plan(N, Hq, Hkv, max_prefix);
-  const size_t seg_rows = (size_t)B * Hkv * pl.n_qg * kAttnRows;
+  const size_t n_seg = (size_t)B * Hkv * pl.n_qg;
+  const size_t seg_rows = n_seg * kAttnRows;
   const size_t rows = seg_rows * pl.slots;
-  return align256(rows * dh * 4) + align256(rows * 4) + align256(seg_rows * 4);
+  // partials, log-sum-exps, then one zeroed range: row counters, segment
+  // flags, the flag count; then the flagged-segment list
+  return align256(rows * dh * 4) + align256(rows * 4) + align256((seg_rows + n_seg + 1) * 4) +
+         align256(n_seg * 4);
 }
 
 template <int DH>
@@ -1217,14 +1305,17 @@ static medusa_status_t launch_bf16(AttnParams& p, void* out, int out_f32, cudaSt
   p.grid = device_sm_count();  // persistent: one CTA per SM
   p.out = out;
   p.out_f32 = out_f32;
-  const size_t n_count = (size_t)p.B * p.Hkv * p.n_qg * kAttnRows;
+  const size_t n_count = (size_t)p.B * p.Hkv * p.n_qg * (kAttnRows + 1) + 1;
   launch(attn_zero_kernel, (int)((n_count + 255) / 256 < 1024 ? (n_count + 255) / 256 : 1024), 256,
          0, stream, p.row_count, n_count);
   medusa_status_t st = check_launch("tree_attention_counters");
   if (st != MEDUSA_OK) return st;
   launch(tree_attn_tc_kernel<DH>, p.grid, kAttnThreads, L::kAlloc, stream, mK, mV, mKn, mVn, mKs0,
          mVs0, mKs1, mVs1, mQ, p);
-  return check_launch("tree_attention");
+  st = check_launch("tree_attention");
+  if (st != MEDUSA_OK) return st;
+  launch(tree_attn_exact_kernel<DH>, p.grid, 256, 0, stream, p);
+  return check_launch("tree_attention_exact");
 }
 
 medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_new, void* Kc,
@@ -1258,12 +1349,17 @@ medusa_status_t tree_attention(const void* q, const void* k_new, const void* v_n
   p.Vc = static_cast<__nv_bfloat16*>(Vc);
   p.prefix_len = prefix_len;
   p.anc_mask = anc_mask;
-  const size_t seg_rows = (size_t)B * Hkv * pl.n_qg * kAttnRows;
+  const size_t n_seg = (size_t)B * Hkv * pl.n_qg;
+  const size_t seg_rows = n_seg * kAttnRows;
   const size_t rows = seg_rows * pl.slots;
-  p.o_part = static_cast<float*>(ws);
-  p.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(rows * dh * 4));
-  p.row_count = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + align256(rows * dh * 4) +
-                                                align256(rows * 4));
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  p.o_part = reinterpret_cast<float*>(w8);
+  p.lse_part = reinterpret_cast<float*>(w8 + align256(rows * dh * 4));
+  p.row_count = reinterpret_cast<unsigned int*>(w8 + align256(rows * dh * 4) + align256(rows * 4));
+  p.seg_flag = reinterpret_cast<int*>(p.row_count + seg_rows);
+  p.n_flag = p.seg_flag + n_seg;
+  p.flag_list = reinterpret_cast<int*>(w8 + align256(rows * dh * 4) + align256(rows * 4) +
+                                       align256((seg_rows + n_seg + 1) * 4));
   p.B = B;
   p.N = N;
   p.Hq = Hq;

@@ -123,3 +123,68 @@ def test_full_size_sampled_rows(name):
     rows = [(int(rng.integers(w.B)), int(rng.integers(w.N))) for _ in range(24)]
     rows += [(0, 0), (w.B - 1, w.N - 1)]
     _compare(inp, spec, w.ctx_hi, rows=rows)
+
+
+def _scaled_v(inp, b, factor, rows=None, tree=False):
+    """V of sequence b (cache rows `rows`, or all; the tree's v_new too when
+    `tree`) multiplied by `factor`, rounded to bf16 like any input."""
+    out = dict(inp)
+    Vc = inp["Vc"].float().clone()
+    sl = slice(None) if rows is None else rows
+    Vc[b, :, sl] *= factor
+    out["Vc"] = Vc.to(inp["Vc"].dtype)
+    if tree:
+        vn = inp["v_new"].float().clone()
+        vn[b] *= factor
+        out["v_new"] = vn.to(inp["v_new"].dtype)
+    return out
+
+
+@pytest.mark.parametrize("case", ["large", "tiny", "mixed_tile", "large_tree"])
+def test_bf16_v_outside_fp16_range(case):
+    """V tiles that fp16 cannot carry (|v| up to about 4e6, or all |v| near
+    1e-6) take the bf16 value product; per sequence the output must match the
+    oracle to the usual relative bounds, whatever the magnitude."""
+    spec = W.sparse_tree(64, 4, 10, 3, max_depth=4)
+    w = W.scaled(W.WORKLOADS["llama3_8b"], B=3, Hq=8, Hkv=2, dh=128, ctx_lo=300, ctx_hi=700,
+                 N=spec.n_nodes)
+    inp = W.attention_inputs(w, seed=11)
+    if case == "large":
+        inp = _scaled_v(inp, 0, 1e6)
+    elif case == "tiny":
+        inp = _scaled_v(inp, 1, 1e-6)
+    elif case == "mixed_tile":  # a few rows of one tile large, the rest of it normal
+        inp = _scaled_v(inp, 2, 3e5, rows=slice(130, 140))
+    else:  # the tree's own values large too (the reload reads v_new)
+        inp = _scaled_v(inp, 0, 1e6, tree=True)
+    mask = _mask(spec, w.B)
+    got, Kg, Vg = _run_gpu(inp, mask, w.ctx_hi, torch.float32)
+    ref = O.tree_attention(f64(inp["q"]), f64(inp["k_new"]), f64(inp["v_new"]), f64(inp["Kc"]),
+                           f64(inp["Vc"]), i64(inp["prefix_len"]), mask, 1.0 / math.sqrt(w.dh))
+    for b in range(w.B):
+        scale = np.abs(ref["out"][b]).max()
+        assert np.abs(got[b] - ref["out"][b]).max() < LOGIT_MAX_ABS * scale, (case, b)
+        assert rel_l2(got[b], ref["out"][b]) < ATTN_REL_L2, (case, b, rel_l2(got[b], ref["out"][b]))
+    np.testing.assert_array_equal(Kg.double().numpy(), ref["Kc"])
+    np.testing.assert_array_equal(Vg.double().numpy(), ref["Vc"])
+
+
+def test_bf16_v_nan_is_reported():
+    """Inf or NaN in V is a device-check error (status 6), not a fault."""
+    spec = W.cartesian_tree([2, 3])
+    w = W.scaled(W.WORKLOADS["llama3_8b"], B=1, Hq=4, Hkv=1, dh=128, ctx_lo=200, ctx_hi=200,
+                 N=spec.n_nodes)
+    inp = W.attention_inputs(w, seed=12)
+    Vc = inp["Vc"].clone()
+    Vc[0, 0, 17, 5] = float("nan")
+    inp["Vc"] = Vc
+    dev = "cuda"
+    mask = _mask(spec, 1)
+    out = torch.empty(1, spec.n_nodes, 4, 128, dtype=torch.float32, device=dev)
+    status = M.new_status()
+    M.medusa_tree_attention(*(inp[k].to(dev) for k in ("q", "k_new", "v_new", "Kc", "Vc")),
+                            inp["prefix_len"].to(dev),
+                            torch.from_numpy(mask.view(np.int32).copy()).to(dev), w.ctx_hi, out,
+                            dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 6
