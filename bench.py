@@ -2,7 +2,7 @@
 """Benchmark of the Medusa decode-verify step on B200.
 
 One step = heads + top-k, tree build, tree attention, verify/accept and KV
-compaction for one batch (the five C-ABI calls).  Default workload: the
+compaction for one batch (four C-ABI calls: the last two are one).  Default workload: the
 Llama-3-8B-shaped configuration (batch 8, hidden 4096, vocab 128256, 4 heads,
 64-node sparse tree, GQA 32/8 heads of 128, ragged prefixes 4096..8192, bf16,
 greedy acceptance).  Inputs are seeded synthetic data of those shapes; every
@@ -36,9 +36,9 @@ import torch  # noqa: E402
 
 METRIC = "Medusa decode-verify steps/s (heads+tree attn+accept); % of HBM roofline"
 UNIT = "steps/s"
-KERNELS_PER_STEP = 10  # W1 GEMM, W2 GEMM, top-k merge, tree build, attention counters,
-#                        attention, attention exact pass (empty list: reads a count),
-#                        verify rows, verify path, KV compaction
+KERNELS_PER_STEP = 9  # W1 GEMM, W2 GEMM, top-k merge, tree build, attention counters,
+#                       attention, attention exact pass (empty list: reads a count),
+#                       verify rows, verify path with the KV compaction
 
 
 def _peaks():
@@ -587,13 +587,12 @@ def main():
                                 att["prefix_len"], step.anc_mask, w.ctx_hi, step.attn_out, None,
                                 step.ws_attn, step.status)
         evs[3].record(stream)
-        M.medusa_verify_accept(logits, step.cand_ids, tree, step.accept_len, step.accepted_nodes,
-                               step.accepted_tokens, step.bonus, step.mode, w.temperature, w.eps,
-                               w.delta, step.ws_verify, step.status)
+        M.medusa_verify_accept_compact(logits, step.cand_ids, tree, step.accept_len,
+                                       step.accepted_nodes, step.accepted_tokens, step.bonus,
+                                       att["Kc"], att["Vc"], att["prefix_len"], step.compact_src,
+                                       step.mode, w.temperature, w.eps, w.delta, step.ws_verify,
+                                       step.status)
         evs[4].record(stream)
-        M.medusa_kv_compact(att["Kc"], att["Vc"], att["prefix_len"], step.accepted_nodes,
-                            step.accept_len, step.compact_src, step.status)
-        evs[5].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         one_step()
@@ -626,11 +625,11 @@ def main():
     ms_step = ms_total / args.steps
     # stage breakdown from a separate, untimed pass with events between the calls
     n_stage = min(args.steps, 50)
-    stage_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_stage)]
+    stage_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_stage)]
     for k in range(n_stage):
         one_step(stage_evs[k])
     torch.cuda.synchronize()
-    names = ["heads_topk", "tree_build", "tree_attention", "verify_accept", "kv_compact"]
+    names = ["heads_topk", "tree_build", "tree_attention", "verify_accept_compact"]
     stages = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in stage_evs) * 1e3
               for i, n in enumerate(names)}  # us
     assert int(step.status.item()) == 0

@@ -15,7 +15,8 @@
  *
  * Around them: medusa_lmhead_verify (the verification from the nodes' hidden
  * states, lm_head fused), medusa_next_step (inputs of the next step),
- * medusa_sample_bonus (a drawn bonus token), medusa_tree_from_accuracies
+ * medusa_sample_bonus (a drawn bonus token), medusa_verify_accept_compact
+ * (the last two calls in one), medusa_tree_from_accuracies
  * (the sparse tree of the most accurate combinations, host only), the
  * vocabulary-sharding calls (medusa_topk_merge, medusa_verify_records,
  * medusa_verify_from_records), medusa_verify_accept_noalloc and
@@ -299,6 +300,32 @@ MEDUSA_API medusa_status_t medusa_kv_compact(void* Kc, void* Vc, medusa_dtype_t 
                                   const int32_t* accepted_nodes, const int32_t* accept_len,
                                   int B, int Hkv, int dh, int cap, int max_depth,
                                   int32_t* compact_src, int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
+ * medusa_verify_accept_compact
+ *
+ * medusa_verify_accept followed by medusa_kv_compact of its result, in the
+ * same launches as medusa_verify_accept alone: the block that picks a
+ * sequence's kept branch then moves that branch's K/V (the sections cited at
+ * the two calls).  Results, in every output of both calls, equal those of
+ * the two calls made one after the other on the same stream.
+ *
+ * Arguments: those of medusa_verify_accept, then the caches Kc, Vc
+ *   [B, Hkv, cap, dh] of dtype kv_dt, prefix_len [B] (in/out) and
+ *   compact_src [B, max_depth+1] (out) as in medusa_kv_compact; its B and
+ *   max_depth are the verification's.  Workspace as medusa_verify_accept.
+ * Host checks: medusa_verify_accept's, then medusa_kv_compact's, then the
+ *   workspace; nothing is launched on an error.
+ * Device checks: medusa_verify_accept's; a kept slot P + node outside
+ *   [0, cap).  A sequence whose tree fails the device check, or whose kept
+ *   slots fail it, is not compacted and its prefix_len is unchanged.
+ * ---------------------------------------------------------------------- */
+MEDUSA_API medusa_status_t medusa_verify_accept_compact(
+    const void* logits, medusa_dtype_t dt, const int32_t* cand_ids, const medusa_tree_t* tree,
+    int B, int V, medusa_accept_t mode, float temperature, float eps, float delta,
+    int32_t* accept_len, int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
+    void* Kc, void* Vc, medusa_dtype_t kv_dt, int32_t* prefix_len, int Hkv, int dh, int cap,
+    int32_t* compact_src, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* ------------------------------------------------------------------------
  * medusa_verify_accept_noalloc

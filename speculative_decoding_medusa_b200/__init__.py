@@ -12,7 +12,8 @@ from ._lib import (  # noqa: F401
     medusa_next_step, medusa_sample_bonus, medusa_topk_merge, medusa_tree_from_accuracies,
     medusa_verify_from_records, medusa_verify_records, medusa_verify_records_workspace_size,
     medusa_tree_attention, medusa_tree_attention_workspace_size,
-    medusa_tree_build, medusa_verify_accept, medusa_verify_accept_noalloc,
+    medusa_tree_build, medusa_verify_accept, medusa_verify_accept_compact,
+    medusa_verify_accept_noalloc,
     medusa_verify_accept_workspace_size, medusa_wait_flag, new_status,
     workspace,
 )

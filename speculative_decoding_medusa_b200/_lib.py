@@ -36,7 +36,7 @@ EXPORTS = (
     "medusa_tree_build",
     "medusa_tree_attention_workspace_size", "medusa_tree_attention",
     "medusa_verify_accept_workspace_size", "medusa_verify_accept",
-    "medusa_kv_compact", "medusa_verify_accept_noalloc",
+    "medusa_kv_compact", "medusa_verify_accept_compact", "medusa_verify_accept_noalloc",
     "medusa_lmhead_verify_workspace_size", "medusa_lmhead_verify", "medusa_next_step",
     "medusa_tree_from_accuracies", "medusa_sample_bonus", "medusa_topk_merge",
     "medusa_verify_records_workspace_size", "medusa_verify_records", "medusa_verify_from_records",
@@ -94,6 +94,10 @@ def lib() -> ctypes.CDLL:
     L.medusa_verify_accept_noalloc.restype = _I
     L.medusa_verify_accept_noalloc.argtypes = [_V, _I, _V, ctypes.POINTER(medusa_tree_t), _I, _I, _I,
                                                _F, _F, _F, _V, _V, _V, _V, _V, _V]
+    L.medusa_verify_accept_compact.restype = _I
+    L.medusa_verify_accept_compact.argtypes = [_V, _I, _V, ctypes.POINTER(medusa_tree_t), _I, _I, _I,
+                                               _F, _F, _F, _V, _V, _V, _V, _V, _V, _I, _V, _I, _I,
+                                               _I, _V, _V, _Z, _V, _V]
     L.medusa_kv_compact.restype = _I
     L.medusa_kv_compact.argtypes = [_V, _V, _I, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V, _V]
     L.medusa_lmhead_verify_workspace_size.restype = _Z
@@ -275,6 +279,28 @@ def medusa_kv_compact(Kc, Vc, prefix_len, accepted_nodes, accept_len, compact_sr
     _check(lib().medusa_kv_compact(_p(Kc), _p(Vc), _dt(Kc), _p(prefix_len), _p(accepted_nodes),
                                    _p(accept_len), B, Hkv, dh, cap, max_depth, _p(compact_src),
                                    _p(dev_status), _stream(stream)))
+
+
+def medusa_verify_accept_compact(logits, cand_ids, tree: Tree, accept_len, accepted_nodes,
+                                 accepted_tokens, bonus, Kc, Vc, prefix_len, compact_src,
+                                 mode: int = MEDUSA_ACCEPT_GREEDY, temperature: float = 1.0,
+                                 eps: float = 0.09, delta: float = 0.3, ws=None, dev_status=None,
+                                 stream=None) -> None:
+    """medusa_verify_accept, then medusa_kv_compact of its result, in the
+    verification's launches."""
+    _req(logits, "logits")
+    _req(Kc, "Kc")
+    _req(Vc, "Vc")
+    B, N, V = logits.shape
+    _, Hkv, cap, dh = Kc.shape
+    if ws is None:
+        ws = workspace(medusa_verify_accept_workspace_size(B, N, V), logits.device)
+    ct = tree.c()
+    _check(lib().medusa_verify_accept_compact(
+        _p(logits), _dt(logits), _p(cand_ids), ctypes.byref(ct), B, V, mode, float(temperature),
+        float(eps), float(delta), _p(accept_len), _p(accepted_nodes), _p(accepted_tokens),
+        _p(bonus), _p(Kc), _p(Vc), _dt(Kc), _p(prefix_len), Hkv, dh, cap, _p(compact_src),
+        _p(ws), ws.numel(), _p(dev_status), _stream(stream)))
 
 
 def medusa_verify_accept_noalloc(logits, cand_ids, tree: Tree, accept_len, accepted_nodes,

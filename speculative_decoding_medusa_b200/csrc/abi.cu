@@ -216,6 +216,41 @@ medusa_status_t medusa_verify_accept(const void* logits, medusa_dtype_t dt,
                                static_cast<cudaStream_t>(stream));
 }
 
+medusa_status_t medusa_verify_accept_compact(
+    const void* logits, medusa_dtype_t dt, const int32_t* cand_ids, const medusa_tree_t* tree,
+    int B, int V, medusa_accept_t mode, float temperature, float eps, float delta,
+    int32_t* accept_len, int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
+    void* Kc, void* Vc, medusa_dtype_t kv_dt, int32_t* prefix_len, int Hkv, int dh, int cap,
+    int32_t* compact_src, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  medusa_status_t st = medusa::check_verify_accept_args(logits, dt, cand_ids, tree, B, V, mode,
+                                                        temperature, eps, delta, accept_len,
+                                                        accepted_nodes, accepted_tokens, bonus);
+  if (st != MEDUSA_OK) return st;
+  // the checks of medusa_kv_compact
+  if (!Kc || !Vc || !prefix_len || !compact_src)
+    return fail(MEDUSA_ERR_INVALID_ARG, "verify_accept_compact: null pointer");
+  if (!valid_dtype(kv_dt)) return fail(MEDUSA_ERR_INVALID_ARG, "verify_accept_compact: bad dtype");
+  if (Hkv < 1 || dh < 1 || cap < 1 || tree->max_depth >= MEDUSA_MAX_HEADS)
+    return fail(MEDUSA_ERR_SHAPE, "verify_accept_compact: Hkv, dh, cap or max_depth out of range");
+  const int row_bytes = dh * (kv_dt == MEDUSA_BF16 ? 2 : 4);
+  if (row_bytes % 16 != 0)
+    return fail(MEDUSA_ERR_SHAPE, "verify_accept_compact: a cache row must be a multiple of 16 bytes");
+  if (!aligned16(Kc) || !aligned16(Vc))
+    return fail(MEDUSA_ERR_ALIGNMENT, "verify_accept_compact: caches not 16-byte aligned");
+  int heads_per_round = 0;
+  size_t smem = 0;
+  if (!medusa::compact_plan(kv_dt, dh, Hkv, tree->max_depth, &heads_per_round, &smem))
+    return fail(MEDUSA_ERR_UNSUPPORTED, "verify_accept_compact: (max_depth+1) * row too large");
+  const size_t need = medusa::verify_accept_workspace_size(B, tree->n_nodes, V);
+  if (ws == nullptr || ws_bytes < need || !aligned256(ws))
+    return fail(MEDUSA_ERR_WORKSPACE, "verify_accept_compact: workspace null, misaligned or too small");
+  const medusa::CompactArgs ca{static_cast<uint8_t*>(Kc), static_cast<uint8_t*>(Vc), row_bytes,
+                               prefix_len, Hkv, cap, heads_per_round, compact_src};
+  return medusa::verify_accept(logits, dt, cand_ids, *tree, B, V, mode, temperature, eps, delta,
+                               accept_len, accepted_nodes, accepted_tokens, bonus, ws, dev_status,
+                               static_cast<cudaStream_t>(stream), ca, smem);
+}
+
 size_t medusa_lmhead_verify_workspace_size(int B, int N, int d, int V) {
   if (B < 1 || N < 1 || d < 1 || V < 1 || (long long)B * N > 65535) return 0;
   return medusa::lmhead_verify_workspace_size(B, N, d, V);

@@ -9,6 +9,7 @@
 #include <stdint.h>
 
 #include "../../include/medusa.h"
+#include "kv_compact.cuh"
 
 namespace medusa {
 
@@ -18,6 +19,11 @@ medusa_status_t fail(medusa_status_t code, const char* msg);
 medusa_status_t check_launch(const char* what);
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// KV compaction staging: kv heads per round and the dynamic shared memory it
+// takes (false when one head's kept rows do not fit)
+bool compact_plan(medusa_dtype_t dt, int dh, int Hkv, int max_depth, int* heads_per_round,
+                  size_t* smem);
 
 // the argument checks of medusa_verify_accept, all but the workspace's
 medusa_status_t check_verify_accept_args(const void* logits, medusa_dtype_t dt,
@@ -77,11 +83,14 @@ medusa_status_t verify_path_from_parts(const RowPart* part, int n_chunks,
                                        int32_t* bonus, int32_t* status, cudaStream_t stream);
 
 size_t verify_accept_workspace_size(int B, int N, int V);
+// ca.Kc != nullptr: the path kernel also compacts the kept branch (ca_smem
+// bytes of dynamic shared memory, from compact_plan)
 medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32_t* cand_ids,
                               const medusa_tree_t& tree, int B, int V, medusa_accept_t mode,
                               float temperature, float eps, float delta, int32_t* accept_len,
                               int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
-                              void* ws, int32_t* status, cudaStream_t stream);
+                              void* ws, int32_t* status, cudaStream_t stream,
+                              const CompactArgs& ca = CompactArgs{}, size_t ca_smem = 0);
 
 size_t lmhead_verify_workspace_size(int B, int N, int d, int V);
 medusa_status_t lmhead_verify(const void* hidden, const void* lm_head, const int32_t* cand_ids,

@@ -16,6 +16,7 @@
 
 #include "abi_internal.h"
 #include "common.cuh"
+#include "kv_compact.cuh"
 
 namespace medusa {
 
@@ -56,35 +57,18 @@ __global__ void __launch_bounds__(kCompactThreads)
     return;
   }
 
-  // Rounds of heads_per_round kv heads: every source row of the round is in
-  // shared memory before any destination row is written (a destination of
-  // one step may be the source of another within a head).
-  const int vec_per_row = row_bytes / 16;
-  const int per_head = (L + 1) * vec_per_row;
-  uint4* sk = reinterpret_cast<uint4*>(stage);
-  uint4* sv = sk + (size_t)heads_per_round * W * vec_per_row;
-  for (int h0 = 0; h0 < Hkv; h0 += heads_per_round) {
-    const int nh = min(heads_per_round, Hkv - h0);
-    const int n_vec = nh * per_head;
-    for (int e = tid; e < n_vec; e += kCompactThreads) {
-      const int hh = e / per_head, r = e - hh * per_head;
-      const int j = r / vec_per_row, c = r - j * vec_per_row;
-      const size_t src = (((size_t)b * Hkv + h0 + hh) * cap + s_src[j]) * row_bytes;
-      sk[e] = reinterpret_cast<const uint4*>(Kc + src)[c];
-      sv[e] = reinterpret_cast<const uint4*>(Vc + src)[c];
-    }
-    __syncthreads();
-    for (int e = tid; e < n_vec; e += kCompactThreads) {
-      const int hh = e / per_head, r = e - hh * per_head;
-      const int j = r / vec_per_row, c = r - j * vec_per_row;
-      const size_t dst = (((size_t)b * Hkv + h0 + hh) * cap + P + j) * row_bytes;
-      reinterpret_cast<uint4*>(Kc + dst)[c] = sk[e];
-      reinterpret_cast<uint4*>(Vc + dst)[c] = sv[e];
-    }
-    __syncthreads();
-  }
-  if (tid < W) compact_src[(size_t)b * W + tid] = tid <= L ? s_src[tid] : -1;
-  if (tid == 0) prefix_len[b] = P + L + 1;
+  const CompactArgs a{Kc, Vc, row_bytes, prefix_len, Hkv, cap, heads_per_round, compact_src};
+  compact_sequence(a, b, P, L, s_src, W, reinterpret_cast<uint4*>(stage));
+}
+
+bool compact_plan(medusa_dtype_t dt, int dh, int Hkv, int max_depth, int* heads_per_round,
+                  size_t* smem) {
+  const int row_bytes = dh * (dt == MEDUSA_BF16 ? 2 : 4);
+  const size_t per_head = 2 * (size_t)(max_depth + 1) * row_bytes;
+  if (per_head > kCompactSmem) return false;
+  *heads_per_round = (int)std::min<size_t>((size_t)Hkv, kCompactSmem / per_head);
+  *smem = per_head * *heads_per_round;
+  return true;
 }
 
 medusa_status_t kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefix_len,
@@ -92,11 +76,10 @@ medusa_status_t kv_compact(void* Kc, void* Vc, medusa_dtype_t dt, int32_t* prefi
                            int Hkv, int dh, int cap, int max_depth, int32_t* compact_src,
                            int32_t* status, cudaStream_t stream) {
   const int row_bytes = dh * (dt == MEDUSA_BF16 ? 2 : 4);
-  const size_t per_head = 2 * (size_t)(max_depth + 1) * row_bytes;
-  if (per_head > kCompactSmem)
+  int heads_per_round = 0;
+  size_t smem = 0;
+  if (!compact_plan(dt, dh, Hkv, max_depth, &heads_per_round, &smem))
     return fail(MEDUSA_ERR_UNSUPPORTED, "kv_compact: (max_depth+1) * row too large");
-  const int heads_per_round = (int)std::min<size_t>((size_t)Hkv, kCompactSmem / per_head);
-  const size_t smem = per_head * heads_per_round;
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(kv_compact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kCompactSmem) != cudaSuccess)

@@ -21,6 +21,7 @@
 
 #include "abi_internal.h"
 #include "common.cuh"
+#include "kv_compact.cuh"
 
 namespace medusa {
 
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(kPathThreads)
                        int N, int max_depth, int V, int typical, float inv_T, float eps,
                        float delta, int32_t* __restrict__ accept_len,
                        int32_t* __restrict__ accepted_nodes, int32_t* __restrict__ accepted_tokens,
-                       int32_t* __restrict__ bonus, int32_t* status) {
+                       int32_t* __restrict__ bonus, int32_t* status, CompactArgs ca) {
   grid_dep_wait();
   grid_dep_launch();
   __shared__ int s_g[MEDUSA_MAX_NODES];
@@ -327,6 +328,8 @@ __global__ void __launch_bounds__(kPathThreads)
   __shared__ int s_cand[MEDUSA_MAX_NODES];
   __shared__ int s_best;
   __shared__ int s_bad;
+  __shared__ int s_src[MEDUSA_MAX_HEADS + 1];  // kept branch's cache slots (compaction)
+  __shared__ int s_keep, s_prefix;
   const int b = blockIdx.x;
   const int i = threadIdx.x;
   if (i == 0) {
@@ -487,7 +490,27 @@ __global__ void __launch_bounds__(kPathThreads)
     accepted_tokens[o + L] = s_g[best];
     accept_len[b] = L;
     bonus[b] = s_g[best];
+    if (ca.Kc != nullptr) {
+      // the kept branch's cache slots, for the compaction below
+      const int P = ca.prefix_len[b];
+      bool ok = P >= 0;
+      for (int j = best; j >= 0; j = s_parent[j]) {
+        const long long slot = (long long)P + j;
+        if (slot >= ca.cap) ok = false;
+        s_src[s_depth[j]] = (int)slot;
+      }
+      s_keep = ok ? L : -1;
+      s_prefix = P;
+      if (!ok) report(status, MEDUSA_ERR_DEVICE_CHECK);
+    }
   }
+  if (ca.Kc == nullptr) return;
+  // Compaction of the kept branch by the same block (one launch less than a
+  // separate compaction call): for j = 0..L, slot P + j <- slot P + node_j.
+  __syncthreads();
+  if (s_keep < 0) return;
+  extern __shared__ __align__(16) uint4 stage[];
+  compact_sequence(ca, b, s_prefix, s_keep, s_src, max_depth + 1, stage);
 }
 
 // CTAs for the persistent row kernel: as many as stay resident, fewer when
@@ -526,7 +549,7 @@ medusa_status_t verify_path_from_parts(const RowPart* part, int n_chunks,
   launch(verify_path_kernel<__nv_bfloat16>, B, kPathThreads, 0, stream, nullptr, hidden, lm_head, d,
          part, n_chunks, n_chunks, 1, path_threads_per_node(N, n_chunks), nullptr, cand_ids,
          tree.parent, tree.depth, N, tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta,
-         accept_len, accepted_nodes, accepted_tokens, bonus, status);
+         accept_len, accepted_nodes, accepted_tokens, bonus, status, CompactArgs{});
   return check_launch("verify_path");
 }
 
@@ -648,7 +671,7 @@ medusa_status_t verify_from_records(const RowPart* records, int G, const float* 
   launch(verify_path_kernel<float>, B, kPathThreads, 0, stream, nullptr, nullptr, nullptr, 0,
          records, G, 1, (long long)B * N, path_threads_per_node(N, G), cand_logit, cand_ids,
          tree.parent, tree.depth, N, tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta,
-         accept_len, accepted_nodes, accepted_tokens, bonus, status);
+         accept_len, accepted_nodes, accepted_tokens, bonus, status, CompactArgs{});
   return check_launch("verify_path");
 }
 
@@ -661,8 +684,19 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
                               const medusa_tree_t& tree, int B, int V, medusa_accept_t mode,
                               float temperature, float eps, float delta, int32_t* accept_len,
                               int32_t* accepted_nodes, int32_t* accepted_tokens, int32_t* bonus,
-                              void* ws, int32_t* status, cudaStream_t stream) {
+                              void* ws, int32_t* status, cudaStream_t stream,
+                              const CompactArgs& ca, size_t ca_smem) {
   const int N = tree.n_nodes;
+  // the compaction tail's staging memory
+  if (ca_smem > 48 * 1024) {
+    const cudaError_t e =
+        dt == MEDUSA_BF16
+            ? cudaFuncSetAttribute(verify_path_kernel<__nv_bfloat16>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ca_smem)
+            : cudaFuncSetAttribute(verify_path_kernel<float>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ca_smem);
+    if (e != cudaSuccess) return fail(MEDUSA_ERR_CUDA, "cudaFuncSetAttribute(verify_path) failed");
+  }
   const int n_chunks = (V + kVChunk - 1) / kVChunk;
   RowPart* part = static_cast<RowPart*>(ws);
   const bool typical = mode == MEDUSA_ACCEPT_TYPICAL;
@@ -682,10 +716,10 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
     }
     medusa_status_t st = check_launch("verify_rows");
     if (st != MEDUSA_OK) return st;
-    launch(verify_path_kernel<__nv_bfloat16>, B, kPathThreads, 0, stream, lg, nullptr, nullptr, 0,
-           part, n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N,
+    launch(verify_path_kernel<__nv_bfloat16>, B, kPathThreads, ca_smem, stream, lg, nullptr, nullptr,
+           0, part, n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N,
            tree.max_depth, V, typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes,
-           accepted_tokens, bonus, status);
+           accepted_tokens, bonus, status, ca);
     return check_launch("verify_path");
   }
   const float* lg = static_cast<const float*>(logits);
@@ -700,10 +734,10 @@ medusa_status_t verify_accept(const void* logits, medusa_dtype_t dt, const int32
   }
   medusa_status_t st = check_launch("verify_rows");
   if (st != MEDUSA_OK) return st;
-  launch(verify_path_kernel<float>, B, kPathThreads, 0, stream, lg, nullptr, nullptr, 0, part,
+  launch(verify_path_kernel<float>, B, kPathThreads, ca_smem, stream, lg, nullptr, nullptr, 0, part,
          n_chunks, n_chunks, 1, tpn, nullptr, cand_ids, tree.parent, tree.depth, N, tree.max_depth,
          V, typical ? 1 : 0, inv_T, eps, delta, accept_len, accepted_nodes, accepted_tokens, bonus,
-         status);
+         status, ca);
   return check_launch("verify_path");
 }
 

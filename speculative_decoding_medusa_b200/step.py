@@ -6,6 +6,7 @@ from __future__ import annotations
 from typing import Optional
 
 import torch
+from torch.cuda import nvtx
 
 from . import _lib as M
 
@@ -47,20 +48,25 @@ class DecodeVerifyStep:
     def run(self, h, W1, b1, W2, root_tok, q, k_new, v_new, Kc, Vc, prefix_len, verify_logits,
             stream=None) -> None:
         """Enqueue one step on ``stream``.  Kc/Vc/prefix_len are updated in place
-        (tree K/V written, then the kept branch compacted, prefix advanced)."""
-        M.medusa_heads_topk(h, W1, b1, W2, self.kmax, self.topk_ids, self.topk_vals,
-                            self.head_logits, self.ws_heads, self.status, stream)
-        M.medusa_tree_build(self.tree, root_tok, self.topk_ids, prefix_len, self.cand_ids,
-                            self.pos_ids, self.anc_mask, self.retrieve, self.status, stream)
-        M.medusa_tree_attention(q, k_new, v_new, Kc, Vc, prefix_len, self.anc_mask,
-                                self.max_prefix, self.attn_out, None, self.ws_attn, self.status,
-                                stream)
-        M.medusa_verify_accept(verify_logits, self.cand_ids, self.tree, self.accept_len,
-                               self.accepted_nodes, self.accepted_tokens, self.bonus, self.mode,
-                               self.temperature, self.eps, self.delta, self.ws_verify,
-                               self.status, stream)
-        M.medusa_kv_compact(Kc, Vc, prefix_len, self.accepted_nodes, self.accept_len,
-                            self.compact_src, self.status, stream)
+        (tree K/V written, then the kept branch compacted, prefix advanced).
+        Each call sits in an NVTX range of its name (for ncu --nvtx filters)."""
+        with nvtx.range("medusa_heads_topk"):
+            M.medusa_heads_topk(h, W1, b1, W2, self.kmax, self.topk_ids, self.topk_vals,
+                                self.head_logits, self.ws_heads, self.status, stream)
+        with nvtx.range("medusa_tree_build"):
+            M.medusa_tree_build(self.tree, root_tok, self.topk_ids, prefix_len, self.cand_ids,
+                                self.pos_ids, self.anc_mask, self.retrieve, self.status, stream)
+        with nvtx.range("medusa_tree_attention"):
+            M.medusa_tree_attention(q, k_new, v_new, Kc, Vc, prefix_len, self.anc_mask,
+                                    self.max_prefix, self.attn_out, None, self.ws_attn,
+                                    self.status, stream)
+        with nvtx.range("medusa_verify_accept_compact"):
+            M.medusa_verify_accept_compact(verify_logits, self.cand_ids, self.tree,
+                                           self.accept_len, self.accepted_nodes,
+                                           self.accepted_tokens, self.bonus, Kc, Vc, prefix_len,
+                                           self.compact_src, self.mode, self.temperature,
+                                           self.eps, self.delta, self.ws_verify, self.status,
+                                           stream)
 
 
 class DecodeLoop:

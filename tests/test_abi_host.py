@@ -144,6 +144,26 @@ def test_attention_verify_compact_checks(L):
     assert compact(dh=4) == 2                     # 8-byte rows are not 16-byte multiples
     assert compact(Kc=v(1032)) == 8
 
+    # verification with the compaction: the verification's checks, then the
+    # compaction's, then the workspace
+    def fused(logits=v(1024), mode=0, Kc=v(1024), kv_dt=0, dh=128, ws=v(4096), ws_bytes=1 << 20):
+        return L.medusa_verify_accept_compact(logits, 0, v(1024), ctypes.byref(tree), 1, 1000,
+                                              mode, 1.0, 0.09, 0.3, v(1024), v(1024), v(1024),
+                                              v(1024), Kc, v(1024), kv_dt, v(1024), 2, dh, 100,
+                                              v(1024), ws, ws_bytes, None, None)
+
+    assert fused(logits=None) == 1
+    assert fused(mode=3) == 1
+    assert fused(logits=v(1032), Kc=None) == 8     # the verification's check comes first
+    assert fused(Kc=None) == 1
+    assert fused(kv_dt=7) == 1
+    assert fused(dh=4) == 2
+    assert fused(Kc=v(1032)) == 8
+    assert fused(ws=None) == 7
+    assert fused(ws_bytes=16) == 7
+    assert fused(ws=v(4100)) == 7                  # workspace not 256-byte aligned
+    assert fused(kv_dt=1, dh=8192) == 3            # (max_depth + 1) rows of K and V > 96 KB
+
     def wait(flag=v(1024), budget=1000, status=v(2048)):
         return L.medusa_wait_flag(flag, 1, budget, status, None)
 
