@@ -2,7 +2,8 @@
 """Benchmark of the Medusa decode-verify step on B200.
 
 One step = heads + top-k, tree build, tree attention, verify/accept and KV
-compaction for one batch (four C-ABI calls: the last two are one).  Default workload: the
+compaction for one batch (three C-ABI calls: heads with the tree build,
+attention, verification with the compaction).  Default workload: the
 Llama-3-8B-shaped configuration (batch 8, hidden 4096, vocab 128256, 4 heads,
 64-node sparse tree, GQA 32/8 heads of 128, ragged prefixes 4096..8192, bf16,
 greedy acceptance).  Inputs are seeded synthetic data of those shapes; every
@@ -36,9 +37,9 @@ import torch  # noqa: E402
 
 METRIC = "Medusa decode-verify steps/s (heads+tree attn+accept); % of HBM roofline"
 UNIT = "steps/s"
-KERNELS_PER_STEP = 9  # W1 GEMM, W2 GEMM, top-k merge, tree build, attention counters,
-#                       attention, attention exact pass (empty list: reads a count),
-#                       verify rows, verify path with the KV compaction
+KERNELS_PER_STEP = 9  # stream-K flags, W1 GEMM, W2 GEMM, top-k merge with the tree
+#                       build, attention counters, attention, attention exact pass (empty
+#                       list: reads a count), verify rows, verify path with the KV compaction
 
 
 def _peaks():
@@ -577,22 +578,21 @@ def main():
                      att["v_new"], att["Kc"], att["Vc"], att["prefix_len"], logits)
             return
         evs[0].record(stream)
-        M.medusa_heads_topk(hin["h"], hin["W1"], hin["b1"], hin["W2"], w.kmax, step.topk_ids,
-                            step.topk_vals, None, step.ws_heads, step.status)
+        M.medusa_heads_topk_tree(hin["h"], hin["W1"], hin["b1"], hin["W2"], w.kmax, step.topk_ids,
+                                 step.topk_vals, tree, root, att["prefix_len"], step.cand_ids,
+                                 step.pos_ids, step.anc_mask, step.retrieve, None, step.ws_heads,
+                                 step.status)
         evs[1].record(stream)
-        M.medusa_tree_build(tree, root, step.topk_ids, att["prefix_len"], step.cand_ids,
-                            step.pos_ids, step.anc_mask, step.retrieve, step.status)
-        evs[2].record(stream)
         M.medusa_tree_attention(att["q"], att["k_new"], att["v_new"], att["Kc"], att["Vc"],
                                 att["prefix_len"], step.anc_mask, w.ctx_hi, step.attn_out, None,
                                 step.ws_attn, step.status)
-        evs[3].record(stream)
+        evs[2].record(stream)
         M.medusa_verify_accept_compact(logits, step.cand_ids, tree, step.accept_len,
                                        step.accepted_nodes, step.accepted_tokens, step.bonus,
                                        att["Kc"], att["Vc"], att["prefix_len"], step.compact_src,
                                        step.mode, w.temperature, w.eps, w.delta, step.ws_verify,
                                        step.status)
-        evs[4].record(stream)
+        evs[3].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         one_step()
@@ -625,11 +625,11 @@ def main():
     ms_step = ms_total / args.steps
     # stage breakdown from a separate, untimed pass with events between the calls
     n_stage = min(args.steps, 50)
-    stage_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_stage)]
+    stage_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_stage)]
     for k in range(n_stage):
         one_step(stage_evs[k])
     torch.cuda.synchronize()
-    names = ["heads_topk", "tree_build", "tree_attention", "verify_accept_compact"]
+    names = ["heads_topk_tree", "tree_attention", "verify_accept_compact"]
     stages = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in stage_evs) * 1e3
               for i, n in enumerate(names)}  # us
     assert int(step.status.item()) == 0
@@ -721,10 +721,10 @@ def main():
         ms_e2e = float(tt.item())
     e2e_value = world * n_e2e / (ms_e2e / 1e3)
 
-    # ---- roofline of the dominant call (heads_topk: W1 + W2 weight stream) ----
+    # ---- roofline of the dominant call (heads + top-k with the tree build: W1 + W2 weight stream) ----
     hbm_peak, _, peak_kind = _peaks()
     ab = algorithmic_bytes(w, prefix_list, N)
-    heads_gbs = ab["heads"] / (stages["heads_topk"] * 1e-6) / 1e9
+    heads_gbs = ab["heads"] / (stages["heads_topk_tree"] * 1e-6) / 1e9
     traffic, traffic_src = heads_traffic(ab["heads"])
     step_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
     value = world * args.steps / (ms_total / 1e3)
@@ -763,7 +763,7 @@ def main():
             "step_bytes": ab["total"],
             "stages_us": stages,
             "step_us": step_us,
-            "roofline": {"bound": "hbm", "kernel": "medusa_heads_topk (W1 GEMM + W2 GEMM + top-k merge)",
+            "roofline": {"bound": "hbm", "kernel": "medusa_heads_topk_tree (W1 GEMM + W2 GEMM + top-k merge with the tree build)",
                          "achieved": heads_gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": heads_gbs / hbm_peak, "traffic": traffic,
                          "traffic_source": "ncu dram bytes ratio, " + traffic_src,

@@ -15,8 +15,9 @@
  *
  * Around them: medusa_lmhead_verify (the verification from the nodes' hidden
  * states, lm_head fused), medusa_next_step (inputs of the next step),
- * medusa_sample_bonus (a drawn bonus token), medusa_verify_accept_compact
- * (the last two calls in one), medusa_tree_from_accuracies
+ * medusa_sample_bonus (a drawn bonus token), medusa_heads_topk_tree and
+ * medusa_verify_accept_compact (the first two and the last two calls, each
+ * pair in one), medusa_tree_from_accuracies
  * (the sparse tree of the most accurate combinations, host only), the
  * vocabulary-sharding calls (medusa_topk_merge, medusa_verify_records,
  * medusa_verify_from_records), medusa_verify_accept_noalloc and
@@ -192,6 +193,31 @@ MEDUSA_API medusa_status_t medusa_tree_build(const medusa_tree_t* tree, const in
                                   int32_t* pos_ids, uint32_t* anc_mask,
                                   int32_t* retrieve, int32_t* dev_status,
                                   void* stream);
+
+/* ------------------------------------------------------------------------
+ * medusa_heads_topk_tree
+ *
+ * medusa_heads_topk followed by medusa_tree_build of its top-k lists, in the
+ * launches of medusa_heads_topk alone: the thread block that finishes the
+ * last of a sequence's K lists builds that sequence's candidates (the
+ * sections cited at the two calls).  Every output equals that of the two
+ * calls made one after the other on the same stream, with the tree build's
+ * K and kmax the heads'.
+ *
+ * Arguments: those of medusa_heads_topk, then those of medusa_tree_build
+ *   (tree, root_tok [B], prefix_len [B]; cand_ids, pos_ids [B, N]; anc_mask
+ *   [N, ceil(N/32)]; retrieve [n_leaves, max_depth+1]).  Workspace as
+ *   medusa_heads_topk.
+ * Host checks: medusa_heads_topk's arguments, then the tree's (as
+ *   medusa_tree_build), then the workspace; nothing is launched on an error.
+ * Device checks: medusa_tree_build's.
+ * ---------------------------------------------------------------------- */
+MEDUSA_API medusa_status_t medusa_heads_topk_tree(
+    const void* h, const void* W1, const void* b1, const void* W2, medusa_dtype_t dt, int B, int d,
+    int V, int K, int kmax, int32_t* topk_ids, float* topk_vals, float* logits, void* ws,
+    size_t ws_bytes, const medusa_tree_t* tree, const int32_t* root_tok, const int32_t* prefix_len,
+    int32_t* cand_ids, int32_t* pos_ids, uint32_t* anc_mask, int32_t* retrieve, int32_t* dev_status,
+    void* stream);
 
 /* ------------------------------------------------------------------------
  * medusa_tree_attention

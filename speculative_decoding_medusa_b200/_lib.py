@@ -36,7 +36,7 @@ EXPORTS = (
     "medusa_tree_build",
     "medusa_tree_attention_workspace_size", "medusa_tree_attention",
     "medusa_verify_accept_workspace_size", "medusa_verify_accept",
-    "medusa_kv_compact", "medusa_verify_accept_compact", "medusa_verify_accept_noalloc",
+    "medusa_kv_compact", "medusa_verify_accept_compact", "medusa_heads_topk_tree", "medusa_verify_accept_noalloc",
     "medusa_lmhead_verify_workspace_size", "medusa_lmhead_verify", "medusa_next_step",
     "medusa_tree_from_accuracies", "medusa_sample_bonus", "medusa_topk_merge",
     "medusa_verify_records_workspace_size", "medusa_verify_records", "medusa_verify_from_records",
@@ -78,6 +78,10 @@ def lib() -> ctypes.CDLL:
     L.medusa_heads_topk_workspace_size.argtypes = [_I] * 5 + [_I]
     L.medusa_heads_topk.restype = _I
     L.medusa_heads_topk.argtypes = [_V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _V, _V, _V, _V, _Z, _V, _V]
+    L.medusa_heads_topk_tree.restype = _I
+    L.medusa_heads_topk_tree.argtypes = [_V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _V, _V, _V, _V, _Z,
+                                         ctypes.POINTER(medusa_tree_t), _V, _V, _V, _V, _V, _V, _V,
+                                         _V]
     L.medusa_tree_build.restype = _I
     L.medusa_tree_build.argtypes = [ctypes.POINTER(medusa_tree_t), _V, _V, _I, _I, _V, _I,
                                     _V, _V, _V, _V, _V, _V]
@@ -212,6 +216,27 @@ def medusa_heads_topk(h, W1, b1, W2, kmax: int, topk_ids, topk_vals, logits=None
     _check(lib().medusa_heads_topk(_p(h), _p(W1), _p(b1), _p(W2), dt, B, d, V, K, kmax,
                                    _p(topk_ids), _p(topk_vals), _p(logits), _p(ws), ws.numel(),
                                    _p(dev_status), _stream(stream)))
+
+
+def medusa_heads_topk_tree(h, W1, b1, W2, kmax: int, topk_ids, topk_vals, tree: Tree, root_tok,
+                           prefix_len, cand_ids, pos_ids, anc_mask, retrieve, logits=None,
+                           ws=None, dev_status=None, stream=None) -> None:
+    """medusa_heads_topk, then medusa_tree_build of its lists, in the heads'
+    launches."""
+    for t, n in ((h, "h"), (W1, "W1"), (b1, "b1"), (W2, "W2"), (topk_ids, "topk_ids"),
+                 (topk_vals, "topk_vals")):
+        _req(t, n)
+    B, d = h.shape
+    K, V, _ = W2.shape
+    dt = _dt(W2)
+    if ws is None:
+        ws = workspace(medusa_heads_topk_workspace_size(B, d, V, K, kmax, dt), h.device)
+    ct = tree.c()
+    _check(lib().medusa_heads_topk_tree(_p(h), _p(W1), _p(b1), _p(W2), dt, B, d, V, K, kmax,
+                                        _p(topk_ids), _p(topk_vals), _p(logits), _p(ws),
+                                        ws.numel(), ctypes.byref(ct), _p(root_tok),
+                                        _p(prefix_len), _p(cand_ids), _p(pos_ids), _p(anc_mask),
+                                        _p(retrieve), _p(dev_status), _stream(stream)))
 
 
 def medusa_tree_build(tree: Tree, root_tok, topk_ids, prefix_len, cand_ids, pos_ids, anc_mask,

@@ -81,10 +81,11 @@ size_t medusa_heads_topk_workspace_size(int B, int d, int V, int K, int kmax, me
   return medusa::heads_topk_workspace_size(B, d, V, K, kmax, dt);
 }
 
-medusa_status_t medusa_heads_topk(const void* h, const void* W1, const void* b1, const void* W2,
-                                  medusa_dtype_t dt, int B, int d, int V, int K, int kmax,
-                                  int32_t* topk_ids, float* topk_vals, float* logits, void* ws,
-                                  size_t ws_bytes, int32_t* dev_status, void* stream) {
+namespace {
+
+medusa_status_t check_heads_args(const void* h, const void* W1, const void* b1, const void* W2,
+                                 medusa_dtype_t dt, int B, int d, int V, int K, int kmax,
+                                 int32_t* topk_ids, float* topk_vals) {
   if (!h || !W1 || !b1 || !W2 || !topk_ids || !topk_vals)
     return fail(MEDUSA_ERR_INVALID_ARG, "heads_topk: null pointer");
   if (!valid_dtype(dt)) return fail(MEDUSA_ERR_INVALID_ARG, "heads_topk: bad dtype");
@@ -99,11 +100,55 @@ medusa_status_t medusa_heads_topk(const void* h, const void* W1, const void* b1,
     if (!aligned16(h) || !aligned16(W1) || !aligned16(b1) || !aligned16(W2))
       return fail(MEDUSA_ERR_ALIGNMENT, "heads_topk: inputs must be 16-byte aligned");
   }
+  return MEDUSA_OK;
+}
+
+medusa_status_t check_heads_ws(int B, int d, int V, int K, int kmax, medusa_dtype_t dt,
+                               const void* ws, size_t ws_bytes) {
   const size_t need = medusa::heads_topk_workspace_size(B, d, V, K, kmax, dt);
   if (ws == nullptr || ws_bytes < need || !aligned256(ws))
     return fail(MEDUSA_ERR_WORKSPACE, "heads_topk: workspace null, misaligned or too small");
+  return MEDUSA_OK;
+}
+
+}  // namespace
+
+medusa_status_t medusa_heads_topk(const void* h, const void* W1, const void* b1, const void* W2,
+                                  medusa_dtype_t dt, int B, int d, int V, int K, int kmax,
+                                  int32_t* topk_ids, float* topk_vals, float* logits, void* ws,
+                                  size_t ws_bytes, int32_t* dev_status, void* stream) {
+  medusa_status_t st = check_heads_args(h, W1, b1, W2, dt, B, d, V, K, kmax, topk_ids, topk_vals);
+  if (st != MEDUSA_OK) return st;
+  st = check_heads_ws(B, d, V, K, kmax, dt, ws, ws_bytes);
+  if (st != MEDUSA_OK) return st;
   return medusa::heads_topk(h, W1, b1, W2, dt, B, d, V, K, kmax, topk_ids, topk_vals, logits, ws,
                             dev_status, static_cast<cudaStream_t>(stream));
+}
+
+medusa_status_t medusa_heads_topk_tree(const void* h, const void* W1, const void* b1,
+                                       const void* W2, medusa_dtype_t dt, int B, int d, int V,
+                                       int K, int kmax, int32_t* topk_ids, float* topk_vals,
+                                       float* logits, void* ws, size_t ws_bytes,
+                                       const medusa_tree_t* tree, const int32_t* root_tok,
+                                       const int32_t* prefix_len, int32_t* cand_ids,
+                                       int32_t* pos_ids, uint32_t* anc_mask, int32_t* retrieve,
+                                       int32_t* dev_status, void* stream) {
+  medusa_status_t st = check_heads_args(h, W1, b1, W2, dt, B, d, V, K, kmax, topk_ids, topk_vals);
+  if (st != MEDUSA_OK) return st;
+  // the checks of medusa_tree_build
+  st = check_tree(tree);
+  if (st != MEDUSA_OK) return st;
+  if (!root_tok || !prefix_len || !cand_ids || !pos_ids || !anc_mask || !retrieve)
+    return fail(MEDUSA_ERR_INVALID_ARG, "heads_topk_tree: null pointer");
+  if (tree->max_depth > K)
+    return fail(MEDUSA_ERR_SHAPE, "heads_topk_tree: tree deeper than K heads");
+  st = check_heads_ws(B, d, V, K, kmax, dt, ws, ws_bytes);
+  if (st != MEDUSA_OK) return st;
+  const medusa::TreeOut t{tree->parent, tree->depth, tree->rank, tree->n_nodes, tree->max_depth,
+                          tree->n_leaves, K, kmax, root_tok, prefix_len, cand_ids, pos_ids,
+                          anc_mask, retrieve, dev_status};
+  return medusa::heads_topk(h, W1, b1, W2, dt, B, d, V, K, kmax, topk_ids, topk_vals, logits, ws,
+                            dev_status, static_cast<cudaStream_t>(stream), &t);
 }
 
 medusa_status_t medusa_tree_build(const medusa_tree_t* tree, const int32_t* root_tok,

@@ -10,6 +10,7 @@
 
 #include "../../include/medusa.h"
 #include "kv_compact.cuh"
+#include "tree_build.cuh"
 
 namespace medusa {
 
@@ -44,7 +45,7 @@ size_t heads_topk_workspace_size(int B, int d, int V, int K, int kmax, medusa_dt
 medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const void* W2,
                            medusa_dtype_t dt, int B, int d, int V, int K, int kmax,
                            int32_t* topk_ids, float* topk_vals, float* logits, void* ws,
-                           int32_t* status, cudaStream_t stream);
+                           int32_t* status, cudaStream_t stream, const TreeOut* tree = nullptr);
 
 medusa_status_t tree_build(const medusa_tree_t& tree, const int32_t* root_tok,
                            const int32_t* topk_ids, int K, int kmax, const int32_t* prefix_len,

@@ -14,7 +14,9 @@
 //      list, which joins a running best list per (head, sequence) that the
 //      CTA keeps in shared memory across its tiles (one list per tile when
 //      those lists do not fit).  Tiles are handed out by an atomic counter.
-//   3. topk_merge: per (sequence, head), the best kmax of all the lists.
+//   3. topk_merge: per (sequence, head), the best kmax of all the lists;
+//      when a tree is given, the cluster that completes a sequence's K lists
+//      also builds that sequence's candidate tree.
 // The weights are the only large operand (K*(d^2 + V*d) bf16): every CTA
 // streams 128-row weight tiles through a TMA -> shared memory -> tcgen05.mma
 // pipeline; the batch sits in the MMA's N dimension (weight rows fill M=128).
@@ -32,6 +34,7 @@
 
 #include "abi_internal.h"
 #include "common.cuh"
+#include "tree_build.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -67,7 +70,7 @@ struct GemmParams {
   // (tile, k-block) sequence; 0 = whole tiles round-robin
   int kpc;
   float* sk_part;  // [grid][kTileM][NB] fp32 partial of a CTA's leading tile tail
-  int* sk_flag;    // [grid] 1 once that partial is written (zeroed before the launch)
+  int* sk_flag;    // [grid] 1 once that partial is written (zeroed by a kernel before the launch)
   int sk_grid;     // CTAs of a stream-K launch
   // second GEMM: tiles handed out by this counter (tiles past the first
   // grid-full are claimed one at a time); the first GEMM zeroes it.  Null:
@@ -191,8 +194,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   grid_dep_launch();
   // the first GEMM resets the second GEMM's tile counter (the second GEMM
   // reads it only after waiting for this kernel)
-  if (MODE == kModeW1 && p.tile_counter != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
-    *p.tile_counter = 0;
+  // (and the merge's per-sequence row counts that follow it)
+  if (MODE == kModeW1 && p.tile_counter != nullptr && blockIdx.x == 0 && threadIdx.x <= p.B)
+    p.tile_counter[threadIdx.x] = 0;
   using L = GemmSmem<NB, S>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -484,6 +488,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// The first GEMM's stream-K flags, cleared before each call by a kernel (so
+// that the launches stay chained by programmatic dependent launch, which a
+// memset node would break).
+__global__ void __launch_bounds__(256) heads_flags_zero_kernel(int* __restrict__ flags, int n) {
+  grid_dep_wait();
+  grid_dep_launch();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) flags[e] = 0;
+}
+
 // ----------------------------------------------------------------------------
 // top-k merge: best kmax of C candidates per row
 //
@@ -507,11 +520,20 @@ struct MergeLayout {
 constexpr int kMergeWarps = 8;
 constexpr int kMergeCtas = 8;    // cluster size (portable)
 constexpr int kMergeUnroll = 2;  // 32-candidate chunks each warp has in flight
+static_assert(kMergeWarps * 32 == kTreeThreads, "the merge's tail builds trees with its CTA");
+
+// The tree built by the merge's tail: rows are (sequence, head) pairs, row =
+// b * tree.K + head; seq_count[b] counts sequence b's finished rows (zero
+// before the launch).  tree.cand_ids == nullptr: no tail.
+struct MergeTree {
+  TreeOut tree;
+  int* seq_count;
+};
 
 __global__ void __cluster_dims__(kMergeCtas, 1, 1) __launch_bounds__(kMergeWarps * 32)
     topk_merge_kernel(const float* __restrict__ vals, const int32_t* __restrict__ ids, long long C,
                       int kmax, int32_t* __restrict__ out_ids, float* __restrict__ out_vals,
-                      MergeLayout lay) {
+                      MergeLayout lay, MergeTree mt) {
   grid_dep_wait();
   grid_dep_launch();
   __shared__ float sv[kMergeWarps][32];
@@ -580,6 +602,23 @@ __global__ void __cluster_dims__(kMergeCtas, 1, 1) __launch_bounds__(kMergeWarps
       out_vals[(size_t)row * kmax + lane] = rv;
     }
   }
+  if (mt.tree.cand_ids != nullptr && crank == 0) {
+    // Count this row in.  The CTA whose row completes sequence b's K lists
+    // builds b's candidate tree from them; no CTA waits for another.
+    __shared__ int s_last;
+    const int b = static_cast<int>(row / mt.tree.K);
+    if (warp == 0) {
+      __threadfence();  // this lane's list entry before the count
+      __syncwarp();
+      if (lane == 0) s_last = atomicAdd(&mt.seq_count[b], 1) == mt.tree.K - 1;
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      const int32_t* lists = out_ids + (size_t)b * mt.tree.K * kmax;
+      build_tree_sequence(mt.tree, b, [lists](int e) { return __ldcg(lists + e); }, b == 0);
+    }
+  }
   // no CTA leaves while CTA 0 may still read its shared memory
   cluster.sync();
 }
@@ -596,9 +635,12 @@ __device__ __forceinline__ float warp_sum(float x) {
 // y[b][k][j] = h[b][j] + SiLU(W1[k][j] . h[b] + b1[k][j]); one warp per j.
 __global__ void __launch_bounds__(256)
     heads_f32_w1_kernel(const float* __restrict__ h, const float* __restrict__ W1,
-                        const float* __restrict__ b1, int B, int d, int K, float* __restrict__ y) {
+                        const float* __restrict__ b1, int B, int d, int K, float* __restrict__ y,
+                        int* __restrict__ seq_count) {
   grid_dep_wait();
   grid_dep_launch();
+  // the merge's per-sequence row counts
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < B) seq_count[threadIdx.x] = 0;
   const int k = blockIdx.y;
   const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -644,7 +686,7 @@ medusa_status_t topk_merge_lists(const float* vals, const int32_t* ids, int rows
                                  float* out_vals, cudaStream_t stream) {
   const MergeLayout lay{row_stride, list_stride, list_len, id_offsets};
   launch(topk_merge_kernel, rows * kMergeCtas, kMergeWarps * 32, 0, stream, vals, ids,
-         (long long)n_lists * list_len, kmax, out_ids, out_vals, lay);
+         (long long)n_lists * list_len, kmax, out_ids, out_vals, lay, MergeTree{});
   return check_launch("topk_merge");
 }
 
@@ -726,13 +768,14 @@ HeadsWs heads_ws_layout(int B, int d, int V, int K, int kmax, medusa_dtype_t dt)
     // flag per CTA
     w.sk_part_bytes = align256((size_t)num_sms() * kTileM * round_nb(B) * 4);
     w.sk_flag_bytes = align256((size_t)num_sms() * 4);
-    // the second GEMM's tile counter
-    w.counter_bytes = 256;
+    // the second GEMM's tile counter, then the merge's row count per sequence
+    w.counter_bytes = align256((size_t)(B + 1) * 4);
     w.total = w.y_bytes + 2 * w.part_bytes + w.sk_part_bytes + w.sk_flag_bytes + w.counter_bytes;
   } else {
     w.y_bytes = align256((size_t)B * K * d * 4);
     w.part_bytes = align256((size_t)B * K * V * 4);
-    w.total = w.y_bytes + w.part_bytes;
+    w.counter_bytes = align256((size_t)B * 4);  // the merge's row count per sequence
+    w.total = w.y_bytes + w.part_bytes + w.counter_bytes;
   }
   return w;
 }
@@ -746,14 +789,17 @@ size_t heads_topk_workspace_size(int B, int d, int V, int K, int kmax, medusa_dt
 medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const void* W2,
                            medusa_dtype_t dt, int B, int d, int V, int K, int kmax,
                            int32_t* topk_ids, float* topk_vals, float* logits, void* ws,
-                           int32_t* status, cudaStream_t stream) {
+                           int32_t* status, cudaStream_t stream, const TreeOut* tree) {
   const HeadsWs w = heads_ws_layout(B, d, V, K, kmax, dt);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
+  MergeTree mt{};
   if (dt == MEDUSA_F32) {
     float* y = reinterpret_cast<float*>(wsb);
     float* z = logits != nullptr ? logits : reinterpret_cast<float*>(wsb + w.y_bytes);
+    int* seq_count = reinterpret_cast<int*>(wsb + w.y_bytes + w.part_bytes);
+    if (tree != nullptr) mt = MergeTree{*tree, seq_count};
     launch(heads_f32_w1_kernel, dim3((d + 7) / 8, K), 256, 0, stream, static_cast<const float*>(h),
-           static_cast<const float*>(W1), static_cast<const float*>(b1), B, d, K, y);
+           static_cast<const float*>(W1), static_cast<const float*>(b1), B, d, K, y, seq_count);
     medusa_status_t st = check_launch("heads_f32_w1");
     if (st != MEDUSA_OK) return st;
     launch(heads_f32_w2_kernel, dim3((V + 7) / 8, K), 256, 0, stream, y,
@@ -762,7 +808,7 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
     if (st != MEDUSA_OK) return st;
     const MergeLayout lay{(long long)V, (long long)V, V, nullptr};
     launch(topk_merge_kernel, B * K * kMergeCtas, kMergeWarps * 32, 0, stream, z, nullptr, V, kmax,
-           topk_ids, topk_vals, lay);
+           topk_ids, topk_vals, lay, mt);
     return check_launch("topk_merge");
   }
 
@@ -805,8 +851,9 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
       p1.sk_grid = (int)((total_kb + p1.kpc - 1) / p1.kpc);
       p1.sk_part = reinterpret_cast<float*>(wsb + w.y_bytes + 2 * w.part_bytes);
       p1.sk_flag = reinterpret_cast<int*>(wsb + w.y_bytes + 2 * w.part_bytes + w.sk_part_bytes);
-      if (cudaMemsetAsync(p1.sk_flag, 0, (size_t)p1.sk_grid * sizeof(int), stream) != cudaSuccess)
-        return check_launch("heads stream-K flags");
+      launch(heads_flags_zero_kernel, 1, 256, 0, stream, p1.sk_flag, p1.sk_grid);
+      const medusa_status_t zst = check_launch("heads stream-K flags");
+      if (zst != MEDUSA_OK) return zst;
     }
   }
   medusa_status_t st = launch_gemm_nb<kModeW1>(nb1, mA1, mB1, p1, stream);
@@ -832,8 +879,9 @@ medusa_status_t heads_topk(const void* h, const void* W1, const void* b1, const 
 
   const long long C = (long long)(p2.run_lists ? gemm_grid(p2) : p2.tiles_per_head) * kmax;
   const MergeLayout lay{C, C, (int)C, nullptr};
+  if (tree != nullptr) mt = MergeTree{*tree, p1.tile_counter + 1};
   launch(topk_merge_kernel, B * K * kMergeCtas, kMergeWarps * 32, 0, stream, part_vals, part_ids, C,
-         kmax, topk_ids, topk_vals, lay);
+         kmax, topk_ids, topk_vals, lay, mt);
   return check_launch("topk_merge");
 }
 

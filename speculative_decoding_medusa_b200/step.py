@@ -1,5 +1,6 @@
-"""One decode-verify step through the C ABI: buffers plus the five calls in
-order (heads + top-k, tree build, tree attention, verify/accept, KV compaction).
+"""One decode-verify step through the C ABI: buffers plus three calls in order
+(heads + top-k with the tree build, tree attention, verify/accept with the KV
+compaction; `DecodeLoop` calls its stages one by one).
 Argument marshalling only; all arithmetic runs in libmedusa_b200.so."""
 from __future__ import annotations
 
@@ -50,12 +51,11 @@ class DecodeVerifyStep:
         """Enqueue one step on ``stream``.  Kc/Vc/prefix_len are updated in place
         (tree K/V written, then the kept branch compacted, prefix advanced).
         Each call sits in an NVTX range of its name (for ncu --nvtx filters)."""
-        with nvtx.range("medusa_heads_topk"):
-            M.medusa_heads_topk(h, W1, b1, W2, self.kmax, self.topk_ids, self.topk_vals,
-                                self.head_logits, self.ws_heads, self.status, stream)
-        with nvtx.range("medusa_tree_build"):
-            M.medusa_tree_build(self.tree, root_tok, self.topk_ids, prefix_len, self.cand_ids,
-                                self.pos_ids, self.anc_mask, self.retrieve, self.status, stream)
+        with nvtx.range("medusa_heads_topk_tree"):
+            M.medusa_heads_topk_tree(h, W1, b1, W2, self.kmax, self.topk_ids, self.topk_vals,
+                                     self.tree, root_tok, prefix_len, self.cand_ids, self.pos_ids,
+                                     self.anc_mask, self.retrieve, self.head_logits,
+                                     self.ws_heads, self.status, stream)
         with nvtx.range("medusa_tree_attention"):
             M.medusa_tree_attention(q, k_new, v_new, Kc, Vc, prefix_len, self.anc_mask,
                                     self.max_prefix, self.attn_out, None, self.ws_attn,

@@ -72,6 +72,30 @@ def test_heads_topk_host_checks(L):
     assert _call_heads(L, kmax=0) == 2 and b"kmax" in L.medusa_last_error()
 
 
+def test_heads_topk_tree_host_checks(L):
+    """The fused heads + tree call: the heads' checks, then the tree's, then
+    the workspace."""
+    v = ctypes.c_void_p
+    good = _lib.medusa_tree_t(9, 2, 6, 1024, 1024, 1024)
+
+    def call(h=1024, K=2, t=good, root=1024, ws=4096, ws_bytes=1 << 20):
+        return L.medusa_heads_topk_tree(v(h) if h else None, v(1024), v(1024), v(1024), 0, 1, 64,
+                                        100, K, 3, v(1024), v(1024), None,
+                                        v(ws) if ws else None, ws_bytes, ctypes.byref(t),
+                                        v(root) if root else None, v(1024), v(1024), v(1024),
+                                        v(1024), v(1024), None, None)
+
+    assert call(h=None) == 1
+    assert call(K=17) == 2
+    assert call(h=None, t=_lib.medusa_tree_t(0, 0, 1, 1024, 1024, 1024)) == 1  # heads first
+    assert call(t=_lib.medusa_tree_t(0, 0, 1, 1024, 1024, 1024)) == 2
+    assert call(root=None) == 1
+    assert call(K=1) == 2                          # tree deeper than K heads
+    assert call(root=None, ws=None) == 1           # the tree before the workspace
+    assert call(ws=None) == 7
+    assert call(ws_bytes=16) == 7
+
+
 def test_tree_checks(L):
     good = _lib.medusa_tree_t(9, 2, 6, 1024, 1024, 1024)
     v = ctypes.c_void_p
