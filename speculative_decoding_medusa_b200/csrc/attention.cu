@@ -171,7 +171,7 @@ struct AttnSmem {
   static constexpr int kBarOff = kVOff + kAttnStages * kKVBytes;
   // kv_full[S], kv_empty[S], v_ready[S], q_full[2], s_full[2], p_full[2], p_empty[2], drain,
   // copy_read[S]
-  static constexpr int kNumBars = 4 * kAttnStages + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 4 * kAttnStages + 2 + 2 + 2 + 2 + 1 + 1;  // ..., exit
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kInfoOff = kMiscOff + 16;           // int info[kAttnStages]
   static constexpr int kAuxOff = kInfoOff + 16;  // int {bh, cache row0, segment, -}[kAttnStages]
@@ -527,6 +527,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 0) {
     const bool ok = build_schedule(p, cumT, pref);
     if (lane == 0) *sched_ok = ok ? 1 : 0;
+    __syncwarp();
   }
   __syncthreads();
   if (!*sched_ok) {
@@ -552,6 +553,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // [stage] a tree tile's cache stores have read the stage (one barrier per
   // stage: the next copy from a stage needs every converter thread past this one)
   uint64_t* copy_read = drain + 1;
+  uint64_t* exit_bar = copy_read + kAttnStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   int* stage_info = reinterpret_cast<int*>(smem + L::kInfoOff);
@@ -571,6 +573,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     mbar_init(drain, 1);
     for (int i = 0; i < kAttnStages; ++i) mbar_init(&copy_read[i], 1);
+    mbar_init(exit_bar, kAttnThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -579,6 +582,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
+  // every warp reconverges first: lane 0 of some warps ran a role alone
+  __syncwarp();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
@@ -1072,9 +1077,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   }
 
+  // TMEM is released once every thread is past its last TMEM access: each
+  // thread arrives on the exit barrier (an mbarrier counts threads, however
+  // the warps' lanes diverged in their roles) and warp 1 waits for all.
   tc_fence_before();
-  __syncthreads();
+  mbar_arrive(exit_bar);
   if (warp == 1) {
+    int no_abort = 0;
+    mbar_wait_bounded(exit_bar, 0, &no_abort, p.status);
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, kAttnTmemCols);
   }

@@ -163,8 +163,8 @@ struct GemmSmem {
   static constexpr int kAOff = 0;
   static constexpr int kBOff = S * kABytes;
   static constexpr int kBarOff = kBOff + S * kBBytes;
-  // full[S], empty[S], tfull[2], tempty[2], drain, epilogue, ring[kTileRing]
-  static constexpr int kNumBars = 2 * S + 6 + kTileRing;
+  // full[S], empty[S], tfull[2], tempty[2], drain, epilogue, ring[kTileRing], exit
+  static constexpr int kNumBars = 2 * S + 7 + kTileRing;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kRingOff = kMiscOff + 16;  // [kTileRing] claimed tile ids
   // per-warp sorted lists of the W2 epilogue: [4 quads][8 sequences][32] (value, index)
@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain = bars + 2 * S + 4;
   uint64_t* epi = bars + 2 * S + 5;
   uint64_t* ring_bar = bars + 2 * S + 6;
+  uint64_t* exit_bar = ring_bar + kTileRing;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   int* ring = reinterpret_cast<int*>(smem + L::kRingOff);
@@ -230,6 +231,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mbar_init(drain, 1);
     mbar_init(epi, 128);
     for (int i = 0; i < kTileRing; ++i) mbar_init(&ring_bar[i], 1);
+    mbar_init(exit_bar, kGemmThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -238,6 +240,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
+  // every warp reconverges first: lane 0 of some warps ran a role alone
+  __syncwarp();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
@@ -352,12 +356,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (; epi_ok && seg.next(tile, kb0, kb1); ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
-      if (!mbar_wait_bounded(&tfull[acc], aph, abort_flag, p.status)) break;
-      tc_fence_after();
       const int head = tile / p.tiles_per_head;
       const int tile_in_head = tile - head * p.tiles_per_head;
       const int r = tile_in_head * kTileM + row;  // row within the head
       const bool valid = r < p.rows_per_head;
+      // The first GEMM's epilogue inputs (bias, residual h of the first 16
+      // sequences) do not depend on the MMA: their loads are issued before
+      // the wait for it.
+      float pre_bias = 0.f;
+      float pre_h[16];
+      if (MODE == kModeW1 && kb0 == 0 && valid) {
+        pre_bias = __bfloat162float(p.b1[(size_t)head * p.d + r]);
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          pre_h[t] = t < p.B ? __bfloat162float(p.h[(size_t)t * p.d + r]) : 0.f;
+      }
+      if (!mbar_wait_bounded(&tfull[acc], aph, abort_flag, p.status)) break;
+      tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * NB;
       if (MODE == kModeW1 && kb0 > 0) {
         // stream-K: the tail of a tile that an earlier CTA finishes.  This
@@ -405,13 +420,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (MODE == kModeW1) {
           if (valid) {
-            const float bias = __bfloat162float(p.b1[(size_t)head * p.d + r]);
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
               const int b = c0 + t;
               if (b < p.B) {
-                const float u = v[t] + bias;
-                const float y = __bfloat162float(p.h[(size_t)b * p.d + r]) + u / (1.0f + expf(-u));
+                const float u = v[t] + pre_bias;
+                const float hb = c0 == 0 ? pre_h[t] : __bfloat162float(p.h[(size_t)b * p.d + r]);
+                const float y = hb + u / (1.0f + expf(-u));
                 const __nv_bfloat16 hi = __float2bfloat16_rn(y);
                 const __nv_bfloat16 lo = __float2bfloat16_rn(y - __bfloat162float(hi));
                 const size_t base = ((size_t)head * 2 * p.B + 2 * b) * p.d + r;
@@ -480,9 +495,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
 
+  // TMEM is released once every thread is past its last TMEM access: each
+  // thread arrives on the exit barrier (an mbarrier counts threads, however
+  // the warps' lanes diverged in their roles) and warp 1 waits for all.
   tc_fence_before();
-  __syncthreads();
+  mbar_arrive(exit_bar);
   if (warp == 1) {
+    int no_abort = 0;
+    mbar_wait_bounded(exit_bar, 0, &no_abort, p.status);
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols<NB>());
   }
@@ -611,6 +632,7 @@ __global__ void __cluster_dims__(kMergeCtas, 1, 1) __launch_bounds__(kMergeWarps
       __threadfence();  // this lane's list entry before the count
       __syncwarp();
       if (lane == 0) s_last = atomicAdd(&mt.seq_count[b], 1) == mt.tree.K - 1;
+      __syncwarp();
     }
     __syncthreads();
     if (s_last) {

@@ -66,8 +66,8 @@ struct LmSmem {
   static constexpr int kRedOff = kBOff + kLmStages * kBBytes;   // RowPart red[4][256]
   static constexpr int kScrOff = kRedOff + 4 * kLmHalf * 16;    // float [4][32][33]
   static constexpr int kBarOff = kScrOff + 4 * 32 * 33 * 4;
-  // full[S], empty[S], tfull, tempty[2], drain, epi
-  static constexpr int kNumBars = 2 * kLmStages + 5;
+  // full[S], empty[S], tfull, tempty[2], drain, epi, exit
+  static constexpr int kNumBars = 2 * kLmStages + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   uint64_t* tempty = tfull + 1;  // [half]
   uint64_t* drain = tfull + 3;
   uint64_t* epi = tfull + 4;
+  uint64_t* exit_bar = tfull + 5;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   const int warp = threadIdx.x >> 5;
@@ -190,6 +191,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     mbar_init(&tempty[1], 128);
     mbar_init(drain, 1);
     mbar_init(epi, 128);
+    mbar_init(exit_bar, kLmThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -198,6 +200,8 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
+  // every warp reconverges first: lane 0 of some warps ran a role alone
+  __syncwarp();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
@@ -429,9 +433,15 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     if (bad) report(p.status, MEDUSA_ERR_DEVICE_CHECK);
   }
 
+  // TMEM is released once every thread is past its last TMEM access: each
+  // thread arrives on the exit barrier (an mbarrier counts threads, however
+  // the warps' lanes diverged in their roles) and warp 1 waits for all.
   tc_fence_before();
-  __syncthreads();
+  mbar_arrive(exit_bar);
   if (warp == 1) {
+    int no_abort = 0;
+    mbar_wait_bounded(exit_bar, 0, &no_abort, p.status);
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, 2 * kLmHalf);
   }

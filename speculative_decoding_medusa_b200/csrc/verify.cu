@@ -507,6 +507,7 @@ __global__ void __launch_bounds__(kPathThreads)
   if (ca.Kc == nullptr) return;
   // Compaction of the kept branch by the same block (one launch less than a
   // separate compaction call): for j = 0..L, slot P + j <- slot P + node_j.
+  __syncwarp();  // warp 0 reconverges: its lane 0 ran the path alone
   __syncthreads();
   if (s_keep < 0) return;
   extern __shared__ __align__(16) uint4 stage[];

@@ -1,6 +1,7 @@
 """One decode-verify step through the C ABI: buffers plus three calls in order
 (heads + top-k with the tree build, tree attention, verify/accept with the KV
-compaction; `DecodeLoop` calls its stages one by one).
+compaction; `DecodeLoop` chains the heads with the tree build, the attention, the
+lm_head verification, the compaction and the hand-off to the next step).
 Argument marshalling only; all arithmetic runs in libmedusa_b200.so."""
 from __future__ import annotations
 
@@ -118,10 +119,10 @@ class DecodeLoop:
              prefix_len, stream=None) -> None:
         """Enqueue step ``r``.  h [B, d] bf16 and root [B] int32 are replaced
         by the next step's; Kc/Vc/prefix_len advance by the kept branch."""
-        M.medusa_heads_topk(h, W1, b1, W2, self.kmax, self.topk_ids, self.topk_vals, None,
-                            self.ws_heads, self.status, stream)
-        M.medusa_tree_build(self.tree, root, self.topk_ids, prefix_len, self.cand_ids,
-                            self.pos_ids, self.anc_mask, self.retrieve, self.status, stream)
+        M.medusa_heads_topk_tree(h, W1, b1, W2, self.kmax, self.topk_ids, self.topk_vals,
+                                 self.tree, root, prefix_len, self.cand_ids, self.pos_ids,
+                                 self.anc_mask, self.retrieve, None, self.ws_heads, self.status,
+                                 stream)
         node_hidden = base_model.forward(self.cand_ids, r)
         M.medusa_tree_attention(q, k_new, v_new, Kc, Vc, prefix_len, self.anc_mask,
                                 self.max_prefix, self.attn_out, None, self.ws_attn, self.status,
