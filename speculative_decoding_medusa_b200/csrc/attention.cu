@@ -171,13 +171,14 @@ struct AttnSmem {
   static constexpr int kBarOff = kVOff + kAttnStages * kKVBytes;
   // kv_full[S], kv_empty[S], v_ready[S], q_full[2], s_full[2], p_full[2], p_empty[2], drain,
   // copy_read[S]
-  static constexpr int kNumBars = 4 * kAttnStages + 2 + 2 + 2 + 2 + 1 + 1;  // ..., exit
+  static constexpr int kNumBars = 4 * kAttnStages + 2 + 2 + 2 + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kInfoOff = kMiscOff + 16;           // int info[kAttnStages]
   static constexpr int kAuxOff = kInfoOff + 16;  // int {bh, cache row0, segment, -}[kAttnStages]
   static constexpr int kCumOff = kAuxOff + 32;             // int cumT[kAttnMaxB + 1]
   static constexpr int kPrefOff = kCumOff + (kAttnMaxB + 1) * 4;  // int P[kAttnMaxB]
-  static constexpr int kBytes = kPrefOff + kAttnMaxB * 4;
+  static constexpr int kExitOff = (kPrefOff + kAttnMaxB * 4 + 7) & ~7;  // exit barrier
+  static constexpr int kBytes = kExitOff + 8;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
@@ -553,7 +554,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // [stage] a tree tile's cache stores have read the stage (one barrier per
   // stage: the next copy from a stage needs every converter thread past this one)
   uint64_t* copy_read = drain + 1;
-  uint64_t* exit_bar = copy_read + kAttnStages;
+  uint64_t* exit_bar = reinterpret_cast<uint64_t*>(smem + L::kExitOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   int* stage_info = reinterpret_cast<int*>(smem + L::kInfoOff);
@@ -1083,6 +1084,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   mbar_arrive(exit_bar);
   if (warp == 1) {
+    // lanes 1..31 wait here, parked, until the MMA thread (lane 0) is done:
+    // spinning on the barrier beside it would take its issue slots
+    __syncwarp();
     int no_abort = 0;
     mbar_wait_bounded(exit_bar, 0, &no_abort, p.status);
     __syncwarp();

@@ -439,6 +439,9 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   tc_fence_before();
   mbar_arrive(exit_bar);
   if (warp == 1) {
+    // lanes 1..31 wait here, parked, until the MMA thread (lane 0) is done:
+    // spinning on the barrier beside it would take its issue slots
+    __syncwarp();
     int no_abort = 0;
     mbar_wait_bounded(exit_bar, 0, &no_abort, p.status);
     __syncwarp();
