@@ -176,3 +176,48 @@ def test_deepest_tree_full_acceptance(mode):
     _assert_same(got, ref)
     assert ref["accept_len"][0] == M.MAX_HEADS - 1
     np.testing.assert_array_equal(ref["accepted_nodes"][0], chain)
+
+
+def _status_of(logits, cand, spec, mode, T=0.7, eps=0.09, delta=0.3):
+    dev = "cuda"
+    tree = M.Tree.from_spec(spec)
+    B, N = cand.shape
+    W1 = spec.max_depth + 1
+    outs = [torch.full(s, -9, dtype=torch.int32, device=dev) for s in ((B,), (B, W1), (B, W1), (B,))]
+    status = M.new_status()
+    M.medusa_verify_accept(logits.to(dev), torch.from_numpy(cand).to(dev), tree, *outs, mode, T,
+                           eps, delta, dev_status=status)
+    torch.cuda.synchronize()
+    return int(status.item())
+
+
+@pytest.mark.parametrize("dtype,mode", [(torch.bfloat16, M.MEDUSA_ACCEPT_GREEDY),
+                                        (torch.bfloat16, M.MEDUSA_ACCEPT_TYPICAL),
+                                        (torch.float32, M.MEDUSA_ACCEPT_GREEDY),
+                                        (torch.float32, M.MEDUSA_ACCEPT_TYPICAL)])
+def test_nan_logit_is_reported(dtype, mode):
+    """A NaN anywhere in the logits (here in the middle of a chunk of one row,
+    and in a row's ragged last chunk) is a device-check error, not a result."""
+    w = W.scaled(W.WORKLOADS["vicuna7b"], B=2, V=5000)
+    spec = W.tree_for(w)
+    cand = _cands(w, spec, 31)
+    logits = W.verify_logits(w, spec, torch.from_numpy(cand), seed=31).to(dtype)
+    assert _status_of(logits, cand, spec, mode) == 0
+    for at in ((1, 3, 777), (0, spec.n_nodes - 1, w.V - 2)):
+        bad = logits.clone()
+        bad[at] = float("nan")
+        assert _status_of(bad, cand, spec, mode) == 6, at
+
+
+@pytest.mark.parametrize("mode", [M.MEDUSA_ACCEPT_GREEDY, M.MEDUSA_ACCEPT_TYPICAL])
+def test_candidate_outside_the_vocabulary_is_reported(mode):
+    """A candidate id outside [0, V) is reported (status 6); its logit is
+    never read."""
+    w = W.scaled(W.WORKLOADS["vicuna7b"], B=2, V=5000)
+    spec = W.tree_for(w)
+    cand = _cands(w, spec, 32)
+    logits = W.verify_logits(w, spec, torch.from_numpy(cand), seed=32)
+    for bad_id in (w.V, -1):
+        c = cand.copy()
+        c[1, 5] = bad_id
+        assert _status_of(logits, c, spec, mode) == 6, bad_id
