@@ -515,7 +515,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         const __grid_constant__ CUtensorMap tmKs1,
                         const __grid_constant__ CUtensorMap tmVs1,
                         const __grid_constant__ CUtensorMap tmQ, AttnParams p) {
-  grid_dep_wait();
+  // The launch before this one is always attn_zero_kernel, which waited for
+  // every earlier grid: the inputs (q, k_new, v_new, the caches, prefix_len,
+  // the mask) are final already.  Only the counters and flags that kernel
+  // zeroes need its completion, so the wait for it (griddepcontrol.wait) is
+  // taken by the threads that touch them, right before they do; the
+  // schedule, the first loads and the first MMAs overlap the zeroing.
   grid_dep_launch();
   using L = AttnSmem<DH>;
   extern __shared__ uint8_t smem_raw[];
@@ -824,6 +829,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t wmax = __reduce_max_sync(0xffffffffu, vm);
       if (lane == 0 && wmax < 0x7F80u && (wmax >= 0x4780u || (wmax != 0u && wmax < 0x3C80u))) {
         const int seg = stage_aux[4 * st + 2];
+        grid_dep_wait();  // the flags are zeroed by the previous launch
         if (atomicCAS(&p.seg_flag[seg], 0, 1) == 0) p.flag_list[atomicAdd(p.n_flag, 1)] = seg;
       }
       fence_proxy_async_smem();
@@ -1018,6 +1024,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       mbar_arrive(&p_full[m]);
       if (x.last) {
+        // the piece's results go to memory the previous launch zeroes (row
+        // counters) or that follows it in the stream order
+        grid_dep_wait();
         // the piece ends: wait for its last PV
         if (!mbar_wait_bounded(&p_empty[m], tcount & 1, abort_flag, p.status)) {
           ok = false;
