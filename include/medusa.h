@@ -1,7 +1,7 @@
 /*
  * medusa.h - C ABI of the Medusa decode-verify step on NVIDIA B200 (sm_100a).
  *
- * One decode-verify step of Medusa speculative decoding, in five calls:
+ * One decode-verify step of Medusa speculative decoding, in five stage calls:
  *
  *   medusa_heads_topk      K Medusa heads on the last hidden state, then a
  *                          top-k over the vocabulary per head;

@@ -1,4 +1,5 @@
-"""GPU parity of the whole decode-verify step (five C calls in a row) against
+"""GPU parity of the whole decode-verify step (DecodeVerifyStep: heads with
+the tree build, tree attention, verification with the KV compaction) against
 the oracle's step, on the same seeded inputs."""
 import math
 
