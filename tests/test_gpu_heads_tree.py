@@ -113,3 +113,20 @@ def test_malformed_tree_reported():
     assert (got["cand"] == -1).all()
     ids, _ = _heads_alone(inp, w.kmax)
     np.testing.assert_array_equal(got["ids"], ids)
+
+
+def test_full_size_llama3_8b():
+    """The configuration the benchmark times: d 4096, V 128256, 8 sequences,
+    4 heads, the 64-node tree (the heads alone are checked against the oracle
+    at this size in test_gpu_heads.py)."""
+    w = W.WORKLOADS["llama3_8b"]
+    spec = W.tree_for(w)
+    inp = W.heads_inputs(w, seed=0, device="cuda")
+    root = W.random_root_tokens(w, seed=0)
+    prefix = W.prefix_lengths(w, seed=0)
+    got, st = _fused(inp, w.kmax, spec, root, prefix)
+    assert st == 0
+    ids, vals = _heads_alone(inp, w.kmax)
+    np.testing.assert_array_equal(got["ids"], ids)
+    np.testing.assert_array_equal(got["vals"], vals)
+    _check(got, spec, root, prefix)
